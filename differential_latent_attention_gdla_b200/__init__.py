@@ -1,0 +1,230 @@
+"""B200-native GDLA forward: Python binding of libgdla.so.
+
+Grouped Differential Latent Attention ("Motif 3: Technical Report",
+Architecture). The functions below only check tensors and marshal pointers and
+sizes into the C ABI of ``include/gdla.h``; every step of the layer runs in the
+library's CUDA kernels. PyTorch supplies device memory and streams.
+
+    prefill(...)        whole forward for B sequences of L tokens
+    decode(...)         one new token per sequence over the latent cache
+    latent_expand(...)  latent RMSNorm + W_UKV expansion + rotary-key RoPE
+    rope_tables(...)    the cos/sin tables the kernels read (set-up, like weights)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _abi
+from ._abi import GDLA_BF16, GDLA_FP32, GDLA_MASK_CAUSAL, GDLA_MASK_SLIDING, GdlaError  # noqa: F401
+
+__all__ = ["prefill", "attend", "decode", "latent_expand", "rope_tables", "prefill_workspace_size", "decode_workspace_size",
+           "workspace_status", "build_info", "GdlaError"]
+
+_DT = {torch.bfloat16: GDLA_BF16, torch.float32: GDLA_FP32}
+
+
+def _lib():
+    return _abi.load()
+
+
+def build_info() -> str:
+    return _lib().gdla_build_info().decode()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("GDLA tensors must be CUDA device tensors")
+    if not t.is_contiguous():
+        raise ValueError("GDLA tensors must be contiguous (row-major)")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype(t) -> int:
+    if t.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {t.dtype}; GDLA takes bfloat16 or float32")
+    return _DT[t.dtype]
+
+
+def _mask(mask: str) -> int:
+    if mask not in ("causal", "sliding"):
+        raise ValueError("mask must be 'causal' or 'sliding'")
+    return GDLA_MASK_CAUSAL if mask == "causal" else GDLA_MASK_SLIDING
+
+
+def rope_tables(max_pos: int, d_rope: int, base: float = 10000.0, device="cuda"):
+    """cos/sin tables [max_pos, d_rope/2] (fp32) of the rotate-half RoPE with
+    frequencies theta_k = base^(-2k/d_rope). Model set-up, computed once in
+    double precision like any other constant input (e.g. a YaRN variant only
+    changes these tables)."""
+    k = torch.arange(d_rope // 2, dtype=torch.float64)
+    theta = base ** (-2.0 * k / d_rope)
+    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * theta[None, :]
+    return ang.cos().float().to(device), ang.sin().float().to(device)
+
+
+# ------------------------------------------------------------------- expansion
+def latent_expand(c_kv, gamma, k_rope, w_ukv, rope_cos, rope_sin, *, n_kv: int, d_nope: int, d_v: int,
+                  rms_eps: float = 0.0, kv_out=None, k_rope_out=None, c_hat_out=None, stream=None):
+    """Latent RMSNorm, W_UKV expansion and rotary-key RoPE. Returns
+    (kv [B,L,n_kv,d_nope+d_v], k_rope_rot [B,L,d_rope], c_hat [B,L,d_c])."""
+    B, L, d_c = c_kv.shape
+    d_rope = k_rope.shape[-1]
+    if kv_out is None:
+        kv_out = torch.empty((B, L, n_kv, d_nope + d_v), dtype=c_kv.dtype, device=c_kv.device)
+    if k_rope_out is None:
+        k_rope_out = torch.empty((B, L, d_rope), dtype=c_kv.dtype, device=c_kv.device)
+    if c_hat_out is None:
+        c_hat_out = torch.empty((B, L, d_c), dtype=c_kv.dtype, device=c_kv.device)
+    a = _abi.ExpandArgs(B, L, d_c, d_rope, n_kv, d_nope, d_v, _dtype(c_kv), rms_eps, rope_cos.shape[0],
+                        _ptr(c_kv), _ptr(gamma), _ptr(k_rope), _ptr(w_ukv), _ptr(rope_cos), _ptr(rope_sin),
+                        _ptr(kv_out), _ptr(k_rope_out), _ptr(c_hat_out))
+    _abi.check(_lib().gdla_latent_expand(ctypes.byref(a), _stream(stream)), "gdla_latent_expand")
+    return kv_out, k_rope_out, c_hat_out
+
+
+# --------------------------------------------------------------------- prefill
+def _prefill_args(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, out, g, mask, window,
+                  softmax_scale, rms_eps, cache_c_hat, cache_k_rope, workspace):
+    B, L, d_c = c_kv.shape
+    d_rope = k_rope.shape[-1]
+    H_q, d_qk = q.shape[2], q.shape[3]
+    if H_q % (g + 1):
+        raise ValueError("q must hold g*n_noise signal heads followed by n_noise noise heads")
+    n_noise = H_q // (g + 1)
+    d_nope = d_qk - d_rope
+    d_v = w_ukv.shape[1] // n_noise - d_nope
+    ws_ptr = _ptr(workspace) if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _abi.PrefillArgs(B, L, d_c, d_rope, n_noise, d_nope, d_v, n_noise, g, _mask(mask), int(window),
+                            float(softmax_scale), float(rms_eps), _dtype(c_kv), rope_cos.shape[0],
+                            _ptr(c_kv), _ptr(gamma), _ptr(k_rope), _ptr(q), _ptr(w_ukv), _ptr(rope_cos),
+                            _ptr(rope_sin), _ptr(lam_logits), _ptr(gate_logits), _ptr(out), _ptr(cache_c_hat),
+                            _ptr(cache_k_rope), ws_ptr, ws_bytes)
+
+
+def prefill_workspace_size(*, B, L, d_c, d_rope, n_kv, d_nope, d_v, g, dtype=torch.bfloat16) -> int:
+    a = _abi.PrefillArgs()
+    a.B, a.L, a.d_c, a.d_rope, a.n_kv, a.d_nope, a.d_v, a.n_noise, a.g = B, L, d_c, d_rope, n_kv, d_nope, d_v, n_kv, g
+    a.dtype = _DT[dtype]
+    return int(_lib().gdla_prefill_workspace_size(ctypes.byref(a)))
+
+
+def prefill(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, *, g: int,
+            mask: str = "causal", window: int = 0, softmax_scale: float = 0.0, rms_eps: float = 0.0, out=None,
+            workspace=None, cache_c_hat=None, cache_k_rope=None, stream=None):
+    """GDLA forward for B sequences of L tokens; returns Y [B, L, n_signal, d_v].
+
+    Shapes: c_kv [B,L,d_c], gamma [d_c], k_rope [B,L,d_rope] (pre-RoPE),
+    q [B,L,n_signal+n_noise,d_nope+d_rope] (signal heads first; rotary part
+    pre-RoPE), w_ukv [d_c, n_kv*(d_nope+d_v)], lam_logits [B,L,n_signal] fp32,
+    gate_logits [B,L,n_signal,d_v]. ``workspace`` is a uint8 CUDA tensor of at
+    least prefill_workspace_size() bytes (allocated here when omitted)."""
+    B, L = c_kv.shape[:2]
+    n_signal = lam_logits.shape[-1]
+    d_v_guess = gate_logits.shape[-1]
+    if out is None:
+        out = torch.empty((B, L, n_signal, d_v_guess), dtype=c_kv.dtype, device=c_kv.device)
+    a = _prefill_args(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, out, g, mask,
+                      window, softmax_scale, rms_eps, cache_c_hat, cache_k_rope, workspace)
+    if workspace is None:
+        need = int(_lib().gdla_prefill_workspace_size(ctypes.byref(a)))
+        workspace = torch.empty(need, dtype=torch.uint8, device=c_kv.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), need
+    _abi.check(_lib().gdla_prefill(ctypes.byref(a), _stream(stream)), "gdla_prefill")
+    return out
+
+
+def attend(q, kv, k_rope_rot, rope_cos, rope_sin, lam_logits, gate_logits, *, g: int, mask: str = "causal",
+           window: int = 0, softmax_scale: float = 0.0, out=None, status=None, stream=None):
+    """Steps 3-8 over an expanded latent (the output of latent_expand); returns
+    Y [B, L, n_signal, d_v]. ``status`` is an optional 256-byte uint8 CUDA
+    tensor that receives the device status word."""
+    B, L, H_q, d_qk = q.shape
+    n_kv, dkv = kv.shape[2], kv.shape[3]
+    d_rope = k_rope_rot.shape[-1]
+    d_nope = d_qk - d_rope
+    d_v = dkv - d_nope
+    if out is None:
+        out = torch.empty((B, L, lam_logits.shape[-1], d_v), dtype=q.dtype, device=q.device)
+    if status is None:
+        status = torch.empty(256, dtype=torch.uint8, device=q.device)
+    a = _abi.AttendArgs(B, L, d_rope, n_kv, d_nope, d_v, H_q // (g + 1), g, _mask(mask), int(window),
+                        float(softmax_scale), _dtype(q), rope_cos.shape[0], _ptr(q), _ptr(kv), _ptr(k_rope_rot),
+                        _ptr(rope_cos), _ptr(rope_sin), _ptr(lam_logits), _ptr(gate_logits), _ptr(out), _ptr(status),
+                        status.numel())
+    _abi.check(_lib().gdla_attend(ctypes.byref(a), _stream(stream)), "gdla_attend")
+    return out
+
+
+# ---------------------------------------------------------------------- decode
+def _decode_args(c_cache, kr_cache, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, seqlens, out, g, mask,
+                 window, softmax_scale, workspace):
+    B, T_max, d_c = c_cache.shape
+    d_rope = kr_cache.shape[-1]
+    H_q, d_qk = q.shape[1], q.shape[2]
+    if H_q % (g + 1):
+        raise ValueError("q must hold g*n_noise signal heads followed by n_noise noise heads")
+    n_noise = H_q // (g + 1)
+    d_nope = d_qk - d_rope
+    d_v = w_ukv.shape[1] // n_noise - d_nope
+    if seqlens.dtype != torch.int32:
+        raise ValueError("seqlens must be int32")
+    ws_ptr = _ptr(workspace) if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return _abi.DecodeArgs(B, T_max, d_c, d_rope, n_noise, d_nope, d_v, n_noise, g, _mask(mask), int(window),
+                           float(softmax_scale), _dtype(c_cache), rope_cos.shape[0], _ptr(seqlens), _ptr(c_cache),
+                           _ptr(kr_cache), _ptr(q), _ptr(w_ukv), _ptr(rope_cos), _ptr(rope_sin), _ptr(lam_logits),
+                           _ptr(gate_logits), _ptr(out), ws_ptr, ws_bytes)
+
+
+def decode_workspace_size(*, B, T_max, d_c, d_rope, n_kv, d_nope, d_v, g, dtype=torch.bfloat16) -> int:
+    a = _abi.DecodeArgs()
+    a.B, a.T_max, a.d_c, a.d_rope, a.n_kv, a.d_nope, a.d_v, a.n_noise, a.g = B, T_max, d_c, d_rope, n_kv, d_nope, d_v, n_kv, g
+    a.dtype = _DT[dtype]
+    return int(_lib().gdla_decode_workspace_size(ctypes.byref(a)))
+
+
+def decode(c_cache, kr_cache, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, seqlens, *, g: int,
+           mask: str = "causal", window: int = 0, softmax_scale: float = 0.0, out=None, workspace=None, stream=None):
+    """One decode step per sequence; returns Y [B, n_signal, d_v].
+
+    c_cache [B,T_max,d_c] normalised latent, kr_cache [B,T_max,d_rope] rotated
+    rotary key, q [B,n_signal+n_noise,d_nope+d_rope] (rotary part pre-RoPE, at
+    position seqlens[b]-1), lam_logits [B,n_signal] fp32, gate_logits
+    [B,n_signal,d_v], seqlens [B] int32 on the device."""
+    B = c_cache.shape[0]
+    if out is None:
+        out = torch.empty((B, lam_logits.shape[-1], gate_logits.shape[-1]), dtype=c_cache.dtype,
+                          device=c_cache.device)
+    a = _decode_args(c_cache, kr_cache, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, seqlens, out, g,
+                     mask, window, softmax_scale, workspace)
+    if workspace is None:
+        need = int(_lib().gdla_decode_workspace_size(ctypes.byref(a)))
+        workspace = torch.empty(need, dtype=torch.uint8, device=c_cache.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), need
+    _abi.check(_lib().gdla_decode(ctypes.byref(a), _stream(stream)), "gdla_decode")
+    return out
+
+
+def workspace_status(workspace, stream=None) -> int:
+    """Device status word of the last call that used ``workspace`` (0 = OK)."""
+    return int(_lib().gdla_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def _mask_const(mask: str) -> int:
+    return _mask(mask)
+
+
+def default_scale(d_nope: int, d_rope: int) -> float:
+    return 1.0 / math.sqrt(d_nope + d_rope)

@@ -1,0 +1,301 @@
+// decode.cu -- GDLA decode over the compact latent cache ("Motif 3: Technical
+// Report", Architecture: GDLA keeps MLA's compact inference state).
+//
+// The cache stores per token the normalised latent c_hat (d_c) and the rotated
+// rotary key (d_rope). Attention against expanded keys k_nope = c_hat W_UK and
+// values v = c_hat W_UV is evaluated without expanding them:
+//   q_nope . (c_hat W_UK) = (W_UK q_nope) . c_hat      (absorbed query)
+//   sum_j p_j (c_hat_j W_UV) = (sum_j p_j c_hat_j) W_UV (latent weighted sum)
+// Kernels: decode_absorb (q_abs = W_UK q_nope, RoPE of q_rope at position
+// seqlen-1), decode_split (split-KV online softmax over the cache, partial
+// results per split), decode_combine (log-sum-exp merge, W_UV, differential
+// and gate epilogue).
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdla {
+
+// One block per (KV group, sequence); one warp per latent row c at a time.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv;
+  const int dqk = p.d_nope + p.d_rope, ncol = p.n_kv * (p.d_nope + p.d_v);
+  const T* q = reinterpret_cast<const T*>(p.q);
+  const T* w = reinterpret_cast<const T*>(p.w_ukv);
+  extern __shared__ float qn[];  // [(g+1)][d_nope]
+  const int G1 = p.g + 1;
+  for (int e = threadIdx.x; e < G1 * p.d_nope; e += blockDim.x) {
+    const int which = e / p.d_nope, k = e % p.d_nope;
+    const int head = which < p.g ? h * p.g + which : n_S + h;
+    qn[e] = to_f(q[((long)b * H_q + head) * dqk + k]);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int c = warp; c < p.d_c; c += blockDim.x >> 5) {
+    const T* wr = w + (long)c * ncol + (long)h * (p.d_nope + p.d_v);
+    float acc[9];
+    for (int u = 0; u < G1; ++u) acc[u] = 0.f;
+    for (int k = lane; k < p.d_nope; k += 32) {
+      const float wv = to_f(wr[k]);
+      for (int u = 0; u < G1; ++u) acc[u] = fmaf(wv, qn[u * p.d_nope + k], acc[u]);
+    }
+    for (int u = 0; u < G1; ++u) {
+      float a = acc[u];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0) {
+        const int head = u < p.g ? h * p.g + u : n_S + h;
+        p.q_abs[((long)b * H_q + head) * p.d_c + c] = a;
+      }
+    }
+  }
+  // RoPE of the rotary query parts at position seqlen-1
+  const int pos = p.seqlens[b] - 1;
+  const int half = p.d_rope >> 1;
+  for (int e = threadIdx.x; e < G1 * half; e += blockDim.x) {
+    const int which = e / half, k = e % half;
+    const int head = which < p.g ? h * p.g + which : n_S + h;
+    const T* qr = q + ((long)b * H_q + head) * dqk + p.d_nope;
+    const float cs = p.cos_tab[(long)pos * half + k], sn = p.sin_tab[(long)pos * half + k];
+    const float x1 = to_f(qr[k]), x2 = to_f(qr[k + half]);
+    float* o = p.q_rot + ((long)b * H_q + head) * p.d_rope;
+    o[k] = x1 * cs - x2 * sn;
+    o[k + half] = x2 * cs + x1 * sn;
+  }
+}
+
+// Split-KV pass (CUDA cores): block (split s, sequence b) covers cache tokens
+// [s*split_len, (s+1)*split_len) of the visible range, for every query head.
+// HPT = heads per thread (H_q <= 8*HPT), CPT = latent columns per thread (d_c = 32*CPT).
+template <typename T, int HPT, int CPT>
+__global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) {
+  constexpr int BT = 32;  // tokens per tile
+  const int s = blockIdx.x, b = blockIdx.y;
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv;
+  const int d_c = p.d_c, d_r = p.d_rope, RW = d_c + d_r + 1;  // padded cache row
+  extern __shared__ float sm[];
+  float* qa = sm;                        // [H_q][d_c]
+  float* qr = qa + H_q * d_c;            // [H_q][d_r]
+  float* ct = qr + H_q * d_r;            // [BT][RW]
+  float* ps = ct + BT * RW;              // [H_q][BT]
+  float* mrow = ps + H_q * BT;           // [H_q]
+  float* lrow = mrow + H_q;              // [H_q]
+  float* arow = lrow + H_q;              // [H_q]
+  const T* cc = reinterpret_cast<const T*>(p.c_cache);
+  const T* kc = reinterpret_cast<const T*>(p.kr_cache);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float sl2 = p.scale * kLog2e;
+
+  for (int e = tid; e < H_q * d_c; e += 256) qa[e] = p.q_abs[(long)b * H_q * d_c + e];
+  for (int e = tid; e < H_q * d_r; e += 256) qr[e] = p.q_rot[(long)b * H_q * d_r + e];
+  for (int e = tid; e < H_q; e += 256) {
+    mrow[e] = -INFINITY;
+    lrow[e] = 0.f;
+  }
+  const int Tb = p.seqlens[b];
+  const int lo = p.sliding ? max(0, Tb - p.window) : 0;
+  const int t0 = max(lo, s * p.split_len), t1 = min(Tb, (s + 1) * p.split_len);
+
+  float acc[HPT][CPT];
+#pragma unroll
+  for (int a = 0; a < HPT; ++a)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[a][c] = 0.f;
+
+  for (int j0 = t0; j0 < t1; j0 += BT) {
+    __syncthreads();
+    for (int e = tid; e < BT * (d_c + d_r); e += 256) {
+      const int r = e / (d_c + d_r), k = e % (d_c + d_r);
+      const int j = j0 + r;
+      float val = 0.f;
+      if (j < t1)
+        val = k < d_c ? to_f(cc[((long)b * p.T_max + j) * d_c + k])
+                      : to_f(kc[((long)b * p.T_max + j) * d_r + (k - d_c)]);
+      ct[r * RW + k] = val;
+    }
+    __syncthreads();
+    // scores: lane = token, warp handles heads warp, warp+8, ...
+    for (int hh = warp; hh < H_q; hh += 8) {
+      const float* qh = qa + hh * d_c;
+      const float* crow = ct + lane * RW;
+      float dot = 0.f;
+      for (int k = 0; k < d_c; ++k) dot = fmaf(qh[k], crow[k], dot);
+      const float* qrh = qr + hh * d_r;
+      for (int k = 0; k < d_r; ++k) dot = fmaf(qrh[k], crow[d_c + k], dot);
+      float sv = (j0 + lane < t1) ? dot * sl2 : -INFINITY;
+      float mx = sv;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_old = mrow[hh];
+      const float m_new = fmaxf(m_old, mx);
+      const float pe = (sv == -INFINITY) ? 0.f : exp2f(sv - m_new);
+      float sum = pe;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      ps[hh * BT + lane] = pe;
+      __syncwarp();
+      if (lane == 0) {
+        const float al = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
+        arow[hh] = al;
+        lrow[hh] = lrow[hh] * al + sum;
+        mrow[hh] = m_new;
+      }
+    }
+    __syncthreads();
+    // O[h][c] = alpha * O + sum_j P[h][j] c_hat[j][c]; thread: heads warp+8a, cols lane+32c
+#pragma unroll
+    for (int a = 0; a < HPT; ++a) {
+      const int hh = warp + 8 * a;
+      if (hh >= H_q) break;
+      const float al = arow[hh];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) acc[a][c] *= al;
+      for (int j = 0; j < BT; ++j) {
+        const float pj = ps[hh * BT + j];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[a][c] = fmaf(pj, ct[j * RW + lane + 32 * c], acc[a][c]);
+      }
+    }
+  }
+  __syncthreads();
+  // partial results of this split
+  const long base = ((long)b * p.n_splits + s) * H_q;
+#pragma unroll
+  for (int a = 0; a < HPT; ++a) {
+    const int hh = warp + 8 * a;
+    if (hh >= H_q) break;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) p.part_o[(base + hh) * d_c + lane + 32 * c] = acc[a][c];
+  }
+  for (int e = tid; e < H_q; e += 256) {
+    p.part_ml[(base + e) * 2 + 0] = mrow[e];
+    p.part_ml[(base + e) * 2 + 1] = lrow[e];
+  }
+}
+
+// Merge the splits of every head of one KV group, apply W_UV, then
+// D = H_S - sigmoid(lam) H_N and Y = sigmoid(G) D.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1;
+  const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v);
+  extern __shared__ float sm[];
+  float* olat = sm;               // [G1][d_c]
+  float* hv = olat + G1 * d_c;    // [G1][DV]
+  float* wgt = hv + G1 * DV;      // [G1][n_splits]
+  const T* w = reinterpret_cast<const T*>(p.w_ukv);
+  const T* gate = reinterpret_cast<const T*>(p.gate);
+  T* out = reinterpret_cast<T*>(p.out);
+  const int tid = threadIdx.x;
+  if (tid < G1) {
+    const int head = tid < p.g ? h * p.g + tid : n_S + h;
+    float M = -INFINITY;
+    for (int s = 0; s < p.n_splits; ++s)
+      M = fmaxf(M, p.part_ml[(((long)b * p.n_splits + s) * H_q + head) * 2]);
+    float den = 0.f;
+    for (int s = 0; s < p.n_splits; ++s) {
+      const float* ml = p.part_ml + (((long)b * p.n_splits + s) * H_q + head) * 2;
+      const float wv = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
+      wgt[tid * p.n_splits + s] = wv;
+      den += wv * ml[1];
+    }
+    for (int s = 0; s < p.n_splits; ++s) wgt[tid * p.n_splits + s] /= den;
+  }
+  __syncthreads();
+  for (int e = tid; e < G1 * d_c; e += 256) {
+    const int u = e / d_c, c = e % d_c;
+    const int head = u < p.g ? h * p.g + u : n_S + h;
+    float a = 0.f;
+    for (int s = 0; s < p.n_splits; ++s)
+      a = fmaf(wgt[u * p.n_splits + s], p.part_o[(((long)b * p.n_splits + s) * H_q + head) * d_c + c], a);
+    olat[e] = a;
+  }
+  __syncthreads();
+  for (int e = tid; e < G1 * DV; e += 256) {
+    const int u = e / DV, n = e % DV;
+    const T* wc = w + (long)h * (p.d_nope + DV) + p.d_nope + n;
+    float a = 0.f;
+    for (int c = 0; c < d_c; ++c) a = fmaf(olat[u * d_c + c], to_f(wc[(long)c * ncol]), a);
+    hv[e] = a;
+  }
+  __syncthreads();
+  for (int e = tid; e < p.g * DV; e += 256) {
+    const int u = e / DV, n = e % DV;
+    const int sh = h * p.g + u;
+    const float lam = sigmoidf_(p.lam[(long)b * n_S + sh]);
+    const long idx = ((long)b * n_S + sh) * DV + n;
+    const float d = hv[u * DV + n] - lam * hv[p.g * DV + n];
+    out[idx] = from_f<T>(sigmoidf_(to_f(gate[idx])) * d);
+  }
+}
+
+cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
+  dim3 grid((unsigned)p.n_kv, (unsigned)p.B);
+  const size_t smem = sizeof(float) * (size_t)(p.g + 1) * p.d_nope;
+  if (dt == GDLA_BF16)
+    decode_absorb_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(p);
+  else
+    decode_absorb_kernel<float><<<grid, 256, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int HPT, int CPT>
+static cudaError_t split_one(const DecodeParams& p, cudaStream_t s) {
+  const int H_q = p.n_kv * (p.g + 1);
+  const size_t smem = sizeof(float) * ((size_t)H_q * p.d_c + (size_t)H_q * p.d_rope +
+                                       32 * (size_t)(p.d_c + p.d_rope + 1) + (size_t)H_q * 32 + 3 * H_q);
+  auto k = decode_split_simt_kernel<T, HPT, CPT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<dim3((unsigned)p.n_splits, (unsigned)p.B), 256, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int HPT>
+static cudaError_t split_h(const DecodeParams& p, cudaStream_t s) {
+  switch (p.d_c) {
+    case 64: return split_one<T, HPT, 2>(p, s);
+    case 128: return split_one<T, HPT, 4>(p, s);
+    case 256: return split_one<T, HPT, 8>(p, s);
+    case 512: return split_one<T, HPT, 16>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename T>
+static cudaError_t split_t(const DecodeParams& p, cudaStream_t s) {
+  const int H_q = p.n_kv * (p.g + 1);
+  if (H_q <= 16) return split_h<T, 2>(p, s);
+  if (H_q <= 32) return split_h<T, 4>(p, s);
+  if (H_q <= 48) return split_h<T, 6>(p, s);
+  if (H_q <= 64) return split_h<T, 8>(p, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
+  return dt == GDLA_BF16 ? split_t<__nv_bfloat16>(p, s) : split_t<float>(p, s);
+}
+
+cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
+  const int G1 = p.g + 1;
+  const size_t smem = sizeof(float) * ((size_t)G1 * p.d_c + (size_t)G1 * p.d_v + (size_t)G1 * p.n_splits);
+  dim3 grid((unsigned)p.n_kv, (unsigned)p.B);
+  if (dt == GDLA_BF16) {
+    auto k = decode_combine_kernel<__nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, 256, smem, s>>>(p);
+  } else {
+    auto k = decode_combine_kernel<float>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, 256, smem, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace gdla

@@ -1,0 +1,285 @@
+// gdla_api.cu -- the C ABI declared in include/gdla.h: argument validation,
+// workspace layout and kernel dispatch. Nothing here computes; every step of
+// the layer runs in the kernels of this directory.
+#include <cuda_runtime.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/gdla.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace gdla;
+
+namespace {
+
+constexpr int kNumSMs = 148;  // B200
+
+size_t esize(gdla_dtype d) { return d == GDLA_FP32 ? 4 : 2; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+bool aligned16(const void* p) { return p && ((uintptr_t)p & 15) == 0; }
+bool opt_aligned16(const void* p) { return !p || ((uintptr_t)p & 15) == 0; }
+
+bool head_dims_ok(int d_nope, int d_rope, int d_v) {
+  return (d_nope == 128 && d_rope == 64 && d_v == 128) || (d_nope == 64 && d_rope == 32 && d_v == 64) ||
+         (d_nope == 32 && d_rope == 16 && d_v == 32);
+}
+bool latent_ok(int d_c) { return d_c == 64 || d_c == 128 || d_c == 256 || d_c == 512; }
+
+gdla_status common_dims(int B, int L, int d_c, int d_rope, int n_kv, int d_nope, int d_v, int n_noise, int g,
+                        int dtype) {
+  if (B < 1 || B > 65535 || L < 1 || n_kv < 1 || n_kv > 65535 || g < 1) return GDLA_ERR_INVALID_ARG;
+  if (dtype != GDLA_BF16 && dtype != GDLA_FP32) return GDLA_ERR_INVALID_ARG;
+  if (n_noise != n_kv) return GDLA_ERR_UNSUPPORTED;
+  if (g > 8 || !head_dims_ok(d_nope, d_rope, d_v) || !latent_ok(d_c)) return GDLA_ERR_UNSUPPORTED;
+  if ((long)n_kv * (g + 1) > 64) return GDLA_ERR_UNSUPPORTED;
+  return GDLA_OK;
+}
+
+struct PrefillLayout {
+  size_t status, c_hat, k_rot, kv, total;
+};
+
+PrefillLayout prefill_layout(const gdla_prefill_args* a) {
+  PrefillLayout l;
+  const size_t tok = (size_t)a->B * (size_t)a->L, es = esize(a->dtype);
+  size_t off = 0;
+  l.status = off;
+  off += kStatusBytes;
+  l.c_hat = off;
+  off = align256(off + tok * a->d_c * es);
+  l.k_rot = off;
+  off = align256(off + tok * a->d_rope * es);
+  l.kv = off;
+  off = align256(off + tok * (size_t)a->n_kv * (a->d_nope + a->d_v) * es);
+  l.total = off;
+  return l;
+}
+
+struct DecodeLayout {
+  size_t status, q_abs, q_rot, part_o, part_ml, total;
+  int n_splits, split_len;
+};
+
+DecodeLayout decode_layout(const gdla_decode_args* a) {
+  DecodeLayout l;
+  const int H_q = a->n_kv * (a->g + 1);
+  const int tile = 128;
+  const int max_splits = (a->T_max + tile - 1) / tile;
+  int n = (2 * kNumSMs + a->B - 1) / a->B;
+  if (n > max_splits) n = max_splits;
+  if (n < 1) n = 1;
+  int len = (a->T_max + n - 1) / n;
+  len = (len + tile - 1) / tile * tile;
+  l.split_len = len;
+  l.n_splits = (a->T_max + len - 1) / len;
+  size_t off = 0;
+  l.status = off;
+  off += kStatusBytes;
+  l.q_abs = off;
+  off = align256(off + sizeof(float) * (size_t)a->B * H_q * a->d_c);
+  l.q_rot = off;
+  off = align256(off + sizeof(float) * (size_t)a->B * H_q * a->d_rope);
+  l.part_o = off;
+  off = align256(off + sizeof(float) * (size_t)a->B * l.n_splits * H_q * a->d_c);
+  l.part_ml = off;
+  off = align256(off + sizeof(float) * (size_t)a->B * l.n_splits * H_q * 2);
+  l.total = off;
+  return l;
+}
+
+gdla_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return GDLA_OK;
+  cudaGetLastError();  // clear a sticky launch error of ours
+  return GDLA_ERR_CUDA;
+}
+
+gdla_status validate_prefill(const gdla_prefill_args* a) {
+  if (!a) return GDLA_ERR_INVALID_ARG;
+  gdla_status st = common_dims(a->B, a->L, a->d_c, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_noise, a->g,
+                               a->dtype);
+  if (st != GDLA_OK) return st;
+  if (a->mask != GDLA_MASK_CAUSAL && a->mask != GDLA_MASK_SLIDING) return GDLA_ERR_INVALID_ARG;
+  if (a->mask == GDLA_MASK_SLIDING && a->window < 1) return GDLA_ERR_INVALID_ARG;
+  if (a->rope_max_pos < a->L) return GDLA_ERR_INVALID_ARG;
+  const void* req[] = {a->c_kv, a->gamma, a->k_rope, a->q, a->w_ukv, a->rope_cos, a->rope_sin,
+                       a->lam_logits, a->gate_logits, a->out, a->workspace};
+  for (const void* p : req)
+    if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  if (!opt_aligned16(a->cache_c_hat) || !opt_aligned16(a->cache_k_rope)) return GDLA_ERR_INVALID_ARG;
+  if (((uintptr_t)a->workspace & 255) != 0) return GDLA_ERR_INVALID_ARG;
+  if (a->workspace_bytes < prefill_layout(a).total) return GDLA_ERR_INVALID_ARG;
+  return GDLA_OK;
+}
+
+gdla_status validate_decode(const gdla_decode_args* a) {
+  if (!a) return GDLA_ERR_INVALID_ARG;
+  gdla_status st = common_dims(a->B, a->T_max, a->d_c, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_noise,
+                               a->g, a->dtype);
+  if (st != GDLA_OK) return st;
+  if (a->mask != GDLA_MASK_CAUSAL && a->mask != GDLA_MASK_SLIDING) return GDLA_ERR_INVALID_ARG;
+  if (a->mask == GDLA_MASK_SLIDING && a->window < 1) return GDLA_ERR_INVALID_ARG;
+  if (a->rope_max_pos < a->T_max) return GDLA_ERR_INVALID_ARG;
+  const void* req[] = {a->seqlens, a->c_cache, a->kr_cache, a->q, a->w_ukv, a->rope_cos, a->rope_sin,
+                       a->lam_logits, a->gate_logits, a->out, a->workspace};
+  for (const void* p : req)
+    if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  if (((uintptr_t)a->workspace & 255) != 0) return GDLA_ERR_INVALID_ARG;
+  if (a->workspace_bytes < decode_layout(a).total) return GDLA_ERR_INVALID_ARG;
+  return GDLA_OK;
+}
+
+float default_scale(float s, int d_nope, int d_rope) {
+  return s > 0.f ? s : 1.0f / sqrtf((float)(d_nope + d_rope));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdla_status_string(gdla_status s) {
+  switch (s) {
+    case GDLA_OK: return "GDLA_OK";
+    case GDLA_ERR_INVALID_ARG: return "GDLA_ERR_INVALID_ARG: bad pointer, alignment, size or workspace";
+    case GDLA_ERR_UNSUPPORTED: return "GDLA_ERR_UNSUPPORTED: valid arguments outside the implemented shapes";
+    case GDLA_ERR_CUDA: return "GDLA_ERR_CUDA: a CUDA launch or query failed";
+    case GDLA_ERR_TIMEOUT: return "GDLA_ERR_TIMEOUT: a device-side wait hit its iteration cap";
+  }
+  return "unknown gdla_status";
+}
+
+const char* gdla_build_info(void) {
+  return "libgdla sm_100a (tcgen05/TMA attention + expansion, split-KV decode); built " __DATE__ " " __TIME__;
+}
+
+gdla_status gdla_latent_expand(const gdla_expand_args* a, void* stream) {
+  if (!a) return GDLA_ERR_INVALID_ARG;
+  gdla_status st = common_dims(a->B, a->L, a->d_c, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_kv, 1, a->dtype);
+  if (st != GDLA_OK) return st;
+  if (a->rope_max_pos < a->L) return GDLA_ERR_INVALID_ARG;
+  const void* req[] = {a->c_kv, a->gamma, a->k_rope, a->w_ukv, a->rope_cos, a->rope_sin,
+                       a->kv_out, a->k_rope_out, a->c_hat_out};
+  for (const void* p : req)
+    if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  NormRopeParams np{(long)a->B * a->L, a->L, a->d_c, a->d_rope, a->rope_max_pos,
+                    a->rms_eps > 0.f ? a->rms_eps : 1e-6f, a->c_kv, a->gamma, a->k_rope,
+                    a->rope_cos, a->rope_sin, a->c_hat_out, a->k_rope_out};
+  cudaError_t e = launch_norm_rope(np, a->dtype, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  GemmParams gp{(long)a->B * a->L, a->n_kv * (a->d_nope + a->d_v), a->d_c, a->c_hat_out, a->w_ukv, a->kv_out};
+  if (a->dtype == GDLA_BF16 && gemm_tc_supported(gp))
+    e = launch_gemm_tc(gp, nullptr, s);
+  else
+    e = launch_gemm_simt(gp, a->dtype, s);
+  return cuda_status(e);
+}
+
+static gdla_status attend_impl(const gdla_attend_args* a, cudaStream_t s, bool clear_status) {
+  AttnParams ap{};
+  ap.B = a->B; ap.L = a->L; ap.n_kv = a->n_kv; ap.g = a->g; ap.d_nope = a->d_nope; ap.d_rope = a->d_rope;
+  ap.d_v = a->d_v; ap.sliding = a->mask == GDLA_MASK_SLIDING; ap.window = ap.sliding ? a->window : 0;
+  ap.rope_max_pos = a->rope_max_pos; ap.scale = default_scale(a->softmax_scale, a->d_nope, a->d_rope);
+  ap.q = a->q; ap.kv = a->kv; ap.kr = a->k_rope_rot; ap.cos_tab = a->rope_cos; ap.sin_tab = a->rope_sin;
+  ap.lam = a->lam_logits; ap.gate = a->gate_logits; ap.out = a->out; ap.status = (int*)a->workspace;
+  cudaError_t e = cudaSuccess;
+  if (clear_status) e = cudaMemsetAsync(a->workspace, 0, kStatusBytes, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (attn_tc_supported(ap, a->dtype))
+    e = launch_attn_tc(ap, s);
+  else
+    e = launch_attn_simt(ap, a->dtype, s);
+  return cuda_status(e);
+}
+
+gdla_status gdla_attend(const gdla_attend_args* a, void* stream) {
+  if (!a) return GDLA_ERR_INVALID_ARG;
+  gdla_status st = common_dims(a->B, a->L, 64, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_noise, a->g, a->dtype);
+  if (st != GDLA_OK) return st;
+  if (a->mask != GDLA_MASK_CAUSAL && a->mask != GDLA_MASK_SLIDING) return GDLA_ERR_INVALID_ARG;
+  if (a->mask == GDLA_MASK_SLIDING && a->window < 1) return GDLA_ERR_INVALID_ARG;
+  if (a->rope_max_pos < a->L) return GDLA_ERR_INVALID_ARG;
+  const void* req[] = {a->q, a->kv, a->k_rope_rot, a->rope_cos, a->rope_sin, a->lam_logits, a->gate_logits,
+                       a->out, a->workspace};
+  for (const void* p : req)
+    if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  if (((uintptr_t)a->workspace & 255) != 0 || a->workspace_bytes < kStatusBytes) return GDLA_ERR_INVALID_ARG;
+  return attend_impl(a, (cudaStream_t)stream, /*clear_status=*/true);
+}
+
+size_t gdla_prefill_workspace_size(const gdla_prefill_args* a) {
+  if (!a || a->B < 1 || a->L < 1) return 0;
+  return prefill_layout(a).total;
+}
+
+gdla_status gdla_prefill(const gdla_prefill_args* a, void* stream) {
+  gdla_status st = validate_prefill(a);
+  if (st != GDLA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const PrefillLayout lay = prefill_layout(a);
+  char* ws = (char*)a->workspace;
+  int* status = (int*)(ws + lay.status);
+  void* c_hat = a->cache_c_hat ? a->cache_c_hat : (void*)(ws + lay.c_hat);
+  void* k_rot = a->cache_k_rope ? a->cache_k_rope : (void*)(ws + lay.k_rot);
+  void* kv = ws + lay.kv;
+  cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, s);
+  if (e != cudaSuccess) return cuda_status(e);
+
+  gdla_expand_args ea{};
+  ea.B = a->B; ea.L = a->L; ea.d_c = a->d_c; ea.d_rope = a->d_rope; ea.n_kv = a->n_kv;
+  ea.d_nope = a->d_nope; ea.d_v = a->d_v; ea.dtype = a->dtype; ea.rms_eps = a->rms_eps;
+  ea.rope_max_pos = a->rope_max_pos; ea.c_kv = a->c_kv; ea.gamma = a->gamma; ea.k_rope = a->k_rope;
+  ea.w_ukv = a->w_ukv; ea.rope_cos = a->rope_cos; ea.rope_sin = a->rope_sin;
+  ea.kv_out = kv; ea.k_rope_out = k_rot; ea.c_hat_out = c_hat;
+  st = gdla_latent_expand(&ea, stream);
+  if (st != GDLA_OK) return st;
+
+  gdla_attend_args aa{};
+  aa.B = a->B; aa.L = a->L; aa.d_rope = a->d_rope; aa.n_kv = a->n_kv; aa.d_nope = a->d_nope; aa.d_v = a->d_v;
+  aa.n_noise = a->n_noise; aa.g = a->g; aa.mask = a->mask; aa.window = a->window;
+  aa.softmax_scale = a->softmax_scale; aa.dtype = a->dtype; aa.rope_max_pos = a->rope_max_pos;
+  aa.q = a->q; aa.kv = kv; aa.k_rope_rot = k_rot; aa.rope_cos = a->rope_cos; aa.rope_sin = a->rope_sin;
+  aa.lam_logits = a->lam_logits; aa.gate_logits = a->gate_logits; aa.out = a->out;
+  aa.workspace = status; aa.workspace_bytes = kStatusBytes;
+  return attend_impl(&aa, s, /*clear_status=*/false);
+}
+
+size_t gdla_decode_workspace_size(const gdla_decode_args* a) {
+  if (!a || a->B < 1 || a->T_max < 1 || a->n_kv < 1 || a->g < 1) return 0;
+  return decode_layout(a).total;
+}
+
+gdla_status gdla_decode(const gdla_decode_args* a, void* stream) {
+  gdla_status st = validate_decode(a);
+  if (st != GDLA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const DecodeLayout lay = decode_layout(a);
+  char* ws = (char*)a->workspace;
+  DecodeParams p{};
+  p.B = a->B; p.T_max = a->T_max; p.d_c = a->d_c; p.d_rope = a->d_rope; p.n_kv = a->n_kv; p.g = a->g;
+  p.d_nope = a->d_nope; p.d_v = a->d_v; p.sliding = a->mask == GDLA_MASK_SLIDING;
+  p.window = p.sliding ? a->window : 0; p.rope_max_pos = a->rope_max_pos;
+  p.scale = default_scale(a->softmax_scale, a->d_nope, a->d_rope);
+  p.n_splits = lay.n_splits; p.split_len = lay.split_len; p.seqlens = a->seqlens;
+  p.c_cache = a->c_cache; p.kr_cache = a->kr_cache; p.q = a->q; p.w_ukv = a->w_ukv;
+  p.cos_tab = a->rope_cos; p.sin_tab = a->rope_sin; p.lam = a->lam_logits; p.gate = a->gate_logits;
+  p.out = a->out; p.q_abs = (float*)(ws + lay.q_abs); p.q_rot = (float*)(ws + lay.q_rot);
+  p.part_o = (float*)(ws + lay.part_o); p.part_ml = (float*)(ws + lay.part_ml);
+  p.status = (int*)(ws + lay.status);
+  cudaError_t e = cudaMemsetAsync(p.status, 0, kStatusBytes, s);
+  if (e == cudaSuccess) e = launch_decode_absorb(p, a->dtype, s);
+  if (e == cudaSuccess) e = launch_decode_split_simt(p, a->dtype, s);
+  if (e == cudaSuccess) e = launch_decode_combine(p, a->dtype, s);
+  return cuda_status(e);
+}
+
+gdla_status gdla_workspace_status(const void* workspace, void* stream) {
+  if (!workspace) return GDLA_ERR_INVALID_ARG;
+  int code = 0;
+  cudaError_t e = cudaMemcpyAsync(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  return code == 0 ? GDLA_OK : (gdla_status)code;
+}
+
+}  // extern "C"

@@ -1,0 +1,205 @@
+/*
+ * gdla.h -- C ABI of the B200 (sm_100a) GDLA forward library, libgdla.so.
+ *
+ * Grouped Differential Latent Attention as stated in "Motif 3: Technical
+ * Report" (montaan.com/papers/2608.09119), section "Architecture", the GDLA
+ * paragraphs: the compressed KV latent is RMS-normalised and expanded by one
+ * up-projection W_UKV into n_kv content-key/value heads shared by the signal
+ * and noise query paths; a decoupled rotary key is shared across heads and
+ * RoPE touches only the rotary query/key parts; g*n_N signal heads and n_N
+ * noise heads attend independently under a full causal or a sliding-window
+ * mask; D_t = H_S,t - lambda_t (.) Repeat_g(H_N,t) with lambda_t = sigmoid of
+ * a per-(token, signal head) logit; Y = sigmoid(G) (.) D is the element-wise
+ * output gate applied before the output projection. Dimensions in that report:
+ * 16 KV heads, d_qk = 192 (128 content + 64 rotary), d_v = 128, d_c = 512.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, dense
+ *    row-major in the layout stated beside them, 16-byte aligned. The library
+ *    allocates no memory and keeps no per-call state; scratch comes from the
+ *    caller's workspace, sized by the matching *_workspace_size function.
+ *  - `stream` is a cudaStream_t passed as void*. All work is enqueued on it and
+ *    the call returns without synchronising.
+ *  - Argument errors (NULL pointer, misalignment, unsupported size, a too
+ *    small workspace or RoPE table) are reported synchronously, BEFORE anything
+ *    is launched, as GDLA_ERR_INVALID_ARG or GDLA_ERR_UNSUPPORTED. A failed
+ *    launch returns GDLA_ERR_CUDA. A device-side wait that hit its iteration
+ *    cap is recorded in the workspace's status word and reported by
+ *    gdla_workspace_status (GDLA_ERR_TIMEOUT). Nothing is thrown across the ABI.
+ *  - Element type: `dtype` selects bf16 or fp32 for every floating tensor
+ *    except the lambda logits and the RoPE tables, which are always fp32.
+ *    bf16 arithmetic accumulates in fp32; the softmax runs in fp32.
+ */
+#ifndef GDLA_H_
+#define GDLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDLA_OK = 0,
+  GDLA_ERR_INVALID_ARG = 1,  /* NULL/misaligned pointer, bad size, small workspace */
+  GDLA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. n_noise != n_kv) */
+  GDLA_ERR_CUDA = 3,         /* a CUDA launch or query failed */
+  GDLA_ERR_TIMEOUT = 4       /* a device wait hit its iteration cap */
+} gdla_status;
+
+typedef enum {
+  GDLA_MASK_CAUSAL = 0,  /* key j visible to query i iff j <= i */
+  GDLA_MASK_SLIDING = 1  /* key j visible to query i iff i - window < j <= i */
+} gdla_mask;
+
+typedef enum { GDLA_BF16 = 0, GDLA_FP32 = 1 } gdla_dtype;
+
+/* Shared sizes. n_signal = g * n_noise; the report pairs every noise head with
+ * one KV head, so n_noise must equal n_kv. Signal head i reads KV head
+ * floor(i/g) and subtracts noise head floor(i/g) (Repeat_g as
+ * repeat-interleave). Supported: d_nope, d_v in {32, 64, 128}; d_rope in
+ * {16, 32, 64}; d_c in {64, 128, 256, 512}; 1 <= g <= 8. */
+
+/* ------------------------------------------------------------------ expansion
+ * Steps 1-3 of the layer for a whole batch: latent RMSNorm, the single W_UKV
+ * up-projection, and RoPE of the shared rotary key ("Motif 3: Technical
+ * Report", Architecture: "normalized and expanded through a single
+ * projection", "RoPE is applied only to the rotary query and key").
+ *   c_hat[t]  = gamma (.) c_kv[t] / sqrt(mean(c_kv[t]^2) + rms_eps)
+ *   kv[t, h]  = c_hat[t] @ W_UKV[:, h*(d_nope+d_v) : (h+1)*(d_nope+d_v)]
+ *   k_rope_rot[t] = RoPE(k_rope[t], position t)
+ * Positions restart at 0 for every sequence. */
+typedef struct {
+  int B, L;                  /* batch, tokens per sequence (>= 1) */
+  int d_c, d_rope, n_kv, d_nope, d_v;
+  gdla_dtype dtype;
+  float rms_eps;             /* <= 0 selects 1e-6 */
+  int rope_max_pos;          /* rows of the RoPE tables; must be >= L */
+  const void* c_kv;          /* [B, L, d_c] pre-norm latent */
+  const void* gamma;         /* [d_c] RMSNorm gain */
+  const void* k_rope;        /* [B, L, d_rope] pre-RoPE rotary key */
+  const void* w_ukv;         /* [d_c, n_kv*(d_nope+d_v)]; per KV head: d_nope key cols, then d_v value cols */
+  const float* rope_cos;     /* [rope_max_pos, d_rope/2]: cos(pos * theta_k) */
+  const float* rope_sin;     /* [rope_max_pos, d_rope/2]: sin(pos * theta_k) */
+  void* kv_out;              /* [B, L, n_kv, d_nope+d_v] expanded key|value heads */
+  void* k_rope_out;          /* [B, L, d_rope] rotated rotary key */
+  void* c_hat_out;           /* [B, L, d_c] normalised latent; required (it feeds the GEMM) */
+} gdla_expand_args;
+
+gdla_status gdla_latent_expand(const gdla_expand_args* args, void* stream);
+
+/* -------------------------------------------------------------------- prefill
+ * The whole GDLA forward for B sequences of L tokens (steps 1-8): expansion as
+ * above into the workspace, then per head the attention
+ *   H_h,i = sum_j softmax_j( tau * (q_nope,h,i . k_nope,j + RoPE(q_rope,h,i) . k_rope_rot,j) ) v_j
+ * over the visible keys, then
+ *   Y_i = sigmoid(G_i) (.) ( H_S,i - sigmoid(lam_i) * H_N,floor(i/g) ).
+ * Heads of q are ordered: signal heads 0..n_signal-1, then noise heads
+ * 0..n_noise-1; each head holds d_nope content dims then d_rope pre-RoPE
+ * rotary dims. If cache_c_hat / cache_k_rope are not NULL, the normalised
+ * latent and rotated rotary key (the compact decode cache) are written there
+ * too. */
+typedef struct {
+  int B, L, d_c, d_rope, n_kv, d_nope, d_v, n_noise, g;
+  gdla_mask mask;
+  int window;                /* used iff mask == GDLA_MASK_SLIDING; >= 1 */
+  float softmax_scale;       /* tau; <= 0 selects 1/sqrt(d_nope + d_rope) */
+  float rms_eps;             /* <= 0 selects 1e-6 */
+  gdla_dtype dtype;
+  int rope_max_pos;          /* >= L */
+  const void* c_kv;          /* [B, L, d_c] */
+  const void* gamma;         /* [d_c] */
+  const void* k_rope;        /* [B, L, d_rope] pre-RoPE */
+  const void* q;             /* [B, L, n_signal+n_noise, d_nope+d_rope] */
+  const void* w_ukv;         /* [d_c, n_kv*(d_nope+d_v)] */
+  const float* rope_cos;     /* [rope_max_pos, d_rope/2] */
+  const float* rope_sin;     /* [rope_max_pos, d_rope/2] */
+  const float* lam_logits;   /* [B, L, n_signal] fp32 */
+  const void* gate_logits;   /* [B, L, n_signal, d_v] */
+  void* out;                 /* [B, L, n_signal, d_v] = Y */
+  void* cache_c_hat;         /* optional [B, L, d_c] */
+  void* cache_k_rope;        /* optional [B, L, d_rope] */
+  void* workspace;           /* >= gdla_prefill_workspace_size(args) bytes, 256-byte aligned */
+  size_t workspace_bytes;
+} gdla_prefill_args;
+
+size_t gdla_prefill_workspace_size(const gdla_prefill_args* args);
+gdla_status gdla_prefill(const gdla_prefill_args* args, void* stream);
+
+/* --------------------------------------------------------------------- attend
+ * Steps 3-8 alone over an already expanded latent (the second half of
+ * gdla_prefill): RoPE of the rotary query parts, signal and noise attention
+ * under the mask, differential subtraction and sigmoid gate, exactly as in
+ * gdla_prefill. `kv` and `k_rope_rot` are the outputs of gdla_latent_expand
+ * for the same batch. The workspace only carries the status word
+ * (>= 256 bytes, 256-byte aligned). */
+typedef struct {
+  int B, L, d_rope, n_kv, d_nope, d_v, n_noise, g;
+  gdla_mask mask;
+  int window;
+  float softmax_scale;       /* <= 0 selects 1/sqrt(d_nope + d_rope) */
+  gdla_dtype dtype;
+  int rope_max_pos;          /* >= L */
+  const void* q;             /* [B, L, n_signal+n_noise, d_nope+d_rope] */
+  const void* kv;            /* [B, L, n_kv, d_nope+d_v] */
+  const void* k_rope_rot;    /* [B, L, d_rope] rotated */
+  const float* rope_cos;     /* [rope_max_pos, d_rope/2] */
+  const float* rope_sin;
+  const float* lam_logits;   /* [B, L, n_signal] fp32 */
+  const void* gate_logits;   /* [B, L, n_signal, d_v] */
+  void* out;                 /* [B, L, n_signal, d_v] */
+  void* workspace;           /* status word */
+  size_t workspace_bytes;
+} gdla_attend_args;
+
+gdla_status gdla_attend(const gdla_attend_args* args, void* stream);
+
+/* --------------------------------------------------------------------- decode
+ * One new token per sequence over the compact latent cache ("Motif 3:
+ * Technical Report", Architecture: GDLA "preserves MLA's compact inference
+ * state"). The cache holds, per token, the normalised latent c_hat (d_c) and
+ * the rotated rotary key (d_rope). The query of sequence b sits at position
+ * seqlens[b]-1 and sees cache tokens 0..seqlens[b]-1 (or the last `window` of
+ * them under GDLA_MASK_SLIDING). The library evaluates the same attention as
+ * prefill with W_UK absorbed into the query and W_UV applied after the
+ * weighted sum of latents, which is equal in exact arithmetic. */
+typedef struct {
+  int B, T_max, d_c, d_rope, n_kv, d_nope, d_v, n_noise, g;
+  gdla_mask mask;
+  int window;
+  float softmax_scale;       /* <= 0 selects 1/sqrt(d_nope + d_rope) */
+  gdla_dtype dtype;
+  int rope_max_pos;          /* > max(seqlens) - 1 */
+  const int* seqlens;        /* [B] int32, 1 <= seqlens[b] <= T_max (device) */
+  const void* c_cache;       /* [B, T_max, d_c] normalised latent */
+  const void* kr_cache;      /* [B, T_max, d_rope] rotated rotary key */
+  const void* q;             /* [B, n_signal+n_noise, d_nope+d_rope], rotary part pre-RoPE */
+  const void* w_ukv;         /* [d_c, n_kv*(d_nope+d_v)] */
+  const float* rope_cos;     /* [rope_max_pos, d_rope/2] */
+  const float* rope_sin;
+  const float* lam_logits;   /* [B, n_signal] fp32 */
+  const void* gate_logits;   /* [B, n_signal, d_v] */
+  void* out;                 /* [B, n_signal, d_v] */
+  void* workspace;           /* >= gdla_decode_workspace_size(args) bytes */
+  size_t workspace_bytes;
+} gdla_decode_args;
+
+size_t gdla_decode_workspace_size(const gdla_decode_args* args);
+gdla_status gdla_decode(const gdla_decode_args* args, void* stream);
+
+/* ---------------------------------------------------------------- utilities */
+const char* gdla_status_string(gdla_status s);
+
+/* Reads (synchronously on `stream`) the device status word at the start of a
+ * prefill or decode workspace: GDLA_OK, or GDLA_ERR_TIMEOUT if a device-side
+ * wait of the last call hit its cap. The word is cleared by every call. */
+gdla_status gdla_workspace_status(const void* workspace, void* stream);
+
+/* Build information, for checks that the native library is the one loaded. */
+const char* gdla_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDLA_H_ */

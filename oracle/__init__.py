@@ -66,7 +66,7 @@ def _load():
             lib.gdla_oracle_prefill_rows.restype = ctypes.c_int
             lib.gdla_oracle_prefill_rows.argtypes = (
                 [ctypes.c_int, ctypes.c_long] + [ctypes.c_int] * 6 + [ctypes.c_int, ctypes.c_long]
-                + [ctypes.c_double] * 3 + [_dp] * 4 + [ctypes.c_long, _lp, _lp] + [_dp] * 5)
+                + [ctypes.c_double] * 3 + [_dp] * 4 + [ctypes.c_long, _lp, _lp] + [_dp] * 3 + [_ip] + [_dp] * 2)
             lib.gdla_oracle_decode_seq.restype = ctypes.c_int
             lib.gdla_oracle_decode_seq.argtypes = (
                 [ctypes.c_long] + [ctypes.c_int] * 6 + [ctypes.c_int, ctypes.c_long, ctypes.c_double,
@@ -162,8 +162,11 @@ def differential_gate(h_s, h_n, lam_logits, gate_logits, g: int) -> np.ndarray:
 # ------------------------------------------------------------------------- composites
 def prefill_rows(*, c_kv, gamma, k_rope, w_ukv, q_rows, lam_rows, gate_rows, row_b, row_i, g: int,
                  d_n: int, d_v: int, mask: int = MASK_CAUSAL, window: int = 0, scale: float | None = None,
-                 eps: float = DEFAULT_EPS, rope_base: float = DEFAULT_ROPE_BASE, want_heads: bool = False):
+                 eps: float = DEFAULT_EPS, rope_base: float = DEFAULT_ROPE_BASE, want_heads: bool = False,
+                 kv_sel=None):
     """Output rows Y [nrows, n_S, d_v] of the prefill for query tokens (row_b, row_i).
+    With ``kv_sel`` (a list of KV group indices) only those groups are computed
+    and the other groups' rows are NaN.
 
     c_kv [B, L, d_c], k_rope [B, L, d_R], w_ukv [d_c, n_kv*(d_n+d_v)], gamma [d_c]
     cover the whole batch; q_rows [nrows, n_S+n_N, d_n+d_R], lam_rows
@@ -185,12 +188,21 @@ def prefill_rows(*, c_kv, gamma, k_rope, w_ukv, q_rows, lam_rows, gate_rows, row
     ri = np.ascontiguousarray(row_i, dtype=np.int64)
     y = np.empty((nrows, n_S, d_v))
     heads = np.empty((nrows, H_q, d_v)) if want_heads else None
+    sel = None
+    if kv_sel is not None:
+        sel = np.zeros(n_kv, dtype=np.int32)
+        sel[np.asarray(kv_sel, dtype=np.int64)] = 1
     rc = _load().gdla_oracle_prefill_rows(
         B, L, d_c, d_R, n_kv, d_n, d_v, g, mask, window, scale, eps, rope_base,
         _p(c_kv), _p(gamma), _p(k_rope), _p(w_ukv), nrows, rb.ctypes.data_as(_lp), ri.ctypes.data_as(_lp),
-        _p(q_rows), _p(lam_rows), _p(gate_rows), _p(y), _p(heads) if want_heads else None)
+        _p(q_rows), _p(lam_rows), _p(gate_rows), sel.ctypes.data_as(_ip) if sel is not None else None, _p(y),
+        _p(heads) if want_heads else None)
     if rc != 0:
         raise ValueError("oracle prefill_rows rejected its arguments")
+    if sel is not None:
+        for h in range(n_kv):
+            if not sel[h]:
+                y[:, h * g:(h + 1) * g] = np.nan
     return (y, heads) if want_heads else y
 
 

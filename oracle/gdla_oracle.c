@@ -76,6 +76,22 @@ void gdla_oracle_latent_norm(const double* c, const double* gamma, long T, int d
   }
 }
 
+/* One token of step 2: out[n] = sum_{k=0}^{d_c-1} c_hat[k] * W[k, col0+n], summed in
+ * increasing k for every n (the loop over n is innermost only for memory order). */
+static void expand_token(const double* c_hat_t, const double* w_ukv, int d_c, long ncol, long col0,
+                         int d_n, int d_v, double* k_n_t, double* v_t) {
+  double acc[1024];
+  const int nn = d_n + d_v;
+  for (int n = 0; n < nn; ++n) acc[n] = 0.0;
+  for (int k = 0; k < d_c; ++k) {
+    const double a = c_hat_t[k];
+    const double* wr = w_ukv + k * ncol + col0;
+    for (int n = 0; n < nn; ++n) acc[n] += a * wr[n];
+  }
+  for (int n = 0; n < d_n; ++n) k_n_t[n] = acc[n];
+  for (int n = 0; n < d_v; ++n) v_t[n] = acc[d_n + n];
+}
+
 /* ---- step 2: one up-projection into n_kv key (nope) and value heads ------------
  * W_UKV is [d_c, n_kv*(d_n+d_v)] row-major; the columns of KV head h are
  * h*(d_n+d_v) .. h*(d_n+d_v)+d_n-1 for the key and the next d_v for the value.
@@ -86,16 +102,8 @@ void gdla_oracle_expand_head(const double* c_hat, const double* w_ukv, long T, i
   const long ncol = (long)n_kv * (d_n + d_v);
   const long col0 = (long)h * (d_n + d_v);
 #pragma omp parallel for schedule(static)
-  for (long t = 0; t < T; ++t) {
-    for (int n = 0; n < d_n + d_v; ++n) {
-      double acc = 0.0;
-      for (int k = 0; k < d_c; ++k) acc += c_hat[t * d_c + k] * w_ukv[k * ncol + col0 + n];
-      if (n < d_n)
-        k_n[t * d_n + n] = acc;
-      else
-        v[t * d_v + (n - d_n)] = acc;
-    }
-  }
+  for (long t = 0; t < T; ++t) expand_token(c_hat + t * d_c, w_ukv, d_c, ncol, col0, d_n, d_v,
+                                            k_n + t * d_n, v + t * d_v);
 }
 
 /* ---- step 3: RoPE, rotate-half pairing -----------------------------------------
@@ -199,6 +207,9 @@ void gdla_oracle_differential_gate(const double* h_s, const double* h_nz, const 
  *   q_rows [nrows, n_S+n_N, d_n+d_R]  heads 0..n_S-1 signal, then the n_N noise
  *          heads; per head the nope part first, then the pre-RoPE rotary part
  *   lam_rows [nrows, n_S]; gate_rows [nrows, n_S, d_v]
+ * kv_sel [n_kv] (optional) restricts the work to the KV groups whose flag is
+ * non-zero (their noise head and g signal heads); the other groups' outputs are
+ * zero.
  * Outputs: y_rows [nrows, n_S, d_v]; heads_out (optional) [nrows, n_S+n_N, d_v]
  * holds every head's H before the differential step.
  * n_N must equal n_kv. Returns 0, or -1 on bad arguments.
@@ -208,9 +219,9 @@ int gdla_oracle_prefill_rows(int B, long L, int d_c, int d_R, int n_kv, int d_n,
                              double rope_base, const double* c_kv, const double* gamma,
                              const double* k_rope, const double* w_ukv, long nrows,
                              const long* row_b, const long* row_i, const double* q_rows,
-                             const double* lam_rows, const double* gate_rows, double* y_rows,
-                             double* heads_out) {
-  if (B < 1 || L < 1 || g < 1 || n_kv < 1 || d_R % 2 || d_R > 512 ||
+                             const double* lam_rows, const double* gate_rows, const int* kv_sel,
+                             double* y_rows, double* heads_out) {
+  if (B < 1 || L < 1 || g < 1 || n_kv < 1 || d_R % 2 || d_R > 512 || d_n + d_v > 1024 ||
       (mask == ORACLE_MASK_SLIDING && window < 1))
     return -1;
   const int n_N = n_kv, n_S = g * n_N, H_q = n_S + n_N, d_qk = d_n + d_R;
@@ -244,21 +255,14 @@ int gdla_oracle_prefill_rows(int B, long L, int d_c, int d_R, int n_kv, int d_n,
       gdla_oracle_rope(k_rope + ((long)b * L + j) * d_R, j, d_R, rope_base, k_r_rot + j * d_R);
 
     for (int h = 0; h < n_kv; ++h) {
+      if (kv_sel && !kv_sel[h]) continue;
       /* step 2 for KV head h, only at the tokens that are needed */
       const long ncol = (long)n_kv * (d_n + d_v);
       const long col0 = (long)h * (d_n + d_v);
 #pragma omp parallel for schedule(static)
-      for (long t = 0; t < T; ++t) {
-        if (!need[t]) continue;
-        for (int n = 0; n < d_n + d_v; ++n) {
-          double acc = 0.0;
-          for (int k = 0; k < d_c; ++k) acc += c_hat[t * d_c + k] * w_ukv[k * ncol + col0 + n];
-          if (n < d_n)
-            k_n[t * d_n + n] = acc;
-          else
-            v[t * d_v + (n - d_n)] = acc;
-        }
-      }
+      for (long t = 0; t < T; ++t)
+        if (need[t])
+          expand_token(c_hat + t * d_c, w_ukv, d_c, ncol, col0, d_n, d_v, k_n + t * d_n, v + t * d_v);
       /* steps 3-6 for the heads that read KV head h: noise head h and signal
        * heads h*g .. h*g+g-1 */
 #pragma omp parallel for schedule(dynamic)
@@ -306,7 +310,7 @@ int gdla_oracle_decode_seq(long T, int d_c, int d_R, int n_kv, int d_n, int d_v,
                            const double* c_hat, const double* k_r_rot, const double* q,
                            const double* w_ukv, const double* lam, const double* gate,
                            const int* kv_sel, double* y, double* heads_out) {
-  if (T < 1 || g < 1 || n_kv < 1 || d_R % 2 || d_R > 512 ||
+  if (T < 1 || g < 1 || n_kv < 1 || d_R % 2 || d_R > 512 || d_n + d_v > 1024 ||
       (mask == ORACLE_MASK_SLIDING && window < 1))
     return -1;
   const int n_N = n_kv, n_S = g * n_N, H_q = n_S + n_N, d_qk = d_n + d_R;

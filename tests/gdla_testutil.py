@@ -1,0 +1,67 @@
+"""Shared test helpers: run the fp64 oracle on (slices of) the same seeded
+tensors the CUDA path receives, and the parity tolerance.
+
+Tolerance: fp32 tensors -> max |Y_gpu - Y_oracle| <= 1e-4 (absolute); bf16
+tensors -> max |Y_gpu - Y_oracle| <= 1e-2 * RMS(Y_oracle) over the compared
+elements.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+FP32_ATOL = 1e-4
+BF16_REL_RMS = 1e-2
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def mask_code(mask: str) -> int:
+    return oracle.MASK_CAUSAL if mask == "causal" else oracle.MASK_SLIDING
+
+
+def oracle_prefill_rows(inp: dict, rows, *, g: int, d_nope: int, d_v: int, mask: str = "causal", window: int = 0,
+                        want_heads: bool = False):
+    """Oracle Y for the (b, i) pairs in ``rows`` from the prefill inputs ``inp``."""
+    rows = list(rows)
+    rb = torch.tensor([r[0] for r in rows], dtype=torch.long)
+    ri = torch.tensor([r[1] for r in rows], dtype=torch.long)
+    dev = inp["q"].device
+    rbd, rid = rb.to(dev), ri.to(dev)
+    return oracle.prefill_rows(
+        c_kv=f64(inp["c_kv"]), gamma=f64(inp["gamma"]), k_rope=f64(inp["k_rope"]), w_ukv=f64(inp["w_ukv"]),
+        q_rows=f64(inp["q"][rbd, rid]), lam_rows=f64(inp["lam_logits"][rbd, rid]),
+        gate_rows=f64(inp["gate_logits"][rbd, rid]), row_b=rb.numpy(), row_i=ri.numpy(), g=g, d_n=d_nope, d_v=d_v,
+        mask=mask_code(mask), window=window, want_heads=want_heads)
+
+
+def oracle_decode(inp: dict, *, g: int, d_nope: int, d_v: int, seqs=None, kv_sel=None, mask="causal", window=0):
+    """Oracle decode output [len(seqs), n_S, d_v] for the selected sequences."""
+    B = inp["c_cache"].shape[0]
+    seqs = range(B) if seqs is None else seqs
+    outs = []
+    for b in seqs:
+        T = int(inp["seqlens"][b])
+        outs.append(oracle.decode_seq(
+            c_hat=f64(inp["c_cache"][b, :T]), k_r_rot=f64(inp["kr_cache"][b, :T]), q=f64(inp["q"][b]),
+            w_ukv=f64(inp["w_ukv"]), lam=f64(inp["lam_logits"][b]), gate=f64(inp["gate_logits"][b]), g=g,
+            d_n=d_nope, d_v=d_v, kv_sel=kv_sel, mask=mask_code(mask), window=window))
+    return np.stack(outs)
+
+
+def assert_parity(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = ""):
+    """The acceptance bar: fp32 -> 1e-4 absolute; bf16 -> 1e-2 x RMS(ref)."""
+    sel = ~np.isnan(ref)
+    got, ref = got[sel], ref[sel]
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = float(np.abs(got - ref).max())
+    if dtype == torch.float32:
+        assert err <= FP32_ATOL, f"{what}: max abs err {err:.3e} > {FP32_ATOL}"
+    else:
+        rms = float(np.sqrt((ref * ref).mean()))
+        assert err <= BF16_REL_RMS * rms, f"{what}: max abs err {err:.3e} > 1e-2 * rms {rms:.3e}"
+    return err

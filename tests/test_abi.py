@@ -1,0 +1,139 @@
+"""The C ABI on the host (no GPU): the library loads, exports every symbol the
+header declares, the ctypes mirror matches the C struct layout, and invalid
+arguments are rejected synchronously before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from differential_latent_attention_gdla_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_abi.LIB_PATH):
+        build.build()
+    return _abi.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdla_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(_abi.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert "sm_100a" in lib.gdla_build_info().decode()
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert lib.gdla_status_string(code)
+    assert b"INVALID" in lib.gdla_status_string(_abi.GDLA_ERR_INVALID_ARG)
+
+
+def _c_layout(struct: str, fields):
+    prog = "#include <stdio.h>\n#include <stddef.h>\n#include \"gdla.h\"\nint main(void){\n"
+    prog += f'printf("%zu\\n", sizeof({struct}));\n'
+    for f in fields:
+        prog += f'printf("%zu\\n", offsetof({struct}, {f}));\n'
+    prog += "return 0;}\n"
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split()
+    return [int(x) for x in out]
+
+
+@pytest.mark.parametrize("cls,cname", [(_abi.ExpandArgs, "gdla_expand_args"), (_abi.PrefillArgs, "gdla_prefill_args"),
+                                       (_abi.AttendArgs, "gdla_attend_args"),
+                                       (_abi.DecodeArgs, "gdla_decode_args")])
+def test_ctypes_mirror_matches_c_layout(cls, cname):
+    fields = [f[0] for f in cls._fields_]
+    got = [ctypes.sizeof(cls)] + [getattr(cls, f).offset for f in fields]
+    assert got == _c_layout(cname, fields)
+
+
+def good_prefill():
+    a = _abi.PrefillArgs(2, 100, 512, 64, 16, 128, 128, 16, 3, _abi.GDLA_MASK_CAUSAL, 0, 0.0, 0.0, _abi.GDLA_BF16, 100)
+    base = 0x10000000
+    for i, f in enumerate(("c_kv", "gamma", "k_rope", "q", "w_ukv", "rope_cos", "rope_sin", "lam_logits",
+                           "gate_logits", "out", "workspace")):
+        setattr(a, f, base + i * 0x1000000)
+    return a
+
+
+def test_prefill_validation_rejects_before_launch(lib):
+    def st(mut):
+        a = good_prefill()
+        a.workspace_bytes = lib.gdla_prefill_workspace_size(ctypes.byref(a))
+        mut(a)
+        return lib.gdla_prefill(ctypes.byref(a), None)
+
+    E, U = _abi.GDLA_ERR_INVALID_ARG, _abi.GDLA_ERR_UNSUPPORTED
+    assert st(lambda a: setattr(a, "B", 0)) == E
+    assert st(lambda a: setattr(a, "L", 0)) == E
+    assert st(lambda a: setattr(a, "q", 0)) == E                      # NULL
+    assert st(lambda a: setattr(a, "q", 0x10000008)) == E             # misaligned
+    assert st(lambda a: setattr(a, "workspace", a.workspace + 16)) == E  # not 256-aligned
+    assert st(lambda a: setattr(a, "workspace_bytes", a.workspace_bytes - 1)) == E
+    assert st(lambda a: setattr(a, "rope_max_pos", 99)) == E
+    assert st(lambda a: (setattr(a, "mask", _abi.GDLA_MASK_SLIDING), setattr(a, "window", 0))) == E
+    assert st(lambda a: setattr(a, "mask", 7)) == E
+    assert st(lambda a: setattr(a, "dtype", 5)) == E
+    assert st(lambda a: setattr(a, "n_noise", 8)) == U                # n_noise != n_kv
+    assert st(lambda a: setattr(a, "g", 9)) == U
+    assert st(lambda a: setattr(a, "d_nope", 96)) == U
+    assert st(lambda a: setattr(a, "d_c", 300)) == U
+    assert st(lambda a: setattr(a, "cache_c_hat", 0x20000004)) == E   # optional but misaligned
+    assert lib.gdla_prefill(None, None) == E
+
+
+def test_prefill_workspace_size_is_monotone(lib):
+    a = good_prefill()
+    s1 = lib.gdla_prefill_workspace_size(ctypes.byref(a))
+    a.L = 200
+    s2 = lib.gdla_prefill_workspace_size(ctypes.byref(a))
+    assert s2 > s1 > 2 * 100 * 16 * 256 * 2
+    assert s1 % 256 == 0
+
+
+def test_decode_validation_rejects_before_launch(lib):
+    def good():
+        a = _abi.DecodeArgs(4, 1000, 512, 64, 16, 128, 128, 16, 2, _abi.GDLA_MASK_CAUSAL, 0, 0.0, _abi.GDLA_BF16,
+                            1000)
+        base = 0x10000000
+        for i, f in enumerate(("seqlens", "c_cache", "kr_cache", "q", "w_ukv", "rope_cos", "rope_sin", "lam_logits",
+                               "gate_logits", "out", "workspace")):
+            setattr(a, f, base + i * 0x1000000)
+        a.workspace_bytes = lib.gdla_decode_workspace_size(ctypes.byref(a))
+        return a
+
+    E, U = _abi.GDLA_ERR_INVALID_ARG, _abi.GDLA_ERR_UNSUPPORTED
+    for mut, want in ((lambda a: setattr(a, "B", 0), E), (lambda a: setattr(a, "c_cache", 0), E),
+                      (lambda a: setattr(a, "workspace_bytes", 1024), E), (lambda a: setattr(a, "rope_max_pos", 10), E),
+                      (lambda a: setattr(a, "n_noise", 4), U), (lambda a: setattr(a, "d_rope", 48), U),
+                      (lambda a: (setattr(a, "mask", 1), setattr(a, "window", -3)), E)):
+        a = good()
+        mut(a)
+        assert lib.gdla_decode(ctypes.byref(a), None) == want
+    assert lib.gdla_decode_workspace_size(ctypes.byref(good())) > 4 * 48 * 512 * 4
+
+
+def test_expand_validation(lib):
+    a = _abi.ExpandArgs(1, 10, 512, 64, 16, 128, 128, _abi.GDLA_BF16, 0.0, 5)
+    assert lib.gdla_latent_expand(ctypes.byref(a), None) == _abi.GDLA_ERR_INVALID_ARG  # table too short
+    a.rope_max_pos = 10
+    assert lib.gdla_latent_expand(ctypes.byref(a), None) == _abi.GDLA_ERR_INVALID_ARG  # NULL pointers

@@ -421,3 +421,16 @@ def test_decode_group_selection():
     part = oracle.decode_seq(kv_sel=[1], **kw)
     np.testing.assert_array_equal(part[2:4], full[2:4])
     assert np.isnan(part[:2]).all() and np.isnan(part[4:]).all()
+
+
+def test_prefill_group_selection_matches_full():
+    inp = tiny_inputs(n_kv=3, g=2)
+    full = run_all_rows(inp)
+    B, L = inp["c_kv"].shape[:2]
+    rb, ri = np.meshgrid(np.arange(B), np.arange(L), indexing="ij")
+    rb, ri = rb.ravel(), ri.ravel()
+    part = oracle.prefill_rows(c_kv=inp["c_kv"], gamma=inp["gamma"], k_rope=inp["k_rope"], w_ukv=inp["w_ukv"],
+                               q_rows=inp["q"][rb, ri], lam_rows=inp["lam"][rb, ri], gate_rows=inp["gate"][rb, ri],
+                               row_b=rb, row_i=ri, g=2, d_n=inp["d_n"], d_v=inp["d_v"], kv_sel=[1]).reshape(full.shape)
+    np.testing.assert_array_equal(part[:, :, 2:4], full[:, :, 2:4])
+    assert np.isnan(part[:, :, :2]).all() and np.isnan(part[:, :, 4:]).all()

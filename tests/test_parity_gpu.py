@@ -1,0 +1,165 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.
+
+Small cases are compared element by element over every output; they span
+several tiles and a ragged tail. The full-size workloads are compared on a
+deterministic sample of query rows (rows 0, 1, 127, 128, W-1, W, W+1, L-1 and
+seeded random rows), all heads of every sampled row.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import differential_latent_attention_gdla_b200 as gdla
+from differential_latent_attention_gdla_b200 import workloads as wl
+from gdla_testutil import assert_parity, f64, oracle_decode, oracle_prefill_rows
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_prefill(shape, inp, **kw):
+    cos, sin = gdla.rope_tables(shape.L, shape.d_R, device=DEV)
+    return gdla.prefill(inp["c_kv"], inp["gamma"], inp["k_rope"], inp["q"], inp["w_ukv"], cos, sin,
+                        inp["lam_logits"], inp["gate_logits"], g=shape.g, mask=shape.mask, window=shape.window, **kw)
+
+
+def all_rows(shape):
+    return [(b, i) for b in range(shape.B) for i in range(shape.L)]
+
+
+SMALL = [
+    wl.PREFILL["tiny_fp32"],
+    wl.PrefillShape("bf16 small causal g=3 ragged", B=2, L=300, n_kv=2, g=3),
+    wl.PrefillShape("bf16 small sliding W=100 g=2 ragged", B=1, L=333, n_kv=3, g=2, mask="sliding", window=100),
+    wl.PrefillShape("bf16 sliding W=1", B=1, L=130, n_kv=1, g=2, mask="sliding", window=1),
+    wl.PrefillShape("bf16 sliding W>=L", B=1, L=200, n_kv=1, g=3, mask="sliding", window=500),
+    wl.PrefillShape("bf16 L=1", B=3, L=1, n_kv=2, g=2),
+    wl.PrefillShape("bf16 d=64", B=1, L=257, d_c=256, d_R=32, n_kv=2, d_n=64, d_v=64, g=4),
+    wl.PrefillShape("fp32 d=128 causal", B=1, L=150, n_kv=1, g=3, dtype="fp32"),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: s.name)
+@pytest.mark.parametrize("act", ["unit", "fan_in"])
+def test_prefill_small_every_element(shape, act):
+    inp = wl.make_prefill_inputs(shape, seed=11, device=DEV, act=act)
+    y = run_prefill(shape, inp)
+    torch.cuda.synchronize()
+    ref = oracle_prefill_rows(inp, all_rows(shape), g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=shape.mask,
+                              window=shape.window)
+    got = f64(y).reshape(ref.shape)
+    assert_parity(got, ref, wl.torch_dtype(shape.dtype), shape.name)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_latent_expand_against_oracle_expansion(dtype):
+    shape = wl.PrefillShape("expand", B=2, L=200, n_kv=3, g=1, dtype=dtype)
+    inp = wl.make_prefill_inputs(shape, seed=3, device=DEV)
+    cos, sin = gdla.rope_tables(shape.L, shape.d_R, device=DEV)
+    kv, krot, chat = gdla.latent_expand(inp["c_kv"], inp["gamma"], inp["k_rope"], inp["w_ukv"], cos, sin,
+                                        n_kv=shape.n_kv, d_nope=shape.d_n, d_v=shape.d_v)
+    torch.cuda.synchronize()
+    w = f64(inp["w_ukv"])
+    for b in range(shape.B):
+        ch = oracle.latent_norm(f64(inp["c_kv"][b]), f64(inp["gamma"]), oracle.DEFAULT_EPS)
+        assert_parity(f64(chat[b]), ch, wl.torch_dtype(dtype), "c_hat")
+        for h in range(shape.n_kv):
+            k, v = oracle.expand_head(ch, w, shape.n_kv, shape.d_n, shape.d_v, h)
+            assert_parity(f64(kv[b, :, h, :shape.d_n]), k, wl.torch_dtype(dtype), f"k_nope head {h}")
+            assert_parity(f64(kv[b, :, h, shape.d_n:]), v, wl.torch_dtype(dtype), f"v head {h}")
+        kr = np.stack([oracle.rope(f64(inp["k_rope"][b, j]), j) for j in range(shape.L)])
+        assert_parity(f64(krot[b]), kr, wl.torch_dtype(dtype), "k_rope_rot")
+
+
+@pytest.mark.parametrize("name", ["b4_l4k_g2", "b1_l32k_g3", "b2_l64k_swa4k"])
+def test_prefill_full_size_sampled_rows(name):
+    shape = wl.PREFILL[name]
+    inp = wl.make_prefill_inputs(shape, seed=0, device=DEV)
+    y = run_prefill(shape, inp)
+    torch.cuda.synchronize()
+    rows = wl.sample_rows(shape, n_random=8 if shape.mask == "sliding" else 12)
+    ref = oracle_prefill_rows(inp, rows, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=shape.mask,
+                              window=shape.window)
+    rb = torch.tensor([r[0] for r in rows], device=DEV)
+    ri = torch.tensor([r[1] for r in rows], device=DEV)
+    got = f64(y[rb, ri])
+    assert_parity(got, ref, torch.bfloat16, name)
+    assert torch.isfinite(y).all()
+
+
+def test_prefill_lambda_one_identical_queries_cancel():
+    """Signal queries equal to their noise head's query with lambda -> 1 give
+    D = 0: the kernel's output must vanish to rounding level."""
+    shape = wl.PrefillShape("cancel", B=1, L=256, n_kv=2, g=3)
+    inp = wl.make_prefill_inputs(shape, seed=5, device=DEV)
+    for i in range(shape.n_S):
+        inp["q"][:, :, i] = inp["q"][:, :, shape.n_S + i // shape.g]
+    inp["lam_logits"].fill_(30.0)
+    y = run_prefill(shape, inp)
+    ref_scale = float(f64(run_prefill(shape, dict(inp, lam_logits=torch.full_like(inp["lam_logits"], -30.0)))).std())
+    assert float(y.float().abs().max()) <= 1e-2 * ref_scale
+
+
+def test_prefill_emits_decode_cache_and_decode_matches_last_row():
+    shape = wl.PrefillShape("prefill->decode", B=2, L=520, n_kv=2, g=2)
+    inp = wl.make_prefill_inputs(shape, seed=9, device=DEV)
+    cache_c = torch.empty((shape.B, shape.L, shape.d_c), dtype=torch.bfloat16, device=DEV)
+    cache_k = torch.empty((shape.B, shape.L, shape.d_R), dtype=torch.bfloat16, device=DEV)
+    y = run_prefill(shape, inp, cache_c_hat=cache_c, cache_k_rope=cache_k)
+    cos, sin = gdla.rope_tables(shape.L, shape.d_R, device=DEV)
+    for T in (1, 129, 520):
+        seqlens = torch.full((shape.B,), T, dtype=torch.int32, device=DEV)
+        yd = gdla.decode(cache_c, cache_k, inp["q"][:, T - 1].contiguous(), inp["w_ukv"], cos, sin,
+                         inp["lam_logits"][:, T - 1].contiguous(), inp["gate_logits"][:, T - 1].contiguous(), seqlens,
+                         g=shape.g)
+        torch.cuda.synchronize()
+        ref = oracle_prefill_rows(inp, [(b, T - 1) for b in range(shape.B)], g=shape.g, d_nope=shape.d_n,
+                                  d_v=shape.d_v)
+        assert_parity(f64(yd), ref, torch.bfloat16, f"decode T={T}")
+        assert_parity(f64(y[:, T - 1]), ref, torch.bfloat16, f"prefill row {T - 1}")
+
+
+DECODE_SMALL = [
+    (wl.DecodeShape("decode small ragged", B=3, T=300, n_kv=2, g=2), [300, 37, 1], "causal", 0),
+    (wl.DecodeShape("decode sliding", B=2, T=700, n_kv=1, g=3), [700, 200], "sliding", 128),
+    (wl.DecodeShape("decode d=32 fp32", B=2, T=150, d_c=64, d_R=16, n_kv=4, d_n=32, d_v=32, g=2, dtype="fp32"),
+     [150, 77], "causal", 0),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_SMALL, ids=lambda c: c[0].name)
+@pytest.mark.parametrize("act", ["unit", "fan_in"])
+def test_decode_small_every_element(case, act):
+    shape, seqlens, mask, window = case
+    inp = wl.make_decode_inputs(shape, seed=4, device=DEV, act=act, seqlens=seqlens)
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g, mask=mask, window=window)
+    torch.cuda.synchronize()
+    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=mask, window=window)
+    assert_parity(f64(y), ref, wl.torch_dtype(shape.dtype), shape.name)
+
+
+def test_decode_full_size_sampled():
+    shape = wl.DECODE["b64_t32k"]
+    inp = wl.make_decode_inputs(shape, seed=0, device=DEV)
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g)
+    torch.cuda.synchronize()
+    assert torch.isfinite(y).all()
+    seqs = [0, 37, 63]
+    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, seqs=seqs, kv_sel=[0, 9, 15])
+    assert_parity(f64(y[seqs]), ref, torch.bfloat16, "decode b64_t32k")
+
+
+def test_binding_raises_on_invalid_arguments():
+    shape = wl.PrefillShape("bad", B=1, L=64, n_kv=1, g=2, mask="sliding", window=0)
+    inp = wl.make_prefill_inputs(shape, seed=1, device=DEV)
+    with pytest.raises(gdla.GdlaError):
+        run_prefill(shape, inp)
