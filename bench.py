@@ -44,7 +44,30 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--prefill", default=PREFILL_NAME, help="prefill workload name (profiling uses smaller ones)")
+    ap.add_argument("--decode", default=DECODE_NAME, help="decode workload name")
     return ap.parse_args()
+
+
+def max_over_ranks(values, world: int, device="cpu"):
+    """Element-wise max of per-rank timings (every rank calls this once)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_value(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / seconds
+
+
+def rank_seed(seed: int, rank: int, which: str) -> int:
+    """Each rank draws an independent problem of the same shape."""
+    return seed + rank + (1000 if which == "decode" else 0)
 
 
 def peaks():
@@ -177,11 +200,11 @@ def run_ours(a):
         if world > 1:
             dist.barrier()
 
-    P = wl.PREFILL[PREFILL_NAME]
-    D = wl.DECODE[DECODE_NAME]
+    P = wl.PREFILL[a.prefill]
+    D = wl.DECODE[a.decode]
     # every rank runs its own independent problem (weak scaling, no collective on the data path)
-    pin = wl.make_prefill_inputs(P, seed=a.seed + rank, device=dev)
-    din = wl.make_decode_inputs(D, seed=a.seed + 1000 + rank, device=dev)
+    pin = wl.make_prefill_inputs(P, seed=rank_seed(a.seed, rank, "prefill"), device=dev)
+    din = wl.make_decode_inputs(D, seed=rank_seed(a.seed, rank, "decode"), device=dev)
     cos, sin = gdla.rope_tables(max(P.L, D.T), P.d_R, device=dev)
     kv = torch.empty((P.B, P.L, P.n_kv, P.d_n + P.d_v), dtype=torch.bfloat16, device=dev)
     krot = torch.empty((P.B, P.L, P.d_R), dtype=torch.bfloat16, device=dev)
@@ -236,19 +259,16 @@ def run_ours(a):
     t_att = sum(e[1].elapsed_time(e[2]) for e in ev) / a.steps
     t_dec = sum(e[2].elapsed_time(e[3]) for e in ev) / a.steps
     t_step = ev[0][0].elapsed_time(ev[-1][3]) / a.steps
-    loc = torch.tensor([t_exp, t_att, t_dec, t_step], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(loc, op=dist.ReduceOp.MAX)
-    t_exp, t_att, t_dec, t_step = [float(x) for x in loc.tolist()]
+    t_exp, t_att, t_dec, t_step = max_over_ranks([t_exp, t_att, t_dec, t_step], world, dev)
 
     pf = P.algorithmic_flops()
     f_exp = 2.0 * P.B * P.L * P.d_c * P.n_kv * (P.d_n + P.d_v)
     f_att = pf - f_exp
     db = D.algorithmic_bytes()
     pk = peaks()
-    value = pf * world / ((t_exp + t_att) * 1e-3) / 1e12
+    value = weak_scaling_value(pf, world, (t_exp + t_att) * 1e-3) / 1e12
     att_tflops = f_att / (t_att * 1e-3) / 1e12
-    dec_gbs = db * world / (t_dec * 1e-3) / 1e9
+    dec_gbs = weak_scaling_value(db, world, t_dec * 1e-3) / 1e9
 
     # end to end through the public call with host buffers (pinned), copies inside the timed region
     e2e = None
@@ -277,12 +297,10 @@ def run_ours(a):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        t = torch.tensor([e0.elapsed_time(e1) / a.e2e_steps], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        (t,) = max_over_ranks([e0.elapsed_time(e1) / a.e2e_steps], world, dev)
         h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
-        e2e = {"value": pf * world / (float(t) * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": yh.numel() * yh.element_size(), "ms_per_step": float(t)}
+        e2e = {"value": weak_scaling_value(pf, world, t * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": yh.numel() * yh.element_size(), "ms_per_step": t}
         del ws, dev_in, host
 
     cpu = None
@@ -297,8 +315,8 @@ def run_ours(a):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) recipe)",
-            "config": {"workload": f"prefill B=1 L=32768 g=3 causal (value, TFLOP/s) + decode B=64 T=32768 g=2 "
-                                   f"(decode.value, GB/s)", "prefill": PREFILL_NAME, "decode": DECODE_NAME,
+            "config": {"workload": f"prefill {P.name} (value, TFLOP/s) + decode {D.name} "
+                                   f"(decode.value, GB/s)", "prefill": a.prefill, "decode": a.decode,
                        "l2": "inputs larger than L2 (q 805 MB, cache 2.4 GB); no flush",
                        "parallelism": f"{world} independent replicas (weak scaling)"},
             "prefill": {"ms": t_exp + t_att, "expand_ms": t_exp, "attend_ms": t_att,

@@ -17,47 +17,60 @@
 
 namespace gdla {
 
-// One block per (KV group, sequence); one warp per latent row c at a time.
+// Sequences per block of the absorb and combine kernels: one W_UK / W_UV slice
+// of a KV group is read once per block and reused for SEQ_PER_BLOCK sequences.
+constexpr int SEQ_PER_BLOCK = 4;
+constexpr int MAX_ROWS = SEQ_PER_BLOCK * 9;  // (g+1) <= 9 heads per KV group
+
+// q_abs[b, head, c] = sum_n W_UKV[c, h*(d_nope+d_v) + n] * q_nope[b, head, n] for the
+// g+1 heads of KV group h, and RoPE of their rotary parts at position seqlen-1.
+// Block (KV group h, chunk of sequences); each thread owns latent rows c.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv;
-  const int dqk = p.d_nope + p.d_rope, ncol = p.n_kv * (p.d_nope + p.d_v);
+  const int h = blockIdx.x, b0 = blockIdx.y * SEQ_PER_BLOCK;
+  const int nb = min(SEQ_PER_BLOCK, p.B - b0);
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1;
+  const int dqk = p.d_nope + p.d_rope, ncol = p.n_kv * (p.d_nope + p.d_v), DN = p.d_nope;
   const T* q = reinterpret_cast<const T*>(p.q);
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
-  extern __shared__ float qn[];  // [(g+1)][d_nope]
-  const int G1 = p.g + 1;
-  for (int e = threadIdx.x; e < G1 * p.d_nope; e += blockDim.x) {
-    const int which = e / p.d_nope, k = e % p.d_nope;
-    const int head = which < p.g ? h * p.g + which : n_S + h;
-    qn[e] = to_f(q[((long)b * H_q + head) * dqk + k]);
+  extern __shared__ float qn[];  // [R][d_nope]
+  for (int e = threadIdx.x; e < R * DN; e += blockDim.x) {
+    const int r = e / DN, k = e % DN, bl = r / G1, u = r % G1;
+    const int head = u < p.g ? h * p.g + u : n_S + h;
+    qn[e] = to_f(q[((long)(b0 + bl) * H_q + head) * dqk + k]);
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int c = warp; c < p.d_c; c += blockDim.x >> 5) {
+  for (int c = threadIdx.x; c < p.d_c; c += blockDim.x) {
     const T* wr = w + (long)c * ncol + (long)h * (p.d_nope + p.d_v);
-    float acc[9];
-    for (int u = 0; u < G1; ++u) acc[u] = 0.f;
-    for (int k = lane; k < p.d_nope; k += 32) {
-      const float wv = to_f(wr[k]);
-      for (int u = 0; u < G1; ++u) acc[u] = fmaf(wv, qn[u * p.d_nope + k], acc[u]);
-    }
-    for (int u = 0; u < G1; ++u) {
-      float a = acc[u];
+    float acc[MAX_ROWS];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0) {
+    for (int r = 0; r < MAX_ROWS; ++r) acc[r] = 0.f;
+    for (int k = 0; k < DN; k += 4) {
+      const float w0 = to_f(wr[k]), w1 = to_f(wr[k + 1]), w2 = to_f(wr[k + 2]), w3 = to_f(wr[k + 3]);
+#pragma unroll
+      for (int r = 0; r < MAX_ROWS; ++r) {
+        if (r < R) {
+          const float* qr = qn + r * DN + k;
+          acc[r] = fmaf(w0, qr[0], fmaf(w1, qr[1], fmaf(w2, qr[2], fmaf(w3, qr[3], acc[r]))));
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < MAX_ROWS; ++r) {
+      if (r < R) {
+        const int bl = r / G1, u = r % G1;
         const int head = u < p.g ? h * p.g + u : n_S + h;
-        p.q_abs[((long)b * H_q + head) * p.d_c + c] = a;
+        p.q_abs[((long)(b0 + bl) * H_q + head) * p.d_c + c] = acc[r];
       }
     }
   }
   // RoPE of the rotary query parts at position seqlen-1
-  const int pos = p.seqlens[b] - 1;
   const int half = p.d_rope >> 1;
-  for (int e = threadIdx.x; e < G1 * half; e += blockDim.x) {
-    const int which = e / half, k = e % half;
-    const int head = which < p.g ? h * p.g + which : n_S + h;
+  for (int e = threadIdx.x; e < R * half; e += blockDim.x) {
+    const int r = e / half, k = e % half, bl = r / G1, u = r % G1;
+    const int b = b0 + bl;
+    const int head = u < p.g ? h * p.g + u : n_S + h;
+    const int pos = p.seqlens[b] - 1;
     const T* qr = q + ((long)b * H_q + head) * dqk + p.d_nope;
     const float cs = p.cos_tab[(long)pos * half + k], sn = p.sin_tab[(long)pos * half + k];
     const float x1 = to_f(qr[k]), x2 = to_f(qr[k + half]);
@@ -177,65 +190,83 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
 }
 
 // Merge the splits of every head of one KV group, apply W_UV, then
-// D = H_S - sigmoid(lam) H_N and Y = sigmoid(G) D.
+// D = H_S - sigmoid(lam) H_N and Y = sigmoid(G) D. Block (KV group h, chunk of
+// sequences); the W_UV slice is streamed once per block.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1;
-  const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v);
+  const int h = blockIdx.x, b0 = blockIdx.y * SEQ_PER_BLOCK;
+  const int nb = min(SEQ_PER_BLOCK, p.B - b0);
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1;
+  const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v), NS = p.n_splits;
   extern __shared__ float sm[];
-  float* olat = sm;               // [G1][d_c]
-  float* hv = olat + G1 * d_c;    // [G1][DV]
-  float* wgt = hv + G1 * DV;      // [G1][n_splits]
+  float* olat = sm;               // [R][d_c]
+  float* hv = olat + R * d_c;     // [R][DV]
+  float* wgt = hv + R * DV;       // [R][n_splits]
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   const T* gate = reinterpret_cast<const T*>(p.gate);
   T* out = reinterpret_cast<T*>(p.out);
   const int tid = threadIdx.x;
-  if (tid < G1) {
-    const int head = tid < p.g ? h * p.g + tid : n_S + h;
+  auto head_of = [&](int r) { const int u = r % G1; return u < p.g ? h * p.g + u : n_S + h; };
+  // split weights: exp2(m_s - M) / sum_s exp2(m_s - M) l_s
+  for (int r = tid; r < R; r += blockDim.x) {
+    const int b = b0 + r / G1, head = head_of(r);
     float M = -INFINITY;
-    for (int s = 0; s < p.n_splits; ++s)
-      M = fmaxf(M, p.part_ml[(((long)b * p.n_splits + s) * H_q + head) * 2]);
+    for (int s = 0; s < NS; ++s) M = fmaxf(M, p.part_ml[(((long)b * NS + s) * H_q + head) * 2]);
     float den = 0.f;
-    for (int s = 0; s < p.n_splits; ++s) {
-      const float* ml = p.part_ml + (((long)b * p.n_splits + s) * H_q + head) * 2;
+    for (int s = 0; s < NS; ++s) {
+      const float* ml = p.part_ml + (((long)b * NS + s) * H_q + head) * 2;
       const float wv = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
-      wgt[tid * p.n_splits + s] = wv;
+      wgt[r * NS + s] = wv;
       den += wv * ml[1];
     }
-    for (int s = 0; s < p.n_splits; ++s) wgt[tid * p.n_splits + s] /= den;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int s = 0; s < NS; ++s) wgt[r * NS + s] *= inv;
   }
   __syncthreads();
-  for (int e = tid; e < G1 * d_c; e += 256) {
-    const int u = e / d_c, c = e % d_c;
-    const int head = u < p.g ? h * p.g + u : n_S + h;
+  for (int e = tid; e < R * d_c; e += blockDim.x) {
+    const int r = e / d_c, c = e % d_c;
+    const int b = b0 + r / G1, head = head_of(r);
     float a = 0.f;
-    for (int s = 0; s < p.n_splits; ++s)
-      a = fmaf(wgt[u * p.n_splits + s], p.part_o[(((long)b * p.n_splits + s) * H_q + head) * d_c + c], a);
+    for (int s = 0; s < NS; ++s) a = fmaf(wgt[r * NS + s], p.part_o[(((long)b * NS + s) * H_q + head) * d_c + c], a);
     olat[e] = a;
   }
   __syncthreads();
-  for (int e = tid; e < G1 * DV; e += 256) {
-    const int u = e / DV, n = e % DV;
+  // hv[r][n] = sum_c olat[r][c] W_UV[c][n]: thread column n, rows rg, rg+RG, ...
+  const int RG = blockDim.x / DV;
+  const int n = tid % DV, rg = tid / DV;
+  if (rg < RG) {
+    float acc[MAX_ROWS];
+#pragma unroll
+    for (int i = 0; i < MAX_ROWS; ++i) acc[i] = 0.f;
     const T* wc = w + (long)h * (p.d_nope + DV) + p.d_nope + n;
-    float a = 0.f;
-    for (int c = 0; c < d_c; ++c) a = fmaf(olat[u * d_c + c], to_f(wc[(long)c * ncol]), a);
-    hv[e] = a;
+    for (int c = 0; c < d_c; ++c) {
+      const float wv = to_f(wc[(long)c * ncol]);
+#pragma unroll
+      for (int i = 0; i < MAX_ROWS; ++i) {
+        const int r = rg + i * RG;
+        if (r < R) acc[i] = fmaf(olat[r * d_c + c], wv, acc[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < MAX_ROWS; ++i) {
+      const int r = rg + i * RG;
+      if (r < R) hv[r * DV + n] = acc[i];
+    }
   }
   __syncthreads();
-  for (int e = tid; e < p.g * DV; e += 256) {
-    const int u = e / DV, n = e % DV;
-    const int sh = h * p.g + u;
+  for (int e = tid; e < nb * p.g * DV; e += blockDim.x) {
+    const int bl = e / (p.g * DV), u = (e / DV) % p.g, nn = e % DV;
+    const int b = b0 + bl, sh = h * p.g + u;
     const float lam = sigmoidf_(p.lam[(long)b * n_S + sh]);
-    const long idx = ((long)b * n_S + sh) * DV + n;
-    const float d = hv[u * DV + n] - lam * hv[p.g * DV + n];
+    const long idx = ((long)b * n_S + sh) * DV + nn;
+    const float d = hv[(bl * G1 + u) * DV + nn] - lam * hv[(bl * G1 + p.g) * DV + nn];
     out[idx] = from_f<T>(sigmoidf_(to_f(gate[idx])) * d);
   }
 }
 
 cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
-  dim3 grid((unsigned)p.n_kv, (unsigned)p.B);
-  const size_t smem = sizeof(float) * (size_t)(p.g + 1) * p.d_nope;
+  dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + SEQ_PER_BLOCK - 1) / SEQ_PER_BLOCK));
+  const size_t smem = sizeof(float) * (size_t)SEQ_PER_BLOCK * (p.g + 1) * p.d_nope;
   if (dt == GDLA_BF16)
     decode_absorb_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(p);
   else
@@ -281,17 +312,18 @@ cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaS
 }
 
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
-  const int G1 = p.g + 1;
-  const size_t smem = sizeof(float) * ((size_t)G1 * p.d_c + (size_t)G1 * p.d_v + (size_t)G1 * p.n_splits);
-  dim3 grid((unsigned)p.n_kv, (unsigned)p.B);
+  const int R = SEQ_PER_BLOCK * (p.g + 1);
+  const size_t smem = sizeof(float) * ((size_t)R * p.d_c + (size_t)R * p.d_v + (size_t)R * p.n_splits);
+  dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + SEQ_PER_BLOCK - 1) / SEQ_PER_BLOCK));
+  cudaError_t e;
   if (dt == GDLA_BF16) {
     auto k = decode_combine_kernel<__nv_bfloat16>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<grid, 256, smem, s>>>(p);
   } else {
     auto k = decode_combine_kernel<float>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<grid, 256, smem, s>>>(p);
   }

@@ -1,0 +1,422 @@
+// decode_tc.cu -- split-KV GDLA decode over the compact latent cache on the
+// 5th-generation tensor cores ("Motif 3: Technical Report", Architecture: GDLA
+// keeps MLA's compact inference state; the cache row of a token is the
+// normalised latent c_hat (d_c = 512) plus the rotated rotary key (d_R = 64)).
+//
+// With W_UK absorbed into the query (q_abs = W_UK q_nope, done beforehand by
+// decode_absorb) one sequence's attention over a tile of cache rows is two
+// small GEMMs in which the cache tile is the big operand:
+//   S^T[tokens x heads] = C[tokens x 576] . Qcat^T[576 x heads]      (M = 64 tokens)
+//   O^T[512 x heads]   += C[:, :512]^T[512 x tokens] . P^T[tokens x heads]  (M = 4 x 128 dims)
+// so the cache is streamed from HBM once, the same shared-memory tile feeds
+// both MMAs (K-major for the first, MN-major for the second), and no head
+// padding is needed (N = number of query heads, a multiple of 16).
+//
+// Block (split s, sequence b), 256 threads:
+//   warp 0      TMA producer: 64-token cache tiles (9 boxes: 8 latent + 1 rotary) in a 2-stage ring;
+//   warp 1      MMA issuer (one lane);
+//   warps 4-7   softmax over S^T (one token per thread, lanes 0-15 of each warp,
+//               the M = 64 accumulator layout), then the split's partial output.
+// The running maximum of each head is CTA-uniform and lives in registers; O is
+// rescaled (in TMEM) only when some head's maximum grows by more than 2^8.
+#include <math.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace gdla {
+namespace {
+
+constexpr int TT = 64;               // tokens per tile
+constexpr int DC = 512, DRD = 64;    // latent, rotary widths
+constexpr int NBOX = (DC + DRD) / 64;  // 9 boxes of 64 columns
+constexpr int NPMAX = 48;            // padded heads (N of both MMAs)
+constexpr int TILE_BYTES = TT * (DC + DRD) * 2;  // 72 KB
+constexpr int QT_BYTES = NPMAX * (DC + DRD) * 2;  // 54 KB
+constexpr int PT_BYTES = NPMAX * TT * 2;          // 6 KB
+constexpr int DSTAGES = 2;
+constexpr int DSMEM = QT_BYTES + DSTAGES * TILE_BYTES + 2 * PT_BYTES + 1024;
+constexpr int DTHREADS = 256;
+constexpr float kThr = 8.0f;
+constexpr uint32_t COL_ST = 0;     // S^T buffers at [0, 64) and [64, 128)
+constexpr uint32_t COL_OT = 128;   // O^T M-tile mt at 128 + 64 mt
+
+struct DBars {
+  uint64_t full[DSTAGES], empty[DSTAGES], s_full[2], p_full[2], p_free[2], o_done, sync, mma_done;
+};
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+}  // namespace
+
+struct DecodeTcArgs {
+  int B, T_max, n_splits, split_len, sliding, window, H_q, NP;
+  const int* seqlens;
+  const float* q_abs;   // [B, H_q, 512]
+  const float* q_rot;   // [B, H_q, 64]
+  float sl2;
+  float* part_o;        // [B, n_splits, H_q, 512]
+  float* part_ml;       // [B, n_splits, H_q, 2]
+  int* status;
+};
+
+__global__ void __launch_bounds__(DTHREADS, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
+                     const DecodeTcArgs a) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qt = smem;                                   // Qcat^T, 9 boxes of [NP x 128 B]
+  uint8_t* tiles = smem + QT_BYTES;                     // stages, 9 boxes of [64 x 128 B]
+  uint8_t* pt = tiles + DSTAGES * TILE_BYTES;           // P^T double buffer [NP x 128 B]
+  __shared__ __align__(8) DBars bars;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int flag[3];
+  __shared__ float wmax[4][NPMAX];
+  __shared__ float lsum[NPMAX];
+  __shared__ float alpha_s[NPMAX];
+  __shared__ volatile int abort_flag;
+
+  if (sm100::earlier_failure(a.status)) return;  // an earlier CTA of this call timed out
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = blockIdx.x, b = blockIdx.y;
+  const int H_q = a.H_q, NP = a.NP;
+  const int Tb = a.seqlens[b];
+  const int lo = a.sliding ? max(0, Tb - a.window) : 0;
+  const int t0 = max(lo, s * a.split_len), t1 = min(Tb, (s + 1) * a.split_len);
+  const int jt0 = (t0 / TT) * TT;
+  const int n_tiles = (t1 > t0) ? (t1 - jt0 + TT - 1) / TT : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < DSTAGES; ++i) {
+      mbar_init(smem_u32(&bars.full[i]), 1);
+      mbar_init(smem_u32(&bars.empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars.s_full[i]), 1);
+      mbar_init(smem_u32(&bars.p_full[i]), 128);
+      mbar_init(smem_u32(&bars.p_free[i]), 1);
+    }
+    mbar_init(smem_u32(&bars.o_done), 1);
+    mbar_init(smem_u32(&bars.sync), 128);
+    mbar_init(smem_u32(&bars.mma_done), 1);
+    fence_mbar_init();
+    flag[0] = flag[1] = flag[2] = 0;
+    abort_flag = 0;
+    prefetch_tmap(&tmC);
+    prefetch_tmap(&tmR);
+  }
+  // Qcat^T in bf16, pre-scaled by tau*log2(e), K-major with the 128-byte swizzle; zero P^T
+  for (int e = threadIdx.x; e < NP * NBOX * 8; e += DTHREADS) {
+    const int h = e / (NBOX * 8), rem = e % (NBOX * 8), bx = rem / 8, c = rem % 8;  // 16-byte chunk
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float v0 = 0.f, v1 = 0.f;
+      if (h < H_q) {
+        const int d = bx * 64 + c * 8 + 2 * u;
+        if (d < DC) {
+          const float* src = a.q_abs + ((long)b * H_q + h) * DC + d;
+          v0 = src[0] * a.sl2;
+          v1 = src[1] * a.sl2;
+        } else {
+          const float* src = a.q_rot + ((long)b * H_q + h) * DRD + (d - DC);
+          v0 = src[0] * a.sl2;
+          v1 = src[1] * a.sl2;
+        }
+      }
+      w[u] = pack_bf16x2(v0, v1);
+    }
+    *reinterpret_cast<uint4*>(qt + bx * (NP * 128) + h * 128 + ((c ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  for (int e = threadIdx.x; e < 2 * PT_BYTES / 16; e += DTHREADS)
+    reinterpret_cast<uint4*>(pt)[e] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int k = 0;
+      for (; k < n_tiles && !abort_flag; ++k) {
+        const int st = k % DSTAGES;
+        if (k >= DSTAGES && !mbar_wait(smem_u32(&bars.empty[st]), ((k / DSTAGES) & 1) ^ 1, a.status, 301, &abort_flag)) {
+          abort_flag = 1;
+          break;
+        }
+        const uint32_t bar = smem_u32(&bars.full[st]);
+        const uint32_t dst = smem_u32(tiles + st * TILE_BYTES);
+        const int j0 = jt0 + k * TT;
+        mbar_expect_tx(bar, TILE_BYTES);
+        for (int bx = 0; bx < NBOX - 1; ++bx) tma_load_3d(dst + bx * (TT * 128), &tmC, bar, bx * 64, j0, b);
+        tma_load_3d(dst + (NBOX - 1) * (TT * 128), &tmR, bar, 0, j0, b);
+      }
+      if (abort_flag)
+        for (int q = (k > DSTAGES ? k - DSTAGES : 0); q < k; ++q)
+          mbar_wait(smem_u32(&bars.full[q % DSTAGES]), (q / DSTAGES) & 1, nullptr, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id1 = idesc_bf16_f32(64, NP, false, false);
+      const uint32_t id2 = idesc_bf16_f32(128, NP, true, false);
+      bool ok = true;
+      const uint32_t qbase = smem_u32(qt);
+      auto mma2 = [&](int k) {
+        // O^T += C^T . P^T for tile k (all four 128-dim M-tiles)
+        const uint32_t cb = smem_u32(tiles + (k % DSTAGES) * TILE_BYTES);
+        const uint32_t pb = smem_u32(pt + (k & 1) * PT_BYTES);
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+          for (int kk = 0; kk < TT / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(cb + 2 * mt * (TT * 128) + kk * 2048, TT * 128, 1024);
+            const uint64_t bd = sdesc_sw128(pb + kk * 32, 16, 1024);
+            mma_ss(tmem + COL_OT + 64 * mt, ad, bd, id2, (k > 0 || kk > 0) ? 1u : 0u);
+          }
+        // p_free[k & 1] completes once per odd/even tile: it says both that P^T buffer
+        // k & 1 may be rewritten and that O^T holds every tile up to k
+        mma_commit(smem_u32(&bars.empty[k % DSTAGES]));
+        mma_commit(smem_u32(&bars.p_free[k & 1]));
+      };
+      for (int k = 0; k < n_tiles && ok; ++k) {
+        ok = mbar_wait(smem_u32(&bars.full[k % DSTAGES]), (k / DSTAGES) & 1, a.status, 311, &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t cb = smem_u32(tiles + (k % DSTAGES) * TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < NBOX * 4; ++kk) {
+          const uint64_t ad = sdesc_sw128(cb + (kk >> 2) * (TT * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(qbase + (kk >> 2) * (NP * 128) + (kk & 3) * 32, 16, 1024);
+          mma_ss(tmem + COL_ST + 64 * (k & 1), ad, bd, id1, kk > 0);
+        }
+        mma_commit(smem_u32(&bars.s_full[k & 1]));
+        if (k > 0) {
+          ok = mbar_wait(smem_u32(&bars.p_full[(k - 1) & 1]), ((k - 1) >> 1) & 1, a.status, 312, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          mma2(k - 1);
+        }
+      }
+      if (ok && n_tiles > 0) {
+        ok = mbar_wait(smem_u32(&bars.p_full[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, a.status, 313, &abort_flag);
+        if (ok) {
+          tc_fence_after();
+          mma2(n_tiles - 1);
+        }
+      }
+      mma_commit(smem_u32(&bars.o_done));
+      if (!ok) abort_flag = 1;
+      mma_commit(smem_u32(&bars.mma_done));
+      mbar_wait(smem_u32(&bars.mma_done), 0, nullptr, 314);
+    }
+  } else if (warp >= 4) {
+    const int q4 = warp & 3;
+    const bool rowl = lane < 16;
+    const int tok_local = q4 * 16 + (lane & 15);
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    float m_ref[NPMAX], lp[NPMAX];
+#pragma unroll
+    for (int h = 0; h < NPMAX; ++h) {
+      m_ref[h] = -INFINITY;
+      lp[h] = 0.f;
+    }
+    uint32_t sync_ph = 0;
+    bool ok = true;
+    auto block_sync = [&]() -> bool {
+      mbar_arrive(smem_u32(&bars.sync));
+      const bool r = mbar_wait(smem_u32(&bars.sync), sync_ph & 1, a.status, 321, &abort_flag);
+      ++sync_ph;
+      return __all_sync(0xffffffffu, r);
+    };
+    for (int k = 0; k < n_tiles; ++k) {
+      ok = mbar_wait(smem_u32(&bars.s_full[k & 1]), (k >> 1) & 1, a.status, 322, &abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      if (k >= 2) {
+        // P^T buffer k & 1 and O^T up to tile k-2 are free/settled (MMA of tile k-2 done)
+        ok = mbar_wait(smem_u32(&bars.p_free[k & 1]), ((k >> 1) & 1) ^ 1, a.status, 324, &abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+      }
+      tc_fence_after();
+      float x[NPMAX];
+      tmem_ld32(tmem + lane_base + COL_ST + 64 * (k & 1), *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+      tmem_ld16(tmem + lane_base + COL_ST + 64 * (k & 1) + 32, *reinterpret_cast<uint32_t(*)[16]>(&x[32]));
+      tmem_wait_ld();
+      const int j = jt0 + k * TT + tok_local;
+      const bool valid = rowl && j >= t0 && j < t1;
+      bool exceed = false;
+#pragma unroll
+      for (int h = 0; h < NPMAX; ++h) {
+        x[h] = (valid && h < H_q) ? x[h] : -INFINITY;
+        exceed |= x[h] > m_ref[h] + kThr || (m_ref[h] == -INFINITY && x[h] > -INFINITY);
+      }
+      if (__any_sync(0xffffffffu, exceed) && lane == 0) atomicOr(&flag[k % 3], 1);
+      if (!(ok = block_sync())) break;
+      if (threadIdx.x == 128) flag[(k + 2) % 3] = 0;
+      if (flag[k % 3]) {
+        // some head's maximum grew: CTA-wide per-head max of this tile
+#pragma unroll
+        for (int h = 0; h < NPMAX; ++h) {
+          float v = x[h];
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+          if (lane == 0) wmax[q4][h] = v;
+        }
+        if (!(ok = block_sync())) break;
+        bool any_resc = false;
+#pragma unroll
+        for (int h = 0; h < NPMAX; ++h) {
+          const float tm = fmaxf(fmaxf(wmax[0][h], wmax[1][h]), fmaxf(wmax[2][h], wmax[3][h]));
+          const bool up = tm > m_ref[h] + kThr || (m_ref[h] == -INFINITY && tm > -INFINITY);
+          const float mn = up ? fmaxf(m_ref[h], tm) : m_ref[h];
+          const float al = (!up || m_ref[h] == -INFINITY) ? (up ? 0.f : 1.f) : ex2f(m_ref[h] - mn);
+          any_resc |= up && m_ref[h] != -INFINITY;
+          lp[h] *= al;
+          m_ref[h] = mn;
+          if ((int)threadIdx.x - 128 == h) alpha_s[h] = al;
+        }
+        if (k > 0 && any_resc) {
+          if (!(ok = block_sync())) break;  // alpha_s visible to every thread
+          // O^T holds tiles < k once the MMA of tile k-1 has landed (p_free of its parity)
+          ok = mbar_wait(smem_u32(&bars.p_free[(k - 1) & 1]), ((k - 1) >> 1) & 1, a.status, 323, &abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int mt = 0; mt < 4; ++mt) {
+            uint32_t o[NPMAX];
+            const uint32_t ta = tmem + lane_base + COL_OT + 64 * mt;
+            tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+            tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < NPMAX; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha_s[h]);
+            tmem_st32(ta, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+            tmem_st16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
+          }
+          tmem_wait_st();
+        }
+      }
+      // P^T tile k (bf16): row h = head, 64 tokens, 128-byte swizzle
+      uint8_t* pb = pt + (k & 1) * PT_BYTES;
+      if (rowl) {
+#pragma unroll
+        for (int h = 0; h < NPMAX; ++h) {
+          const float p = (h < H_q) ? ex2f(x[h] - (m_ref[h] == -INFINITY ? 0.f : m_ref[h])) : 0.f;
+          lp[h] += p;
+          if (h < NP) {
+            const int c = tok_local >> 3;
+            *reinterpret_cast<__nv_bfloat16*>(pb + h * 128 + ((c ^ (h & 7)) << 4) + (tok_local & 7) * 2) =
+                __float2bfloat16_rn(p);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars.p_full[k & 1]));
+    }
+    // ---- partial results of this split: (m, l) per head and O^T
+    if (ok) {
+      ok = mbar_wait(smem_u32(&bars.o_done), 0, a.status, 325, &abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      if (threadIdx.x < 128 + NPMAX) lsum[threadIdx.x - 128] = 0.f;
+      ok = block_sync();
+    }
+    if (ok) {
+#pragma unroll
+      for (int h = 0; h < NPMAX; ++h) {
+        float v = rowl ? lp[h] : 0.f;
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        if (lane == 0 && h < H_q) atomicAdd(&lsum[h], v);
+      }
+      ok = block_sync();
+    }
+    const long base = ((long)b * a.n_splits + s) * H_q;
+    if (ok) {
+#pragma unroll
+      for (int h = 0; h < NPMAX; ++h)
+        if ((int)threadIdx.x - 128 == h && h < H_q) {
+          a.part_ml[(base + h) * 2 + 0] = m_ref[h];
+          a.part_ml[(base + h) * 2 + 1] = lsum[h];
+        }
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t o[NPMAX];
+        const uint32_t ta = tmem + lane_base + COL_OT + 64 * mt;
+        tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+        tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
+        tmem_wait_ld();
+        const int dim = mt * 128 + q4 * 32 + lane;
+#pragma unroll
+        for (int h = 0; h < NPMAX; ++h)
+          if (h < H_q) a.part_o[(base + h) * DC + dim] = n_tiles > 0 ? __uint_as_float(o[h]) : 0.f;
+      }
+    } else {
+      abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+bool decode_tc_supported(const DecodeParams& p, gdla_dtype dt) {
+  const int H_q = p.n_kv * (p.g + 1);
+  return dt == GDLA_BF16 && p.d_c == DC && p.d_rope == DRD && H_q <= NPMAX && p.split_len % TT == 0 &&
+         get_encode_tiled() != nullptr;
+}
+
+cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s) {
+  const int H_q = p.n_kv * (p.g + 1);
+  CUtensorMap tc, tr;
+  {
+    const uint64_t dims[3] = {(uint64_t)DC, (uint64_t)p.T_max, (uint64_t)p.B};
+    const uint64_t str[2] = {(uint64_t)DC * 2, (uint64_t)p.T_max * DC * 2};
+    const uint32_t box[3] = {64, TT, 1};
+    if (!make_tmap_bf16(&tc, p.c_cache, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)DRD, (uint64_t)p.T_max, (uint64_t)p.B};
+    const uint64_t str[2] = {(uint64_t)DRD * 2, (uint64_t)p.T_max * DRD * 2};
+    const uint32_t box[3] = {64, TT, 1};
+    if (!make_tmap_bf16(&tr, p.kr_cache, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  DecodeTcArgs a{};
+  a.B = p.B; a.T_max = p.T_max; a.n_splits = p.n_splits; a.split_len = p.split_len;
+  a.sliding = p.sliding; a.window = p.window; a.H_q = H_q; a.NP = NPMAX;
+  a.seqlens = p.seqlens; a.q_abs = p.q_abs; a.q_rot = p.q_rot; a.sl2 = p.scale * kLog2e;
+  a.part_o = p.part_o; a.part_ml = p.part_ml; a.status = p.status;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<<<dim3((unsigned)p.n_splits, (unsigned)p.B), DTHREADS, DSMEM, s>>>(tc, tr, a);
+  return cudaGetLastError();
+}
+
+}  // namespace gdla

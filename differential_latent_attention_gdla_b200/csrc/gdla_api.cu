@@ -64,13 +64,23 @@ struct DecodeLayout {
 DecodeLayout decode_layout(const gdla_decode_args* a) {
   DecodeLayout l;
   const int H_q = a->n_kv * (a->g + 1);
-  const int tile = 128;
-  const int max_splits = (a->T_max + tile - 1) / tile;
-  int n = (2 * kNumSMs + a->B - 1) / a->B;
-  if (n > max_splits) n = max_splits;
-  if (n < 1) n = 1;
-  int len = (a->T_max + n - 1) / n;
-  len = (len + tile - 1) / tile * tile;
+  // split the cache of every sequence into n chunks (multiples of 64 tokens) so
+  // that B*n blocks fill whole waves of one block per SM: minimise
+  // waves(B*n) * tiles_per_split(n), with a mild penalty for more partials
+  const int tile = 64;
+  const int tiles = (a->T_max + tile - 1) / tile;
+  int best_n = 1;
+  double best = 1e300;
+  for (int n = 1; n <= tiles && n <= 256; ++n) {
+    const long waves = ((long)a->B * n + kNumSMs - 1) / kNumSMs;
+    const long per = (tiles + n - 1) / n;
+    const double cost = (double)waves * per * (1.0 + 0.002 * n);
+    if (cost < best) {
+      best = cost;
+      best_n = n;
+    }
+  }
+  const int len = ((tiles + best_n - 1) / best_n) * tile;
   l.split_len = len;
   l.n_splits = (a->T_max + len - 1) / len;
   size_t off = 0;
@@ -268,7 +278,8 @@ gdla_status gdla_decode(const gdla_decode_args* a, void* stream) {
   p.status = (int*)(ws + lay.status);
   cudaError_t e = cudaMemsetAsync(p.status, 0, kStatusBytes, s);
   if (e == cudaSuccess) e = launch_decode_absorb(p, a->dtype, s);
-  if (e == cudaSuccess) e = launch_decode_split_simt(p, a->dtype, s);
+  if (e == cudaSuccess)
+    e = decode_tc_supported(p, a->dtype) ? launch_decode_split_tc(p, s) : launch_decode_split_simt(p, a->dtype, s);
   if (e == cudaSuccess) e = launch_decode_combine(p, a->dtype, s);
   return cuda_status(e);
 }

@@ -68,5 +68,8 @@ struct DecodeParams {
 cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
 cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
+// tcgen05/TMA split-KV pass (bf16, d_c = 512, d_rope = 64, at most 48 query heads).
+bool decode_tc_supported(const DecodeParams& p, gdla_dtype dt);
+cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
 
 }  // namespace gdla

@@ -46,22 +46,34 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Bounded wait: gives up after ~`limit_ns` of wall time, records GDLA_ERR_TIMEOUT
-// and the caller's tag in the workspace status word (if any) and returns false.
-constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far beyond any legal wait
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, int* status, int tag) {
+// Bounded wait: gives up after ~kWaitLimitNs of wall time, or as soon as the
+// CTA's abort flag or the workspace status word is set by another waiter;
+// records GDLA_ERR_TIMEOUT and the caller's tag in the status word (if any) and
+// returns false.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legal wait
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, int* status, int tag,
+                                          const volatile int* abort = nullptr) {
   if (mbar_try_wait(bar, phase)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, phase)) return true;
-    if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitLimitNs) {
-      if (status) {
-        atomicCAS(status, 0, (int)GDLA_ERR_TIMEOUT);
-        atomicCAS(status + 1, 0, tag);
+    if ((it & 255u) == 255u) {
+      const bool gave_up = globaltimer_ns() - t0 > kWaitLimitNs;
+      const bool other = (abort && *abort) || (status && *reinterpret_cast<volatile int*>(status));
+      if (gave_up || other) {
+        if (status && gave_up) {
+          atomicCAS(status, 0, (int)GDLA_ERR_TIMEOUT);
+          atomicCAS(status + 1, 0, tag);
+        }
+        return false;
       }
-      return false;
     }
   }
+}
+
+// A CTA that starts after another one recorded a failure does no work.
+__device__ __forceinline__ bool earlier_failure(const int* status) {
+  return status && *reinterpret_cast<const volatile int*>(status) != 0;
 }
 
 // ---------------------------------------------------------------------- TMA

@@ -19,8 +19,7 @@ order):
     near-uniform attention);
   * lambda logits and gate logits: N(0,1).
 The decode cache holds the normalised latent and the rotated rotary key, which
-are drawn directly: c_hat ~ gamma-free N(0,1)/sqrt(576)*sqrt(576/d_c)... see
-``make_decode_inputs``.
+are drawn directly (see ``make_decode_inputs``).
 """
 from __future__ import annotations
 
@@ -133,6 +132,8 @@ PREFILL = {
 }
 DECODE = {
     "b64_t32k": DecodeShape("bf16 decode, B=64, 32768-token latent cache, g=2", B=64, T=32768, g=2),
+    # a quarter-size case for profiler captures (0.6 GB of cache, still far above L2)
+    "b16_t32k": DecodeShape("bf16 decode, B=16, 32768-token latent cache, g=2", B=16, T=32768, g=2),
 }
 
 

@@ -68,8 +68,12 @@ def oracle_decode(inp: dict, *, g: int, d_nope: int, d_v: int, seqs=None, kv_sel
     return np.stack(outs)
 
 
-def assert_parity(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = ""):
-    """The acceptance bar (see the module docstring)."""
+def assert_parity(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: str = "", elementwise: bool = True):
+    """The acceptance bar (see the module docstring). ``elementwise=False``
+    keeps only the RMS bar: for deliberately extreme logits, where a bf16
+    operand of the score moves the exponent by |s| * 2^-9, a single element can
+    legitimately move by more than the element bound while the RMS bar still
+    catches any logic error."""
     sel = ~np.isnan(ref)
     got, ref = got[sel], ref[sel]
     assert np.isfinite(got).all(), f"{what}: non-finite output"
@@ -79,5 +83,6 @@ def assert_parity(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype, what: st
         return err
     rel_rms, rel_elem = bf16_errors(got, ref)
     assert rel_rms <= BF16_REL_RMS, f"{what}: rms err / rms = {rel_rms:.3e} > {BF16_REL_RMS}"
-    assert rel_elem <= BF16_ELEM_RMS, f"{what}: max(|e| - 2^-6|ref|) / rms = {rel_elem:.3e} > {BF16_ELEM_RMS}"
+    if elementwise:
+        assert rel_elem <= BF16_ELEM_RMS, f"{what}: max(|e| - 2^-6|ref|) / rms = {rel_elem:.3e} > {BF16_ELEM_RMS}"
     return rel_rms

@@ -94,15 +94,20 @@ def test_prefill_full_size_sampled_rows(name):
 
 def test_prefill_lambda_one_identical_queries_cancel():
     """Signal queries equal to their noise head's query with lambda -> 1 give
-    D = 0: the kernel's output must vanish to rounding level."""
+    D = 0. On the GPU the noise head's output is held in bf16 for the
+    epilogue, so each element may keep a residual of half a bf16 ulp of H:
+    |Y(lambda=1)| <= 2^-8 |Y(lambda=0)| element by element (Y(lambda=0) =
+    sigmoid(G) H_S with H_S = H_N here)."""
     shape = wl.PrefillShape("cancel", B=1, L=256, n_kv=2, g=3)
     inp = wl.make_prefill_inputs(shape, seed=5, device=DEV)
     for i in range(shape.n_S):
         inp["q"][:, :, i] = inp["q"][:, :, shape.n_S + i // shape.g]
     inp["lam_logits"].fill_(30.0)
-    y = run_prefill(shape, inp)
-    ref_scale = float(f64(run_prefill(shape, dict(inp, lam_logits=torch.full_like(inp["lam_logits"], -30.0)))).std())
-    assert float(y.float().abs().max()) <= 1e-2 * ref_scale
+    y1 = f64(run_prefill(shape, inp))
+    y0 = f64(run_prefill(shape, dict(inp, lam_logits=torch.full_like(inp["lam_logits"], -30.0))))
+    rms0 = float(np.sqrt((y0 ** 2).mean()))
+    assert float((np.abs(y1) - 2.0 ** -8 * np.abs(y0)).max()) <= 1e-3 * rms0
+    assert float(np.sqrt((y1 ** 2).mean())) <= 2e-3 * rms0
 
 
 def test_prefill_emits_decode_cache_and_decode_matches_last_row():
@@ -163,3 +168,21 @@ def test_binding_raises_on_invalid_arguments():
     inp = wl.make_prefill_inputs(shape, seed=1, device=DEV)
     with pytest.raises(gdla.GdlaError):
         run_prefill(shape, inp)
+
+
+@pytest.mark.parametrize("scale", [20.0, 30.0])
+def test_decode_peaked_softmax_rescale_path(scale):
+    """Very peaked attention (q scaled up) makes the running maximum of many
+    heads jump across tiles, which exercises the O-rescale path."""
+    shape = wl.DecodeShape("decode peaked", B=3, T=2000, n_kv=16, g=2)
+    inp = wl.make_decode_inputs(shape, seed=12, device=DEV, act="unit", seqlens=[2000, 1333, 700])
+    inp["q"] = (inp["q"].float() * scale).to(torch.bfloat16)
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g)
+    torch.cuda.synchronize()
+    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
+    # logits reach |s| ~ 50-150 here: the bf16 absorbed query moves single
+    # exponents by ~|s| 2^-9, so only the RMS bar applies (a wrong rescale
+    # would be an O(1) error)
+    assert_parity(f64(y), ref, torch.bfloat16, f"decode peaked x{scale}", elementwise=False)
