@@ -368,8 +368,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             const int j = key0 + c;
-            const bool vis = j <= i && (!a.sliding || j > i - a.window);
-            if (!vis) sr[c] = __float_as_uint(-INFINITY);
+            // bitwise operators: a select per element, no branches
+            const bool vis = (j <= i) & ((a.sliding == 0) | (j > i - a.window));
+            sr[c] = vis ? sr[c] : __float_as_uint(-INFINITY);
           }
         }
         float mr = -INFINITY;

@@ -8,8 +8,8 @@
 //   sum_j p_j (c_hat_j W_UV) = (sum_j p_j c_hat_j) W_UV (latent weighted sum)
 // Kernels: decode_absorb (q_abs = W_UK q_nope, RoPE of q_rope at position
 // seqlen-1), decode_split (split-KV online softmax over the cache, partial
-// results per split), decode_combine (log-sum-exp merge, W_UV, differential
-// and gate epilogue).
+// results per split), decode_merge (log-sum-exp merge of the splits) and
+// decode_combine (W_UV, differential and gate epilogue).
 #include <math.h>
 
 #include "common.cuh"
@@ -17,54 +17,64 @@
 
 namespace gdla {
 
-// Sequences per block of the absorb and combine kernels: one W_UK / W_UV slice
-// of a KV group is read once per block and reused for SEQ_PER_BLOCK sequences.
-constexpr int SEQ_PER_BLOCK = 4;
-constexpr int MAX_ROWS = SEQ_PER_BLOCK * 9;  // (g+1) <= 9 heads per KV group
+// Rows per combine block: max(1, 12 / (g+1)) sequences times the g+1 heads of
+// a KV group; one W_UV slice is staged once per block for all of them.
+constexpr int MAX_ROWS = 12;  // rows (sequence, head of the group) per combine block
+// Absorb blocks: KV group x 64 latent rows x ABS_SEQ sequences.
+constexpr int ABS_ROWS = 64;
+constexpr int ABS_SEQ = 16;
 
 // q_abs[b, head, c] = sum_n W_UKV[c, h*(d_nope+d_v) + n] * q_nope[b, head, n] for the
 // g+1 heads of KV group h, and RoPE of their rotary parts at position seqlen-1.
-// Block (KV group h, chunk of sequences); each thread owns latent rows c.
+// Block (KV group h, 64 latent rows, up to 16 sequences): the W_UK rows and the
+// query rows are staged in shared memory with coalesced loads, then every
+// thread computes (latent row, query row) dot products from shared memory.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
-  const int h = blockIdx.x, b0 = blockIdx.y * SEQ_PER_BLOCK;
-  const int nb = min(SEQ_PER_BLOCK, p.B - b0);
+  const int h = blockIdx.x, c0 = blockIdx.y * ABS_ROWS, b0 = blockIdx.z * ABS_SEQ;
+  const int nb = min(ABS_SEQ, p.B - b0);
   const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1;
   const int dqk = p.d_nope + p.d_rope, ncol = p.n_kv * (p.d_nope + p.d_v), DN = p.d_nope;
+  const int DNP = DN + 1;  // padded row (bank-conflict free column reads)
+  const int nrows = min(ABS_ROWS, p.d_c - c0);
   const T* q = reinterpret_cast<const T*>(p.q);
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
-  extern __shared__ float qn[];  // [R][d_nope]
-  for (int e = threadIdx.x; e < R * DN; e += blockDim.x) {
-    const int r = e / DN, k = e % DN, bl = r / G1, u = r % G1;
+  extern __shared__ float sm[];
+  float* ws = sm;                   // [ABS_ROWS][DNP]
+  float* qs = ws + ABS_ROWS * DNP;  // [R][DN]
+  constexpr int VEC = 16 / (int)sizeof(T);  // elements per 16-byte load
+  const int vrow = DN / VEC;
+#pragma unroll 4
+  for (int e = threadIdx.x; e < nrows * vrow; e += blockDim.x) {
+    const int cr = e / vrow, v = e % vrow;
+    const uint4 x = *reinterpret_cast<const uint4*>(w + (long)(c0 + cr) * ncol + (long)h * (p.d_nope + p.d_v) + v * VEC);
+    const T* xe = reinterpret_cast<const T*>(&x);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) ws[cr * DNP + v * VEC + i] = to_f(xe[i]);
+  }
+#pragma unroll 4
+  for (int e = threadIdx.x; e < R * vrow; e += blockDim.x) {
+    const int r = e / vrow, v = e % vrow, bl = r / G1, u = r % G1;
     const int head = u < p.g ? h * p.g + u : n_S + h;
-    qn[e] = to_f(q[((long)(b0 + bl) * H_q + head) * dqk + k]);
+    const uint4 x = *reinterpret_cast<const uint4*>(q + ((long)(b0 + bl) * H_q + head) * dqk + v * VEC);
+    const T* xe = reinterpret_cast<const T*>(&x);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) qs[r * DN + v * VEC + i] = to_f(xe[i]);
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < p.d_c; c += blockDim.x) {
-    const T* wr = w + (long)c * ncol + (long)h * (p.d_nope + p.d_v);
-    float acc[MAX_ROWS];
-#pragma unroll
-    for (int r = 0; r < MAX_ROWS; ++r) acc[r] = 0.f;
-    for (int k = 0; k < DN; k += 4) {
-      const float w0 = to_f(wr[k]), w1 = to_f(wr[k + 1]), w2 = to_f(wr[k + 2]), w3 = to_f(wr[k + 3]);
-#pragma unroll
-      for (int r = 0; r < MAX_ROWS; ++r) {
-        if (r < R) {
-          const float* qr = qn + r * DN + k;
-          acc[r] = fmaf(w0, qr[0], fmaf(w1, qr[1], fmaf(w2, qr[2], fmaf(w3, qr[3], acc[r]))));
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < MAX_ROWS; ++r) {
-      if (r < R) {
-        const int bl = r / G1, u = r % G1;
-        const int head = u < p.g ? h * p.g + u : n_S + h;
-        p.q_abs[((long)(b0 + bl) * H_q + head) * p.d_c + c] = acc[r];
-      }
-    }
+  for (int e = threadIdx.x; e < nrows * R; e += blockDim.x) {
+    const int cr = e % nrows, r = e / nrows;  // consecutive threads: consecutive latent rows
+    const float* wr = ws + cr * DNP;
+    const float* qr = qs + r * DN;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < DN; ++k) acc = fmaf(wr[k], qr[k], acc);
+    const int bl = r / G1, u = r % G1;
+    const int head = u < p.g ? h * p.g + u : n_S + h;
+    p.q_abs[((long)(b0 + bl) * H_q + head) * p.d_c + c0 + cr] = acc;
   }
-  // RoPE of the rotary query parts at position seqlen-1
+  // RoPE of the rotary query parts at position seqlen-1 (once per block row 0)
+  if (blockIdx.y != 0) return;
   const int half = p.d_rope >> 1;
   for (int e = threadIdx.x; e < R * half; e += blockDim.x) {
     const int r = e / half, k = e % half, bl = r / G1, u = r % G1;
@@ -189,46 +199,78 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
   }
 }
 
-// Merge the splits of every head of one KV group, apply W_UV, then
-// D = H_S - sigmoid(lam) H_N and Y = sigmoid(G) D. Block (KV group h, chunk of
-// sequences); the W_UV slice is streamed once per block.
+// Merge of the split partials of one (sequence, head): O_lat = sum_s w_s O_s with
+// w_s = exp2(m_s - M) / sum_s' exp2(m_s' - M) l_s'. One block per (sequence,
+// head); the result goes to o_lat [B, H_q, d_c] (the absorbed-query buffer,
+// which the split pass no longer needs).
+__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
+  const int head = blockIdx.x, b = blockIdx.y;
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, NS = p.n_splits, d_c = p.d_c;
+  __shared__ float wgt[256];
+  __shared__ float red[2];
+  const int tid = threadIdx.x;
+  if (tid < 32) {
+    float M = -INFINITY;
+    for (int s = tid; s < NS; s += 32) M = fmaxf(M, p.part_ml[(((long)b * NS + s) * H_q + head) * 2]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+    for (int s = tid; s < NS; s += 32) {
+      const float* ml = p.part_ml + (((long)b * NS + s) * H_q + head) * 2;
+      const float wv = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
+      wgt[s] = wv;
+      den += wv * ml[1];
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (tid == 0) red[0] = den > 0.f ? 1.f / den : 0.f;
+  }
+  __syncthreads();
+  const float inv = red[0];
+  const float* src = p.part_o + ((long)b * NS * H_q + head) * d_c;
+  for (int c = tid; c < d_c; c += blockDim.x) {
+    float acc = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < NS; ++s) acc = fmaf(wgt[s], src[(long)s * H_q * d_c + c], acc);
+    p.q_abs[((long)b * H_q + head) * d_c + c] = acc * inv;
+  }
+}
+
+// Rows (sequence, head of the group) per combine block and the W_UV slice
+// staged once per block: max(1, 12 / (g+1)) sequences x (g+1) heads.
+__host__ __device__ inline int combine_seqs(int g) { return max(1, 12 / (g + 1)); }
+
+// H = O_lat W_UV for the g+1 heads of KV group h, then D = H_S - sigmoid(lam) H_N
+// and Y = sigmoid(G) D. Block (KV group h, chunk of sequences).
 template <typename T>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
-  const int h = blockIdx.x, b0 = blockIdx.y * SEQ_PER_BLOCK;
-  const int nb = min(SEQ_PER_BLOCK, p.B - b0);
-  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1;
-  const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v), NS = p.n_splits;
+  const int spb = combine_seqs(p.g);
+  const int h = blockIdx.x, b0 = blockIdx.y * spb;
+  const int nb = min(spb, p.B - b0);
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1, RM = spb * G1;
+  const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v);
   extern __shared__ float sm[];
-  float* olat = sm;               // [R][d_c]
-  float* hv = olat + R * d_c;     // [R][DV]
-  float* wgt = hv + R * DV;       // [R][n_splits]
+  float* olat = sm;                        // [R][d_c]
+  float* hv = olat + RM * d_c;             // [R][DV]
+  T* wsm = reinterpret_cast<T*>(hv + RM * DV);  // [d_c][DV] W_UV slice
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   const T* gate = reinterpret_cast<const T*>(p.gate);
   T* out = reinterpret_cast<T*>(p.out);
   const int tid = threadIdx.x;
-  auto head_of = [&](int r) { const int u = r % G1; return u < p.g ? h * p.g + u : n_S + h; };
-  // split weights: exp2(m_s - M) / sum_s exp2(m_s - M) l_s
-  for (int r = tid; r < R; r += blockDim.x) {
-    const int b = b0 + r / G1, head = head_of(r);
-    float M = -INFINITY;
-    for (int s = 0; s < NS; ++s) M = fmaxf(M, p.part_ml[(((long)b * NS + s) * H_q + head) * 2]);
-    float den = 0.f;
-    for (int s = 0; s < NS; ++s) {
-      const float* ml = p.part_ml + (((long)b * NS + s) * H_q + head) * 2;
-      const float wv = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
-      wgt[r * NS + s] = wv;
-      den += wv * ml[1];
-    }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    for (int s = 0; s < NS; ++s) wgt[r * NS + s] *= inv;
+  constexpr int VEC = 16 / (int)sizeof(T);
+  const int per_row = DV / VEC;
+#pragma unroll 8
+  for (int e = tid; e < d_c * per_row; e += blockDim.x) {
+    const int c = e / per_row, v = e % per_row;
+    *reinterpret_cast<uint4*>(wsm + c * DV + v * VEC) =
+        *reinterpret_cast<const uint4*>(w + (long)c * ncol + (long)h * (p.d_nope + DV) + p.d_nope + v * VEC);
   }
-  __syncthreads();
-  for (int e = tid; e < R * d_c; e += blockDim.x) {
-    const int r = e / d_c, c = e % d_c;
-    const int b = b0 + r / G1, head = head_of(r);
-    float a = 0.f;
-    for (int s = 0; s < NS; ++s) a = fmaf(wgt[r * NS + s], p.part_o[(((long)b * NS + s) * H_q + head) * d_c + c], a);
-    olat[e] = a;
+#pragma unroll 4
+  for (int e = tid; e < R * (d_c / 4); e += blockDim.x) {
+    const int r = e / (d_c / 4), v = e % (d_c / 4), u = r % G1;
+    const int head = u < p.g ? h * p.g + u : n_S + h;
+    reinterpret_cast<float4*>(olat + r * d_c)[v] =
+        reinterpret_cast<const float4*>(p.q_abs + ((long)(b0 + r / G1) * H_q + head) * d_c)[v];
   }
   __syncthreads();
   // hv[r][n] = sum_c olat[r][c] W_UV[c][n]: thread column n, rows rg, rg+RG, ...
@@ -238,9 +280,9 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     float acc[MAX_ROWS];
 #pragma unroll
     for (int i = 0; i < MAX_ROWS; ++i) acc[i] = 0.f;
-    const T* wc = w + (long)h * (p.d_nope + DV) + p.d_nope + n;
+#pragma unroll 4
     for (int c = 0; c < d_c; ++c) {
-      const float wv = to_f(wc[(long)c * ncol]);
+      const float wv = to_f(wsm[c * DV + n]);
 #pragma unroll
       for (int i = 0; i < MAX_ROWS; ++i) {
         const int r = rg + i * RG;
@@ -265,12 +307,22 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
 }
 
 cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
-  dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + SEQ_PER_BLOCK - 1) / SEQ_PER_BLOCK));
-  const size_t smem = sizeof(float) * (size_t)SEQ_PER_BLOCK * (p.g + 1) * p.d_nope;
-  if (dt == GDLA_BF16)
-    decode_absorb_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(p);
-  else
-    decode_absorb_kernel<float><<<grid, 256, smem, s>>>(p);
+  dim3 grid((unsigned)p.n_kv, (unsigned)((p.d_c + ABS_ROWS - 1) / ABS_ROWS),
+            (unsigned)((p.B + ABS_SEQ - 1) / ABS_SEQ));
+  const size_t smem =
+      sizeof(float) * ((size_t)ABS_ROWS * (p.d_nope + 1) + (size_t)ABS_SEQ * (p.g + 1) * p.d_nope);
+  cudaError_t e;
+  if (dt == GDLA_BF16) {
+    auto k = decode_absorb_kernel<__nv_bfloat16>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, 256, smem, s>>>(p);
+  } else {
+    auto k = decode_absorb_kernel<float>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, 256, smem, s>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -312,10 +364,14 @@ cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaS
 }
 
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
-  const int R = SEQ_PER_BLOCK * (p.g + 1);
-  const size_t smem = sizeof(float) * ((size_t)R * p.d_c + (size_t)R * p.d_v + (size_t)R * p.n_splits);
-  dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + SEQ_PER_BLOCK - 1) / SEQ_PER_BLOCK));
-  cudaError_t e;
+  decode_merge_kernel<<<dim3((unsigned)(p.n_kv * (p.g + 1)), (unsigned)p.B), 256, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t esz = dt == GDLA_BF16 ? 2 : 4;
+  const int spb = combine_seqs(p.g);
+  const size_t RM = (size_t)spb * (p.g + 1);
+  const size_t smem = sizeof(float) * (RM * p.d_c + RM * p.d_v) + esz * (size_t)p.d_c * p.d_v;
+  dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + spb - 1) / spb));
   if (dt == GDLA_BF16) {
     auto k = decode_combine_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -6,19 +6,21 @@
 // With W_UK absorbed into the query (q_abs = W_UK q_nope, done beforehand by
 // decode_absorb) one sequence's attention over a tile of cache rows is two
 // small GEMMs in which the cache tile is the big operand:
-//   S^T[tokens x heads] = C[tokens x 576] . Qcat^T[576 x heads]      (M = 64 tokens)
-//   O^T[512 x heads]   += C[:, :512]^T[512 x tokens] . P^T[tokens x heads]  (M = 4 x 128 dims)
-// so the cache is streamed from HBM once, the same shared-memory tile feeds
-// both MMAs (K-major for the first, MN-major for the second), and no head
-// padding is needed (N = number of query heads, a multiple of 16).
+//   S^T[tokens x heads] = C[tokens x 576] . Qcat^T[576 x heads]          (M = 64 tokens, N = 48)
+//   O^T[512 x heads]   += C[:, :512]^T[512 x tokens] . P^T[tokens x heads]  (M = 4 x 128 dims, N = 64)
+// so the cache is streamed from HBM once and the same shared-memory tile feeds
+// both MMAs (K-major for the first, MN-major for the second).
 //
 // Block (split s, sequence b), 256 threads:
 //   warp 0      TMA producer: 64-token cache tiles (9 boxes: 8 latent + 1 rotary) in a 2-stage ring;
-//   warp 1      MMA issuer (one lane);
-//   warps 4-7   softmax over S^T (one token per thread, lanes 0-15 of each warp,
-//               the M = 64 accumulator layout), then the split's partial output.
-// The running maximum of each head is CTA-uniform and lives in registers; O is
-// rescaled (in TMEM) only when some head's maximum grows by more than 2^8.
+//   warp 1      issues the score MMAs (one lane); warp 2 the value MMAs;
+//   warps 4-7   softmax over S^T: each warp's lanes 0-15 own 16 tokens (the M = 64
+//               accumulator layout) and lanes 16-31 take the upper 24 heads of
+//               the same tokens; P^T is written token-major (16-byte stores).
+// The running maximum of each head is CTA-uniform and lives in registers; the
+// four softmax warps agree on whether it moved with one barrier-reduction per
+// tile, and O^T is rescaled (in TMEM) only when some head's maximum grows by
+// more than 2^8.
 #include <math.h>
 
 #include "kernels.h"
@@ -27,22 +29,24 @@
 namespace gdla {
 namespace {
 
-constexpr int TT = 64;               // tokens per tile
-constexpr int DC = 512, DRD = 64;    // latent, rotary widths
+constexpr int TT = 64;                 // tokens per tile
+constexpr int DC = 512, DRD = 64;      // latent, rotary widths
 constexpr int NBOX = (DC + DRD) / 64;  // 9 boxes of 64 columns
-constexpr int NPMAX = 48;            // padded heads (N of both MMAs)
+constexpr int NQ = 48;                 // query heads (N of the score MMA)
+constexpr int HH = NQ / 2;             // heads per lane half
+constexpr int NPV = 64;                // N of the value MMA: heads padded to one 128-byte row
 constexpr int TILE_BYTES = TT * (DC + DRD) * 2;  // 72 KB
-constexpr int QT_BYTES = NPMAX * (DC + DRD) * 2;  // 54 KB
-constexpr int PT_BYTES = NPMAX * TT * 2;          // 6 KB
+constexpr int QT_BYTES = NQ * (DC + DRD) * 2;    // 54 KB
+constexpr int PT_BYTES = TT * NPV * 2;           // 8 KB
 constexpr int DSTAGES = 2;
 constexpr int DSMEM = QT_BYTES + DSTAGES * TILE_BYTES + 2 * PT_BYTES + 1024;
 constexpr int DTHREADS = 256;
 constexpr float kThr = 8.0f;
-constexpr uint32_t COL_ST = 0;     // S^T buffers at [0, 64) and [64, 128)
-constexpr uint32_t COL_OT = 128;   // O^T M-tile mt at 128 + 64 mt
+constexpr uint32_t COL_ST = 0;    // S^T buffers at [0, 48) and [64, 112)
+constexpr uint32_t COL_OT = 128;  // O^T M-tile mt at 128 + 64 mt
 
 struct DBars {
-  uint64_t full[DSTAGES], empty[DSTAGES], s_full[2], p_full[2], p_free[2], o_done, sync, mma_done;
+  uint64_t full[DSTAGES], empty[DSTAGES], s_full[2], p_full[2], p_free[2], o_done, mma_done;
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -50,11 +54,25 @@ __device__ __forceinline__ float ex2f(float x) {
   asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// barrier 1 over the 128 softmax threads, OR-reducing a predicate
+__device__ __forceinline__ bool bar_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_sync128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 }  // namespace
 
 struct DecodeTcArgs {
-  int B, T_max, n_splits, split_len, sliding, window, H_q, NP;
+  int B, T_max, n_splits, split_len, sliding, window, H_q;
   const int* seqlens;
   const float* q_abs;   // [B, H_q, 512]
   const float* q_rot;   // [B, H_q, 64]
@@ -70,21 +88,20 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qt = smem;                                   // Qcat^T, 9 boxes of [NP x 128 B]
-  uint8_t* tiles = smem + QT_BYTES;                     // stages, 9 boxes of [64 x 128 B]
-  uint8_t* pt = tiles + DSTAGES * TILE_BYTES;           // P^T double buffer [NP x 128 B]
+  uint8_t* qt = smem;                          // Qcat^T, 9 boxes of [NQ x 128 B]
+  uint8_t* tiles = smem + QT_BYTES;            // stages, 9 boxes of [64 x 128 B]
+  uint8_t* pt = tiles + DSTAGES * TILE_BYTES;  // P^T double buffer [64 tokens x 128 B]
   __shared__ __align__(8) DBars bars;
   __shared__ uint32_t tmem_slot;
-  __shared__ int flag[3];
-  __shared__ float wmax[4][NPMAX];
-  __shared__ float lsum[NPMAX];
-  __shared__ float alpha_s[NPMAX];
+  __shared__ float wmax[4][NQ];
+  __shared__ float lsum[NQ];
+  __shared__ float alpha_s[NQ];
   __shared__ volatile int abort_flag;
 
   if (sm100::earlier_failure(a.status)) return;  // an earlier CTA of this call timed out
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.x, b = blockIdx.y;
-  const int H_q = a.H_q, NP = a.NP;
+  const int H_q = a.H_q;
   const int Tb = a.seqlens[b];
   const int lo = a.sliding ? max(0, Tb - a.window) : 0;
   const int t0 = max(lo, s * a.split_len), t1 = min(Tb, (s + 1) * a.split_len);
@@ -102,16 +119,14 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       mbar_init(smem_u32(&bars.p_free[i]), 1);
     }
     mbar_init(smem_u32(&bars.o_done), 1);
-    mbar_init(smem_u32(&bars.sync), 128);
-    mbar_init(smem_u32(&bars.mma_done), 1);
+    mbar_init(smem_u32(&bars.mma_done), 2);  // one commit per MMA-issuing warp
     fence_mbar_init();
-    flag[0] = flag[1] = flag[2] = 0;
     abort_flag = 0;
     prefetch_tmap(&tmC);
     prefetch_tmap(&tmR);
   }
-  // Qcat^T in bf16, pre-scaled by tau*log2(e), K-major with the 128-byte swizzle; zero P^T
-  for (int e = threadIdx.x; e < NP * NBOX * 8; e += DTHREADS) {
+  // Qcat^T in bf16, pre-scaled by tau*log2(e), K-major with the 128-byte swizzle
+  for (int e = threadIdx.x; e < NQ * NBOX * 8; e += DTHREADS) {
     const int h = e / (NBOX * 8), rem = e % (NBOX * 8), bx = rem / 8, c = rem % 8;  // 16-byte chunk
     uint32_t w[4];
 #pragma unroll
@@ -119,20 +134,17 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       float v0 = 0.f, v1 = 0.f;
       if (h < H_q) {
         const int d = bx * 64 + c * 8 + 2 * u;
-        if (d < DC) {
-          const float* src = a.q_abs + ((long)b * H_q + h) * DC + d;
-          v0 = src[0] * a.sl2;
-          v1 = src[1] * a.sl2;
-        } else {
-          const float* src = a.q_rot + ((long)b * H_q + h) * DRD + (d - DC);
-          v0 = src[0] * a.sl2;
-          v1 = src[1] * a.sl2;
-        }
+        const float* src = d < DC ? a.q_abs + ((long)b * H_q + h) * DC + d
+                                  : a.q_rot + ((long)b * H_q + h) * DRD + (d - DC);
+        v0 = src[0] * a.sl2;
+        v1 = src[1] * a.sl2;
       }
       w[u] = pack_bf16x2(v0, v1);
     }
-    *reinterpret_cast<uint4*>(qt + bx * (NP * 128) + h * 128 + ((c ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(qt + bx * (NQ * 128) + h * 128 + ((c ^ (h & 7)) << 4)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
+  // P^T buffers start at zero: the padding heads 48..63 stay zero
   for (int e = threadIdx.x; e < 2 * PT_BYTES / 16; e += DTHREADS)
     reinterpret_cast<uint4*>(pt)[e] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
@@ -150,7 +162,8 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       int k = 0;
       for (; k < n_tiles && !abort_flag; ++k) {
         const int st = k % DSTAGES;
-        if (k >= DSTAGES && !mbar_wait(smem_u32(&bars.empty[st]), ((k / DSTAGES) & 1) ^ 1, a.status, 301, &abort_flag)) {
+        if (k >= DSTAGES &&
+            !mbar_wait(smem_u32(&bars.empty[st]), ((k / DSTAGES) & 1) ^ 1, a.status, 301, &abort_flag)) {
           abort_flag = 1;
           break;
         }
@@ -165,216 +178,229 @@ __global__ void __launch_bounds__(DTHREADS, 1)
         for (int q = (k > DSTAGES ? k - DSTAGES : 0); q < k; ++q)
           mbar_wait(smem_u32(&bars.full[q % DSTAGES]), (q / DSTAGES) & 1, nullptr, 0);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
+    // warp 1 issues the score MMAs, warp 2 the value MMAs: neither waits behind
+    // the other's instructions
     if (lane == 0) {
-      const uint32_t id1 = idesc_bf16_f32(64, NP, false, false);
-      const uint32_t id2 = idesc_bf16_f32(128, NP, true, false);
+      constexpr uint32_t id1 = idesc_bf16_f32(64, NQ, false, false);
+      constexpr uint32_t id2 = idesc_bf16_f32(128, NPV, true, true);
+      // descriptors of the fixed operands; per-step offsets are added to the
+      // 16-byte address field (addresses stay below 2^18 bytes, so no carry)
+      static_assert(DSTAGES == 2, "stage selection below assumes two stages");
+      const uint64_t qd0 = sdesc_sw128(smem_u32(qt), 16, 1024);
+      const uint64_t cdA = sdesc_sw128(smem_u32(tiles), 16, 1024);
+      const uint64_t cdB = sdesc_sw128(smem_u32(tiles + TILE_BYTES), 16, 1024);
+      const uint64_t cmA = sdesc_sw128(smem_u32(tiles), TT * 128, 1024);
+      const uint64_t cmB = sdesc_sw128(smem_u32(tiles + TILE_BYTES), TT * 128, 1024);
+      const uint64_t pdA = sdesc_sw128(smem_u32(pt), 8192, 1024);
+      const uint64_t pdB = sdesc_sw128(smem_u32(pt + PT_BYTES), 8192, 1024);
       bool ok = true;
-      const uint32_t qbase = smem_u32(qt);
-      auto mma2 = [&](int k) {
-        // O^T += C^T . P^T for tile k (all four 128-dim M-tiles)
-        const uint32_t cb = smem_u32(tiles + (k % DSTAGES) * TILE_BYTES);
-        const uint32_t pb = smem_u32(pt + (k & 1) * PT_BYTES);
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-          for (int kk = 0; kk < TT / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(cb + 2 * mt * (TT * 128) + kk * 2048, TT * 128, 1024);
-            const uint64_t bd = sdesc_sw128(pb + kk * 32, 16, 1024);
-            mma_ss(tmem + COL_OT + 64 * mt, ad, bd, id2, (k > 0 || kk > 0) ? 1u : 0u);
-          }
-        // p_free[k & 1] completes once per odd/even tile: it says both that P^T buffer
-        // k & 1 may be rewritten and that O^T holds every tile up to k
-        mma_commit(smem_u32(&bars.empty[k % DSTAGES]));
-        mma_commit(smem_u32(&bars.p_free[k & 1]));
-      };
-      for (int k = 0; k < n_tiles && ok; ++k) {
-        ok = mbar_wait(smem_u32(&bars.full[k % DSTAGES]), (k / DSTAGES) & 1, a.status, 311, &abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t cb = smem_u32(tiles + (k % DSTAGES) * TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < NBOX * 4; ++kk) {
-          const uint64_t ad = sdesc_sw128(cb + (kk >> 2) * (TT * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(qbase + (kk >> 2) * (NP * 128) + (kk & 3) * 32, 16, 1024);
-          mma_ss(tmem + COL_ST + 64 * (k & 1), ad, bd, id1, kk > 0);
-        }
-        mma_commit(smem_u32(&bars.s_full[k & 1]));
-        if (k > 0) {
-          ok = mbar_wait(smem_u32(&bars.p_full[(k - 1) & 1]), ((k - 1) >> 1) & 1, a.status, 312, &abort_flag);
+      if (warp == 1) {
+        for (int k = 0; k < n_tiles && ok; ++k) {
+          ok = mbar_wait(smem_u32(&bars.full[k % DSTAGES]), (k / DSTAGES) & 1, a.status, 311, &abort_flag);
+          // S^T buffer k & 1 was last read by the softmax of tile k-2
+          if (ok && k >= 2)
+            ok = mbar_wait(smem_u32(&bars.p_full[k & 1]), ((k >> 1) & 1) ^ 1, a.status, 312, &abort_flag);
           if (!ok) break;
           tc_fence_after();
-          mma2(k - 1);
+          const uint64_t c0 = (k & 1) ? cdB : cdA;
+#pragma unroll
+          for (int kk = 0; kk < NBOX * 4; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            mma_ss(tmem + COL_ST + 64 * (k & 1), c0 + (((kk >> 2) * (TT * 128) + off) >> 4),
+                   qd0 + (((kk >> 2) * (NQ * 128) + off) >> 4), id1, kk > 0);
+          }
+          mma_commit(smem_u32(&bars.s_full[k & 1]));
         }
-      }
-      if (ok && n_tiles > 0) {
-        ok = mbar_wait(smem_u32(&bars.p_full[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1, a.status, 313, &abort_flag);
-        if (ok) {
+      } else {
+        for (int k = 0; k < n_tiles && ok; ++k) {
+          ok = mbar_wait(smem_u32(&bars.p_full[k & 1]), (k >> 1) & 1, a.status, 313, &abort_flag);
+          if (!ok) break;
           tc_fence_after();
-          mma2(n_tiles - 1);
+          // O^T += C^T . P^T for tile k (all four 128-dim M-tiles)
+          const uint64_t a0 = (k & 1) ? cmB : cmA, b0 = (k & 1) ? pdB : pdA;
+#pragma unroll
+          for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int kk = 0; kk < TT / 16; ++kk)
+              mma_ss(tmem + COL_OT + 64 * mt, a0 + ((2 * mt * (TT * 128) + kk * 2048) >> 4),
+                     b0 + ((kk * 2048) >> 4), id2, (k > 0 || kk > 0) ? 1u : 0u);
+          // p_free[k & 1] completes once per odd/even tile: P^T buffer k & 1 may be
+          // rewritten, and O^T holds every tile up to k
+          mma_commit(smem_u32(&bars.empty[k % DSTAGES]));
+          mma_commit(smem_u32(&bars.p_free[k & 1]));
         }
+        mma_commit(smem_u32(&bars.o_done));
       }
-      mma_commit(smem_u32(&bars.o_done));
       if (!ok) abort_flag = 1;
+      // every MMA this thread issued has completed before TMEM is released
       mma_commit(smem_u32(&bars.mma_done));
       mbar_wait(smem_u32(&bars.mma_done), 0, nullptr, 314);
     }
   } else if (warp >= 4) {
     const int q4 = warp & 3;
-    const bool rowl = lane < 16;
+    const int hf = lane >> 4;                 // lane half: heads [24 hf, 24 hf + 24)
+    const int hb = hf * HH;
     const int tok_local = q4 * 16 + (lane & 15);
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    float m_ref[NPMAX], lp[NPMAX];
+    // thr[h] = m_ref[h] + 2^8 margin (log2 units); -inf until the head has a
+    // finite maximum, +inf for padding heads. One compare per score decides
+    // whether any maximum moved (no branches in the per-score loop).
+    float m_ref[HH], lp[HH], thr[HH];
 #pragma unroll
-    for (int h = 0; h < NPMAX; ++h) {
+    for (int h = 0; h < HH; ++h) {
       m_ref[h] = -INFINITY;
       lp[h] = 0.f;
+      thr[h] = (hb + h < H_q) ? -INFINITY : INFINITY;
     }
-    uint32_t sync_ph = 0;
     bool ok = true;
-    auto block_sync = [&]() -> bool {
-      mbar_arrive(smem_u32(&bars.sync));
-      const bool r = mbar_wait(smem_u32(&bars.sync), sync_ph & 1, a.status, 321, &abort_flag);
-      ++sync_ph;
-      return __all_sync(0xffffffffu, r);
-    };
     for (int k = 0; k < n_tiles; ++k) {
-      ok = mbar_wait(smem_u32(&bars.s_full[k & 1]), (k >> 1) & 1, a.status, 322, &abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
+      bool w_ok = mbar_wait(smem_u32(&bars.s_full[k & 1]), (k >> 1) & 1, a.status, 322, &abort_flag);
+      w_ok = __all_sync(0xffffffffu, w_ok);
+      if (w_ok && k >= 2) {
+        // P^T buffer k & 1 is free and O^T holds tiles < k-1 (MMA of tile k-2 done)
+        w_ok = mbar_wait(smem_u32(&bars.p_free[k & 1]), ((k >> 1) & 1) ^ 1, a.status, 324, &abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
       }
-      if (k >= 2) {
-        // P^T buffer k & 1 and O^T up to tile k-2 are free/settled (MMA of tile k-2 done)
-        ok = mbar_wait(smem_u32(&bars.p_free[k & 1]), ((k >> 1) & 1) ^ 1, a.status, 324, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
+      float y[HH];
+      bool exceed = false;
+      if (w_ok) {
+        tc_fence_after();
+        uint32_t xr[NQ];
+        const uint32_t tS = tmem + lane_base + COL_ST + 64 * (k & 1);
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&xr[0]));
+        tmem_ld16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&xr[32]));
+        tmem_wait_ld();
+        const int j = jt0 + k * TT + tok_local;
+        const bool valid = j >= t0 && j < t1;
+        const bool tile_full = (jt0 + k * TT >= t0) && (jt0 + k * TT + TT <= t1);
+#pragma unroll
+        for (int h = 0; h < HH; ++h) {
+          const float hi = __shfl_sync(0xffffffffu, __uint_as_float(xr[HH + h]), lane & 15);
+          y[h] = hf ? hi : __uint_as_float(xr[h]);
+        }
+        if (!tile_full) {
+#pragma unroll
+          for (int h = 0; h < HH; ++h) y[h] = valid ? y[h] : -INFINITY;
+        }
+#pragma unroll
+        for (int h = 0; h < HH; ++h) exceed |= y[h] > thr[h];
+      }
+      if (bar_or(exceed || !w_ok)) {
+        if (bar_or(!w_ok)) {
           ok = false;
           break;
         }
-      }
-      tc_fence_after();
-      float x[NPMAX];
-      tmem_ld32(tmem + lane_base + COL_ST + 64 * (k & 1), *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-      tmem_ld16(tmem + lane_base + COL_ST + 64 * (k & 1) + 32, *reinterpret_cast<uint32_t(*)[16]>(&x[32]));
-      tmem_wait_ld();
-      const int j = jt0 + k * TT + tok_local;
-      const bool valid = rowl && j >= t0 && j < t1;
-      bool exceed = false;
+        // some head's maximum grew: CTA-wide per-head maximum of this tile
 #pragma unroll
-      for (int h = 0; h < NPMAX; ++h) {
-        x[h] = (valid && h < H_q) ? x[h] : -INFINITY;
-        exceed |= x[h] > m_ref[h] + kThr || (m_ref[h] == -INFINITY && x[h] > -INFINITY);
-      }
-      if (__any_sync(0xffffffffu, exceed) && lane == 0) atomicOr(&flag[k % 3], 1);
-      if (!(ok = block_sync())) break;
-      if (threadIdx.x == 128) flag[(k + 2) % 3] = 0;
-      if (flag[k % 3]) {
-        // some head's maximum grew: CTA-wide per-head max of this tile
-#pragma unroll
-        for (int h = 0; h < NPMAX; ++h) {
-          float v = x[h];
+        for (int h = 0; h < HH; ++h) {
+          float v = y[h];
           v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
           v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
           v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
           v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-          if (lane == 0) wmax[q4][h] = v;
+          if ((lane & 15) == 0) wmax[q4][hb + h] = v;
         }
-        if (!(ok = block_sync())) break;
-        bool any_resc = false;
+        bar_sync128();
+        bool resc = false;
 #pragma unroll
-        for (int h = 0; h < NPMAX; ++h) {
-          const float tm = fmaxf(fmaxf(wmax[0][h], wmax[1][h]), fmaxf(wmax[2][h], wmax[3][h]));
+        for (int h = 0; h < HH; ++h) {
+          const float tm = fmaxf(fmaxf(wmax[0][hb + h], wmax[1][hb + h]), fmaxf(wmax[2][hb + h], wmax[3][hb + h]));
           const bool up = tm > m_ref[h] + kThr || (m_ref[h] == -INFINITY && tm > -INFINITY);
           const float mn = up ? fmaxf(m_ref[h], tm) : m_ref[h];
           const float al = (!up || m_ref[h] == -INFINITY) ? (up ? 0.f : 1.f) : ex2f(m_ref[h] - mn);
-          any_resc |= up && m_ref[h] != -INFINITY;
+          resc |= up && m_ref[h] != -INFINITY;
           lp[h] *= al;
           m_ref[h] = mn;
-          if ((int)threadIdx.x - 128 == h) alpha_s[h] = al;
+          if (hb + h < H_q) thr[h] = mn + kThr;
+          if (q4 == 0 && (lane & 15) == 0) alpha_s[hb + h] = al;
         }
-        if (k > 0 && any_resc) {
-          if (!(ok = block_sync())) break;  // alpha_s visible to every thread
+        // the reduction is also the barrier that publishes alpha_s
+        if (bar_or(resc) && k > 0) {
           // O^T holds tiles < k once the MMA of tile k-1 has landed (p_free of its parity)
-          ok = mbar_wait(smem_u32(&bars.p_free[(k - 1) & 1]), ((k - 1) >> 1) & 1, a.status, 323, &abort_flag);
-          if (!__all_sync(0xffffffffu, ok)) {
+          bool r_ok =
+              mbar_wait(smem_u32(&bars.p_free[(k - 1) & 1]), ((k - 1) >> 1) & 1, a.status, 323, &abort_flag);
+          r_ok = __all_sync(0xffffffffu, r_ok);
+          if (bar_or(!r_ok)) {
             ok = false;
             break;
           }
           tc_fence_after();
 #pragma unroll 1
           for (int mt = 0; mt < 4; ++mt) {
-            uint32_t o[NPMAX];
+            uint32_t o[NQ];
             const uint32_t ta = tmem + lane_base + COL_OT + 64 * mt;
             tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
             tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < NPMAX; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha_s[h]);
+            for (int h = 0; h < NQ; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha_s[h]);
             tmem_st32(ta, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
             tmem_st16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
           }
           tmem_wait_st();
         }
       }
-      // P^T tile k (bf16): row h = head, 64 tokens, 128-byte swizzle
-      uint8_t* pb = pt + (k & 1) * PT_BYTES;
-      if (rowl) {
+      // P^T row of this token: heads [hb, hb + 24) = three 16-byte chunks
+      uint8_t* prow = pt + (k & 1) * PT_BYTES + tok_local * 128;
 #pragma unroll
-        for (int h = 0; h < NPMAX; ++h) {
-          const float p = (h < H_q) ? ex2f(x[h] - (m_ref[h] == -INFINITY ? 0.f : m_ref[h])) : 0.f;
-          lp[h] += p;
-          if (h < NP) {
-            const int c = tok_local >> 3;
-            *reinterpret_cast<__nv_bfloat16*>(pb + h * 128 + ((c ^ (h & 7)) << 4) + (tok_local & 7) * 2) =
-                __float2bfloat16_rn(p);
-          }
+      for (int c = 0; c < 3; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int h0 = c * 8 + 2 * u;
+          const float p0 = ex2f(y[h0] - (m_ref[h0] == -INFINITY ? 0.f : m_ref[h0]));
+          const float p1 = ex2f(y[h0 + 1] - (m_ref[h0 + 1] == -INFINITY ? 0.f : m_ref[h0 + 1]));
+          lp[h0] += p0;
+          lp[h0 + 1] += p1;
+          w[u] = pack_bf16x2(p0, p1);
         }
+        const int chunk = hf * 3 + c;
+        *reinterpret_cast<uint4*>(prow + ((chunk ^ (tok_local & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(&bars.p_full[k & 1]));
     }
     // ---- partial results of this split: (m, l) per head and O^T
-    if (ok) {
-      ok = mbar_wait(smem_u32(&bars.o_done), 0, a.status, 325, &abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
+    bool fin = ok;
+    if (fin) {
+      bool w_ok = mbar_wait(smem_u32(&bars.o_done), 0, a.status, 325, &abort_flag);
+      fin = !bar_or(!__all_sync(0xffffffffu, w_ok));
     }
-    if (ok) {
+    if (fin) {
       tc_fence_after();
-      if (threadIdx.x < 128 + NPMAX) lsum[threadIdx.x - 128] = 0.f;
-      ok = block_sync();
-    }
-    if (ok) {
+      if (threadIdx.x - 128 < NQ) lsum[threadIdx.x - 128] = 0.f;
+      bar_sync128();
 #pragma unroll
-      for (int h = 0; h < NPMAX; ++h) {
-        float v = rowl ? lp[h] : 0.f;
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
+      for (int h = 0; h < HH; ++h) {
+        float v = lp[h];
         v += __shfl_xor_sync(0xffffffffu, v, 8);
         v += __shfl_xor_sync(0xffffffffu, v, 4);
         v += __shfl_xor_sync(0xffffffffu, v, 2);
         v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (lane == 0 && h < H_q) atomicAdd(&lsum[h], v);
+        if ((lane & 15) == 0) atomicAdd(&lsum[hb + h], v);
       }
-      ok = block_sync();
-    }
-    const long base = ((long)b * a.n_splits + s) * H_q;
-    if (ok) {
+      bar_sync128();
+      const long base = ((long)b * a.n_splits + s) * H_q;
+      if (q4 == 0 && (lane & 15) == 0) {
 #pragma unroll
-      for (int h = 0; h < NPMAX; ++h)
-        if ((int)threadIdx.x - 128 == h && h < H_q) {
-          a.part_ml[(base + h) * 2 + 0] = m_ref[h];
-          a.part_ml[(base + h) * 2 + 1] = lsum[h];
-        }
+        for (int h = 0; h < HH; ++h)
+          if (hb + h < H_q) {
+            a.part_ml[(base + hb + h) * 2 + 0] = m_ref[h];
+            a.part_ml[(base + hb + h) * 2 + 1] = lsum[hb + h];
+          }
+      }
 #pragma unroll 1
       for (int mt = 0; mt < 4; ++mt) {
-        uint32_t o[NPMAX];
+        uint32_t o[NQ];
         const uint32_t ta = tmem + lane_base + COL_OT + 64 * mt;
         tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
         tmem_ld16(ta + 32, *reinterpret_cast<uint32_t(*)[16]>(&o[32]));
         tmem_wait_ld();
         const int dim = mt * 128 + q4 * 32 + lane;
 #pragma unroll
-        for (int h = 0; h < NPMAX; ++h)
+        for (int h = 0; h < NQ; ++h)
           if (h < H_q) a.part_o[(base + h) * DC + dim] = n_tiles > 0 ? __uint_as_float(o[h]) : 0.f;
       }
     } else {
@@ -389,7 +415,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
 
 bool decode_tc_supported(const DecodeParams& p, gdla_dtype dt) {
   const int H_q = p.n_kv * (p.g + 1);
-  return dt == GDLA_BF16 && p.d_c == DC && p.d_rope == DRD && H_q <= NPMAX && p.split_len % TT == 0 &&
+  return dt == GDLA_BF16 && p.d_c == DC && p.d_rope == DRD && H_q <= NQ && p.split_len % TT == 0 &&
          get_encode_tiled() != nullptr;
 }
 
@@ -410,7 +436,7 @@ cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s) {
   }
   DecodeTcArgs a{};
   a.B = p.B; a.T_max = p.T_max; a.n_splits = p.n_splits; a.split_len = p.split_len;
-  a.sliding = p.sliding; a.window = p.window; a.H_q = H_q; a.NP = NPMAX;
+  a.sliding = p.sliding; a.window = p.window; a.H_q = H_q;
   a.seqlens = p.seqlens; a.q_abs = p.q_abs; a.q_rot = p.q_rot; a.sl2 = p.scale * kLog2e;
   a.part_o = p.part_o; a.part_ml = p.part_ml; a.status = p.status;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DSMEM);
