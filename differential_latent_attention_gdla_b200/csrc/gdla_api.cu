@@ -64,17 +64,20 @@ struct DecodeLayout {
 DecodeLayout decode_layout(const gdla_decode_args* a) {
   DecodeLayout l;
   const int H_q = a->n_kv * (a->g + 1);
-  // split the cache of every sequence into n chunks (multiples of 64 tokens) so
-  // that B*n blocks fill whole waves of one block per SM: minimise
-  // waves(B*n) * tiles_per_split(n), with a mild penalty for more partials
+  // split the cache of every sequence into n chunks (multiples of 64 tokens):
+  // B*n blocks run in waves of one block per SM, and a block moves its cache
+  // tiles plus its partial result (written here, read back by the merge).
+  // Minimise waves(B*n) * (bytes one block moves).
   const int tile = 64;
   const int tiles = (a->T_max + tile - 1) / tile;
+  const double tile_bytes = (double)tile * (a->d_c + a->d_rope) * 2.0;
+  const double partial_bytes = 2.0 * H_q * (a->d_c + 2) * 4.0;
   int best_n = 1;
   double best = 1e300;
   for (int n = 1; n <= tiles && n <= 256; ++n) {
     const long waves = ((long)a->B * n + kNumSMs - 1) / kNumSMs;
     const long per = (tiles + n - 1) / n;
-    const double cost = (double)waves * per * (1.0 + 0.002 * n);
+    const double cost = (double)waves * (per * tile_bytes + partial_bytes);
     if (cost < best) {
       best = cost;
       best_n = n;
