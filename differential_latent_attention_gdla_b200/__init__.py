@@ -20,7 +20,7 @@ import torch
 from . import _abi
 from ._abi import GDLA_BF16, GDLA_FP32, GDLA_MASK_CAUSAL, GDLA_MASK_SLIDING, GdlaError  # noqa: F401
 
-__all__ = ["prefill", "attend", "decode", "latent_expand", "rope_tables", "prefill_workspace_size", "decode_workspace_size",
+__all__ = ["prefill", "attend", "decode", "decode_noalloc", "latent_expand", "rope_tables", "prefill_workspace_size", "decode_workspace_size",
            "workspace_status", "build_info", "GdlaError"]
 
 _DT = {torch.bfloat16: GDLA_BF16, torch.float32: GDLA_FP32}
@@ -214,6 +214,24 @@ def decode(c_cache, kr_cache, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_log
         workspace = torch.empty(need, dtype=torch.uint8, device=c_cache.device)
         a.workspace, a.workspace_bytes = workspace.data_ptr(), need
     _abi.check(_lib().gdla_decode(ctypes.byref(a), _stream(stream)), "gdla_decode")
+    return out
+
+
+def decode_noalloc(c_cache, kr_cache, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, seqlens, *, g: int,
+                   mask: str = "causal", window: int = 0, softmax_scale: float = 0.0, out=None, stream=None):
+    """decode() for callers that cannot provide device scratch: the library's
+    own fixed 32 MiB array is used instead of a workspace (see
+    gdla_decode_noalloc in include/gdla.h: calls on one device share it and
+    must not overlap; the first call on a device should come before any stream
+    capture). Raises GdlaError (GDLA_ERR_SCRATCH_LIMIT) for a batch too large
+    for the array."""
+    B = c_cache.shape[0]
+    if out is None:
+        out = torch.empty((B, lam_logits.shape[-1], gate_logits.shape[-1]), dtype=c_cache.dtype,
+                          device=c_cache.device)
+    a = _decode_args(c_cache, kr_cache, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, seqlens, out, g,
+                     mask, window, softmax_scale, None)
+    _abi.check(_lib().gdla_decode_noalloc(ctypes.byref(a), _stream(stream)), "gdla_decode_noalloc")
     return out
 
 

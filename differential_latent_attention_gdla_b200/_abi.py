@@ -12,7 +12,8 @@ import threading
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdla.so")
 
-GDLA_OK, GDLA_ERR_INVALID_ARG, GDLA_ERR_UNSUPPORTED, GDLA_ERR_CUDA, GDLA_ERR_TIMEOUT = range(5)
+GDLA_OK, GDLA_ERR_INVALID_ARG, GDLA_ERR_UNSUPPORTED, GDLA_ERR_CUDA, GDLA_ERR_TIMEOUT, GDLA_ERR_SCRATCH_LIMIT = range(6)
+GDLA_DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 GDLA_MASK_CAUSAL, GDLA_MASK_SLIDING = 0, 1
 GDLA_BF16, GDLA_FP32 = 0, 1
 
@@ -56,7 +57,7 @@ class DecodeArgs(ctypes.Structure):
 
 # Every symbol include/gdla.h declares.
 EXPORTED = ("gdla_latent_expand", "gdla_prefill_workspace_size", "gdla_prefill", "gdla_attend", "gdla_decode_workspace_size",
-            "gdla_decode", "gdla_status_string", "gdla_workspace_status", "gdla_build_info")
+            "gdla_decode", "gdla_decode_noalloc", "gdla_status_string", "gdla_workspace_status", "gdla_build_info")
 
 _lock = threading.Lock()
 _lib = None
@@ -85,6 +86,8 @@ def load(path: str = LIB_PATH):
         lib.gdla_decode_workspace_size.restype = ctypes.c_size_t
         lib.gdla_decode.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         lib.gdla_decode.restype = ctypes.c_int
+        lib.gdla_decode_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
+        lib.gdla_decode_noalloc.restype = ctypes.c_int
         lib.gdla_status_string.argtypes = [ctypes.c_int]
         lib.gdla_status_string.restype = ctypes.c_char_p
         lib.gdla_workspace_status.argtypes = [_vp, _vp]

@@ -157,6 +157,8 @@ const char* gdla_status_string(gdla_status s) {
     case GDLA_ERR_UNSUPPORTED: return "GDLA_ERR_UNSUPPORTED: valid arguments outside the implemented shapes";
     case GDLA_ERR_CUDA: return "GDLA_ERR_CUDA: a CUDA launch or query failed";
     case GDLA_ERR_TIMEOUT: return "GDLA_ERR_TIMEOUT: a device-side wait hit its iteration cap";
+    case GDLA_ERR_SCRATCH_LIMIT:
+      return "GDLA_ERR_SCRATCH_LIMIT: the call needs more scratch than gdla_decode_noalloc's fixed array";
   }
   return "unknown gdla_status";
 }

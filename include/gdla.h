@@ -45,7 +45,8 @@ typedef enum {
   GDLA_ERR_INVALID_ARG = 1,  /* NULL/misaligned pointer, bad size, small workspace */
   GDLA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. n_noise != n_kv) */
   GDLA_ERR_CUDA = 3,         /* a CUDA launch or query failed */
-  GDLA_ERR_TIMEOUT = 4       /* a device wait hit its iteration cap */
+  GDLA_ERR_TIMEOUT = 4,      /* a device wait hit its iteration cap */
+  GDLA_ERR_SCRATCH_LIMIT = 5 /* gdla_decode_noalloc: the call needs more than its fixed scratch */
 } gdla_status;
 
 typedef enum {
@@ -187,6 +188,30 @@ typedef struct {
 
 size_t gdla_decode_workspace_size(const gdla_decode_args* args);
 gdla_status gdla_decode(const gdla_decode_args* args, void* stream);
+
+/* ---------------------------------------------------------- decode, no alloc
+ * Not part of the layer itself (the report has no counterpart): the same
+ * decode as gdla_decode for callers that cannot provide a workspace -- code
+ * that must not allocate device memory while it runs, such as a step replayed
+ * from a captured CUDA graph, a latency-bound serving loop, or a plugin that
+ * only receives its inputs and outputs. The scratch comes from a fixed array
+ * inside the library instead of args->workspace (which is ignored):
+ *  - size: GDLA_DECODE_NOALLOC_SCRATCH_BYTES (32 MiB), held on every GPU that
+ *    loads the library until the process exits. A call whose
+ *    gdla_decode_workspace_size() exceeds it returns GDLA_ERR_SCRATCH_LIMIT
+ *    before launching anything (e.g. B=16 sequences of 4096 tokens fit,
+ *    B=64 sequences of 32768 tokens do not);
+ *  - the first call on a device looks up the array's device address (with that
+ *    device current) and caches it: make that first call before any stream
+ *    capture;
+ *  - every call on a device shares the one array and leaves the previous
+ *    call's data in it (the status word is cleared by each call): calls that
+ *    can overlap on the GPU, from any stream or thread, race and must be
+ *    serialised by the caller;
+ *  - it allocates and frees nothing; errors as for gdla_decode, and
+ *    gdla_workspace_status cannot be used on it. */
+#define GDLA_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+gdla_status gdla_decode_noalloc(const gdla_decode_args* args, void* stream);
 
 /* ---------------------------------------------------------------- utilities */
 const char* gdla_status_string(gdla_status s);

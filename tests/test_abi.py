@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(5):
+    for code in range(6):
         assert lib.gdla_status_string(code)
     assert b"INVALID" in lib.gdla_status_string(_abi.GDLA_ERR_INVALID_ARG)
 
