@@ -3,26 +3,35 @@
 // Report", Architecture: RoPE only on the rotary parts; signal and noise heads
 // attend independently; D = H_S - lambda (.) Repeat_g(H_N); Y = sigmoid(G) (.) D).
 //
-// One CTA owns (sequence b, KV group h, 128 query rows) and every head that
-// reads KV head h: the noise head and its g signal heads. The heads are taken
-// two at a time ("slots" A and B) so that each expanded K/V tile brought in
-// from L2 serves two heads:
+// One CTA owns (sequence b, KV group h, 64 query rows) and every head that
+// reads KV head h: the noise head and its g signal heads, taken two at a time:
 //   pair 0 = (noise, signal 0), pair 1 = (signal 1, signal 2), ...
-// Warp roles (384 threads):
-//   warp 0      TMA producer: the pair's Q tiles; K tiles (64 keys x 192) run two
-//               tiles ahead of V tiles (64 keys x 128), each in a 2-deep ring;
-//   warp 1      MMA issuer (one lane): S = Q K^T (128x64x192, both operands in
-//               shared memory) and O += P V (128x128x64, P read from TMEM);
-//   warps 4-7   softmax + epilogue of slot A (one query row per thread);
-//   warps 8-11  softmax + epilogue of slot B.
-// TMEM (512 columns): per slot two S buffers (64 columns each; P overwrites the
-// first half of its S buffer as bf16) and O (128 columns). S of tile j+2 is
-// computed while the softmax of tile j runs, so a slot's softmax never waits for
-// the tensor core in steady state. The noise head's normalised output H_N is
-// parked in shared memory (bf16) for the epilogues of all g signal heads, so
-// neither H_S nor H_N goes to global memory.
-// O is rescaled only when a row's running maximum grows by more than 2^8, and
-// only then does the softmax wait for the previous PV to land.
+// The two heads of a pair are stacked into one 128-row operand (rows 0-63 the
+// first head, rows 64-127 the second), so every tensor-core instruction is
+// M = 128 x N = 128: S = Q K^T over a 128-key tile (K = 192) and O += P V
+// (K = 128 keys, N = 128 value dims), and every K/V tile brought in from L2
+// serves both heads. Both Q (rotated once per pair) and P live in TMEM, so the
+// tensor core reads only K and V from shared memory.
+// Warp roles (640 threads):
+//   warp 0      TMA producer: the pair's Q in three 64-dim chunks through a
+//               2-deep staging ring; K tiles (128 keys x 192) and V tiles
+//               (128 keys x 128), each in a 2-deep ring;
+//   warp 1      MMA issuer (one lane): S(j) into S buffer j % 2, then
+//               O += P(j) V(j), then S(j+2);
+//   warps 4-19  four warpgroups; warpgroup c owns key columns 32c .. 32c+31 of
+//               every tile and value columns 32c .. 32c+31 of O. A thread takes
+//               one stacked row; the four threads of a row agree on the row
+//               maximum and sum through shared memory.
+// TMEM (512 columns): S buffers at 0 and 128 (P overwrites the first 64 columns
+// of its S buffer as bf16), O at 256, Q at 384 (96 columns of bf16 pairs). While
+// the softmax of tile j runs, the tensor core computes PV(j-1) and S(j+1). The
+// tensor core runs the MMAs of one thread in issue order, so S(j+2) (issued after
+// PV(j)) never overwrites P(j) too early.
+// The noise head's normalised output H_N is parked in shared memory (bf16) for
+// the epilogues of all g signal heads, so neither H_S nor H_N goes to global
+// memory. O is rescaled only when a row's running maximum grows by more than
+// 2^8.
+#include <limits.h>
 #include <math.h>
 
 #include "kernels.h"
@@ -31,34 +40,44 @@
 namespace gdla {
 namespace {
 
-constexpr int BM = 128;  // query rows per CTA
-constexpr int BN = 64;   // keys per tile
+constexpr int BM = 64;    // query rows per head
+constexpr int BN = 128;   // keys per tile
 constexpr int DN = 128, DR = 64, DV = 128;
-constexpr int Q_BYTES = BM * (DN + DR) * 2;  // 48 KB: 3 boxes of 128 rows x 128 B
-constexpr int K_BYTES = BN * (DN + DR) * 2;  // 24 KB: 3 boxes of 64 keys x 128 B
-constexpr int V_BYTES = BN * DV * 2;         // 16 KB: 2 boxes of 64 keys x 128 B
-constexpr int HN_BYTES = BM * DV * 2;        // 32 KB: parked H_N (bf16)
-constexpr int SMEM_BYTES = 2 * Q_BYTES + 2 * K_BYTES + 2 * V_BYTES + HN_BYTES + 1024;
-constexpr int NTHREADS = 384;
+constexpr int ROWS = 2 * BM;                // stacked rows of a pair
+constexpr int NWG = 4;                      // softmax warpgroups
+constexpr int CW = BN / NWG;                // key columns per softmax thread
+constexpr int QS_BYTES = ROWS * 128;        // 16 KB: one 64-dim chunk of the stacked Q rows
+constexpr int K_CHUNK = BN * 128;           // 16 KB: 128 keys x 64 dims
+constexpr int K_BYTES = 3 * K_CHUNK;        // 48 KB
+constexpr int V_BLOCK = BN * 128;           // 16 KB: 128 keys x 64 value dims
+constexpr int V_BYTES = 2 * V_BLOCK;        // 32 KB
+constexpr int HN_BYTES = BM * DV * 2;       // 16 KB: parked H_N (bf16)
+constexpr int XM_BYTES = 2 * NWG * ROWS * 4;  // 4 KB: per-warpgroup row maxima / sums, double-buffered
+constexpr int OFF_K = 2 * QS_BYTES;
+constexpr int OFF_V = OFF_K + 2 * K_BYTES;
+constexpr int OFF_HN = OFF_V + 2 * V_BYTES;
+constexpr int OFF_XM = OFF_HN + HN_BYTES;
+constexpr int OFF_BARS = OFF_XM + XM_BYTES;
+constexpr int NTHREADS = 128 + 128 * NWG;
+constexpr int kPrefetch = 2;               // K/V tiles prefetched into L2 ahead of the ring loads
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-// TMEM columns of slot s: S buffers at 256 s + 64 buf, O at 256 s + 128.
-__host__ __device__ constexpr uint32_t col_s(int s, int buf) { return 256u * (uint32_t)s + 64u * (uint32_t)buf; }
-__host__ __device__ constexpr uint32_t col_o(int s) { return 256u * (uint32_t)s + 128u; }
+// TMEM columns: S buffer u at 128 u, O at 256, Q at 384 (dim d of a row in column 384 + d/2)
+__host__ __device__ constexpr uint32_t col_s(int u) { return 128u * (uint32_t)u; }
+constexpr uint32_t kColO = 256u, kColQ = 384u;
 
 struct Bars {
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t q_full[2], q_ready[2], s_full[2][2], p_full[2][2], pv_done[2], o_full[2];
-  uint64_t q_empty, hn_ready, mma_done;
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2], q_full[2], q_free[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t pv_done, q_ready, o_full, mx_ready, ml_ready, hn_ready, mma_done;
+  uint32_t tmem_slot;
+  int abort_flag;
+  int skip_cta;
 };
+constexpr int SMEM_BYTES = OFF_BARS + (int)sizeof(Bars);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// parked H_N: row r, 16-byte chunk c (of 16) stored at chunk c ^ (r & 15)
+// parked H_N: row r (of 64), 16-byte chunk c (of 16) stored at chunk c ^ (r & 15)
 __device__ __forceinline__ uint32_t hn_off(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 15)) << 4)); }
 
 }  // namespace
@@ -78,27 +97,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                    const __grid_constant__ CUtensorMap tmKR, const AttnTcArgs a) {
   using namespace sm100;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_sm[2] = {smem, smem + Q_BYTES};
-  uint8_t* k_sm = smem + 2 * Q_BYTES;      // 2 x K_BYTES
-  uint8_t* v_sm = k_sm + 2 * K_BYTES;      // 2 x V_BYTES
-  uint8_t* hn_sm = v_sm + 2 * V_BYTES;     // HN_BYTES
-  __shared__ __align__(8) Bars bars;
-  __shared__ uint32_t tmem_slot;
-  __shared__ volatile int abort_flag;
+  // all shared state lives in the dynamic window, which then starts 1024-byte aligned
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    // the swizzled operand tiles need 1024-byte alignment: report instead of computing garbage
+    if (threadIdx.x == 0 && a.status) {
+      atomicCAS(a.status, 0, (int)GDLA_ERR_CUDA);
+      atomicCAS(a.status + 1, 0, 299);
+    }
+    return;
+  }
+  uint8_t* qs_sm = smem;                   // 2 x QS_BYTES
+  uint8_t* k_sm = smem + OFF_K;            // 2 x K_BYTES
+  uint8_t* v_sm = smem + OFF_V;            // 2 x V_BYTES
+  uint8_t* hn_sm = smem + OFF_HN;          // HN_BYTES
+  float* xm = reinterpret_cast<float*>(smem + OFF_XM);  // [2 buffers][NWG][128 rows]
+  Bars& bars = *reinterpret_cast<Bars*>(smem + OFF_BARS);
+  volatile int& abort_flag = bars.abort_flag;
 
-  if (sm100::earlier_failure(a.status)) return;  // an earlier CTA of this call timed out
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G1 = a.g + 1;
   const int n_pairs = (G1 + 1) / 2;
   const int n_S = a.g * a.n_kv;
-  // heaviest query tiles first across the whole grid
+  // KV-group-major order, heaviest query blocks first within a group: the CTAs
+  // resident at one time stream the K/V of one or two groups, which stay in L2
   const int t = blockIdx.x;
-  const int per_tile = a.n_kv * a.B;
-  const int m_idx = a.n_qtiles - 1 - t / per_tile;
-  const int h = t % a.n_kv;
-  const int b = (t / a.n_kv) % a.B;
+  const int m_idx = a.n_qtiles - 1 - t % a.n_qtiles;
+  const int h = (t / a.n_qtiles) % a.n_kv;
+  const int b = t / (a.n_qtiles * a.n_kv);
   const int m0 = m_idx * BM;
   const int L = a.L;
   const int last_row = min(L - 1, m0 + BM - 1);
@@ -107,7 +133,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int n_tiles = last_row / BN - j_lo + 1;
 
   auto head_of = [&](int hl) { return hl == 0 ? n_S + h : h * a.g + hl - 1; };
-  auto slots_in_pair = [&](int p) { return (2 * p + 1 < G1) ? 2 : 1; };
+  // head in half s of pair p; a pair without a second head repeats the first (its rows are discarded)
+  auto head_in = [&](int p, int s) { return head_of(2 * p + s < G1 ? 2 * p + s : 2 * p); };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -116,38 +143,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(smem_u32(&bars.v_full[i]), 1);
       mbar_init(smem_u32(&bars.v_empty[i]), 1);
       mbar_init(smem_u32(&bars.q_full[i]), 1);
-      mbar_init(smem_u32(&bars.q_ready[i]), 128);
-      mbar_init(smem_u32(&bars.s_full[i][0]), 1);
-      mbar_init(smem_u32(&bars.s_full[i][1]), 1);
-      // one per S buffer: the four warps of a slot may be one tile apart
-      mbar_init(smem_u32(&bars.p_full[i][0]), 128);
-      mbar_init(smem_u32(&bars.p_full[i][1]), 128);
-      mbar_init(smem_u32(&bars.pv_done[i]), 1);
-      mbar_init(smem_u32(&bars.o_full[i]), 1);
+      mbar_init(smem_u32(&bars.q_free[i]), 128 * NWG);
+      mbar_init(smem_u32(&bars.s_full[i]), 1);
+      mbar_init(smem_u32(&bars.p_full[i]), 128 * NWG);
     }
-    mbar_init(smem_u32(&bars.q_empty), 1);
-    mbar_init(smem_u32(&bars.hn_ready), 128);
+    mbar_init(smem_u32(&bars.pv_done), 1);
+    mbar_init(smem_u32(&bars.q_ready), 128 * NWG);
+    mbar_init(smem_u32(&bars.o_full), 1);
+    mbar_init(smem_u32(&bars.mx_ready), 128 * NWG);
+    mbar_init(smem_u32(&bars.ml_ready), 128 * NWG);
+    mbar_init(smem_u32(&bars.hn_ready), 64 * NWG);
     mbar_init(smem_u32(&bars.mma_done), 1);
     fence_mbar_init();
     abort_flag = 0;
+    // an earlier CTA of this call timed out: this one does no work (decided once for the CTA)
+    bars.skip_cta = sm100::earlier_failure(a.status) ? 1 : 0;
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmKV);
     prefetch_tmap(&tmKR);
   }
+  __syncthreads();
+  if (bars.skip_cta) return;
   if (warp == 1) {
-    tmem_alloc(smem_u32(&tmem_slot), 512);
+    tmem_alloc(smem_u32(&bars.tmem_slot), 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_slot;
+  const uint32_t tmem = bars.tmem_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int kc = 0, vc = 0;  // K / V loads issued so far (ring position and phase)
-      int q_issued[2] = {0, 0};
+      int kc = 0, vc = 0, qk = 0;  // K / V / Q-chunk loads issued so far (ring position and phase)
       bool ok = true;
       auto load_k = [&](int jj) -> bool {
         const int sl = kc & 1;
@@ -157,8 +186,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t bar = smem_u32(&bars.k_full[sl]);
         mbar_expect_tx(bar, K_BYTES);
         tma_load_4d(smem_u32(ks), &tmKV, bar, 0, h, key0, b);
-        tma_load_4d(smem_u32(ks + BN * 128), &tmKV, bar, 64, h, key0, b);
-        tma_load_3d(smem_u32(ks + 2 * BN * 128), &tmKR, bar, 0, key0, b);
+        tma_load_4d(smem_u32(ks + K_CHUNK), &tmKV, bar, 64, h, key0, b);
+        tma_load_3d(smem_u32(ks + 2 * K_CHUNK), &tmKR, bar, 0, key0, b);
+        if (jj + kPrefetch < n_tiles) {
+          // bring the tile kPrefetch ahead into L2, so that its ring load later hits
+          const int key1 = key0 + kPrefetch * BN;
+          tma_prefetch_4d(&tmKV, 0, h, key1, b);
+          tma_prefetch_4d(&tmKV, 64, h, key1, b);
+          tma_prefetch_3d(&tmKR, 0, key1, b);
+        }
         ++kc;
         return true;
       };
@@ -170,23 +206,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t bar = smem_u32(&bars.v_full[sl]);
         mbar_expect_tx(bar, V_BYTES);
         tma_load_4d(smem_u32(vs), &tmKV, bar, DN, h, key0, b);
-        tma_load_4d(smem_u32(vs + BN * 128), &tmKV, bar, DN + 64, h, key0, b);
+        tma_load_4d(smem_u32(vs + V_BLOCK), &tmKV, bar, DN + 64, h, key0, b);
+        if (jj + kPrefetch < n_tiles) {
+          const int key1 = key0 + kPrefetch * BN;
+          tma_prefetch_4d(&tmKV, DN, h, key1, b);
+          tma_prefetch_4d(&tmKV, DN + 64, h, key1, b);
+        }
         ++vc;
         return true;
       };
+      // one 64-dim chunk of the pair's stacked Q rows into staging buffer qk % 2
+      auto load_q = [&](int p, int k) -> bool {
+        const int sl = qk & 1;
+        if (qk >= 2 && !mbar_wait(smem_u32(&bars.q_free[sl]), ((qk >> 1) & 1) ^ 1, a.status, 201, &abort_flag)) return false;
+        const uint32_t bar = smem_u32(&bars.q_full[sl]);
+        mbar_expect_tx(bar, QS_BYTES);
+        for (int s = 0; s < 2; ++s)
+          tma_load_4d(smem_u32(qs_sm + sl * QS_BYTES + s * (BM * 128)), &tmQ, bar, k * 64, head_in(p, s), m0, b);
+        ++qk;
+        return true;
+      };
       for (int p = 0; p < n_pairs && ok && !abort_flag; ++p) {
-        if (p > 0 && !mbar_wait(smem_u32(&bars.q_empty), (p - 1) & 1, a.status, 201, &abort_flag)) {
-          ok = false;
-          break;
-        }
-        for (int s = 0; s < slots_in_pair(p); ++s) {
-          const uint32_t bar = smem_u32(&bars.q_full[s]);
-          ++q_issued[s];
-          mbar_expect_tx(bar, Q_BYTES);
-          for (int bx = 0; bx < 3; ++bx)
-            tma_load_4d(smem_u32(q_sm[s] + bx * (BM * 128)), &tmQ, bar, bx * 64, head_of(2 * p + s), m0, b);
-        }
-        ok = load_k(0) && (n_tiles < 2 || load_k(1));
+        // the last Q chunk reuses the staging buffer of the first, which the softmax
+        // warps free only after the previous pair's epilogue: K(0), K(1) go first
+        ok = load_q(p, 0) && load_q(p, 1);
+        // consumption order of the tensor core: S(0), S(1), PV(0), S(2), PV(1), ...
+        if (ok) ok = load_k(0) && (n_tiles < 2 || load_k(1));
+        if (ok) ok = load_q(p, 2);
         for (int jj = 0; jj < n_tiles && ok; ++jj) {
           ok = load_v(jj);
           if (ok && jj + 2 < n_tiles) ok = load_k(jj + 2);
@@ -199,91 +245,65 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_wait(smem_u32(&bars.k_full[c & 1]), (c >> 1) & 1, nullptr, 0);
         for (int c = (vc > 2 ? vc - 2 : 0); c < vc; ++c)
           mbar_wait(smem_u32(&bars.v_full[c & 1]), (c >> 1) & 1, nullptr, 0);
-        for (int q = 0; q < 2; ++q)
-          if (q_issued[q] > 0) mbar_wait(smem_u32(&bars.q_full[q]), (q_issued[q] - 1) & 1, nullptr, 0);
+        for (int c = (qk > 2 ? qk - 2 : 0); c < qk; ++c)
+          mbar_wait(smem_u32(&bars.q_full[c & 1]), (c >> 1) & 1, nullptr, 0);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
-      constexpr uint32_t idO = idesc_bf16_f32(BM, DV, false, true);
+      constexpr uint32_t idS = idesc_bf16_f32(ROWS, BN, false, false);
+      constexpr uint32_t idO = idesc_bf16_f32(ROWS, DV, false, true);
       int kc = 0, vc = 0;
-      int tcnt[2] = {0, 0};  // tiles issued per slot (S buffer index and phase)
+      int sg = 0, pg = 0;  // S / PV tiles issued over the whole CTA (S buffer index and phases)
       bool ok = true;
-      // S_s(next) = Q_s K^T into the slot's next S buffer
-      auto issue_s = [&](int s, uint32_t kbase) {
-        const uint32_t qa = smem_u32(q_sm[s]);
-        const int buf = tcnt[s] & 1;
-#pragma unroll
-        for (int kk = 0; kk < (DN + DR) / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * (BM * 128) + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kbase + (kk >> 2) * (BN * 128) + off, 16, 1024);
-          mma_ss(tmem + col_s(s, buf), ad, bd, idS, kk > 0);
-        }
-        mma_commit(smem_u32(&bars.s_full[s][buf]));
-        ++tcnt[s];
-      };
-      // wait for the next K tile, issue S for every slot, release the K buffer
-      auto s_for_next_k = [&](int ns) -> bool {
-        const int sl = kc & 1;
+      // S(jj) = Q K(jj)^T into S buffer sg % 2 (Q from TMEM); releases the K buffer when done
+      auto issue_s = [&]() -> bool {
+        const int u = sg & 1, sl = kc & 1;
         if (!mbar_wait(smem_u32(&bars.k_full[sl]), (kc >> 1) & 1, a.status, 212, &abort_flag)) return false;
         tc_fence_after();
-        const uint32_t kbase = smem_u32(k_sm + sl * K_BYTES);
-        for (int s = 0; s < ns; ++s) issue_s(s, kbase);
+        const uint32_t kb = smem_u32(k_sm + sl * K_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < (DN + DR) / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(kb + (kk >> 2) * K_CHUNK + (kk & 3) * 32, 16, 1024);
+          mma_ts(tmem + col_s(u), tmem + kColQ + kk * 8, bd, idS, kk > 0);
+        }
+        mma_commit(smem_u32(&bars.s_full[u]));
         mma_commit(smem_u32(&bars.k_empty[sl]));
         ++kc;
+        ++sg;
+        return true;
+      };
+      // O += P(jj) V(jj); releases the V buffer when done
+      auto issue_pv = [&](int jj) -> bool {
+        const int u = pg & 1, sl = vc & 1;
+        if (!mbar_wait(smem_u32(&bars.p_full[u]), (pg >> 1) & 1, a.status, 214, &abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&bars.v_full[sl]), (vc >> 1) & 1, a.status, 213, &abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vb = smem_u32(v_sm + sl * V_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(vb + kk * 2048, V_BLOCK, 1024);
+          mma_ts(tmem + kColO, tmem + col_s(u) + kk * 8, bd, idO, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&bars.pv_done));
+        mma_commit(smem_u32(&bars.v_empty[sl]));
+        ++pg;
+        ++vc;
         return true;
       };
       for (int p = 0; p < n_pairs && ok; ++p) {
-        const int ns = slots_in_pair(p);
-        for (int s = 0; s < ns && ok; ++s) ok = mbar_wait(smem_u32(&bars.q_ready[s]), p & 1, a.status, 211, &abort_flag);
+        // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
+        ok = mbar_wait(smem_u32(&bars.q_ready), p & 1, a.status, 211, &abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const int tbase[2] = {tcnt[0], tcnt[1]};  // S buffer of tile jj of slot s: (tbase[s] + jj) & 1
-        ok = s_for_next_k(ns) && (n_tiles < 2 || s_for_next_k(ns));
+        ok = issue_s() && (n_tiles < 2 || issue_s());
         for (int jj = 0; jj < n_tiles && ok; ++jj) {
-          const int vs = vc & 1;
-          ok = mbar_wait(smem_u32(&bars.v_full[vs]), (vc >> 1) & 1, a.status, 213, &abort_flag);
-          if (!ok) break;
-          const uint32_t vbase = smem_u32(v_sm + vs * V_BYTES);
-          const bool more = jj + 2 < n_tiles;
-          const int ksl = kc & 1;
-          bool k_ready = false;
-          for (int s = 0; s < ns && ok; ++s) {
-            const int tt = tbase[s] + jj;  // this slot's running tile number
-            ok = mbar_wait(smem_u32(&bars.p_full[s][tt & 1]), (tt >> 1) & 1, a.status, 214, &abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t pcol = col_s(s, tt & 1);
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              const uint64_t bd = sdesc_sw128(vbase + kk * 2048, BN * 128, 1024);
-              mma_ts(tmem + col_o(s), tmem + pcol + kk * 8, bd, idO, (jj > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(smem_u32(&bars.pv_done[s]));
-            if (jj + 1 == n_tiles) mma_commit(smem_u32(&bars.o_full[s]));
-            if (more) {
-              // S of tile jj+2 into the buffer whose P the PV above just consumed
-              if (!k_ready) {
-                ok = mbar_wait(smem_u32(&bars.k_full[ksl]), (kc >> 1) & 1, a.status, 215, &abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                k_ready = true;
-              }
-              issue_s(s, smem_u32(k_sm + ksl * K_BYTES));
-            }
-          }
-          if (!ok) break;
-          mma_commit(smem_u32(&bars.v_empty[vs]));
-          ++vc;
-          if (more) {
-            mma_commit(smem_u32(&bars.k_empty[ksl]));
-            ++kc;
-          }
+          ok = issue_pv(jj);
+          if (ok && jj + 2 < n_tiles) ok = issue_s();
         }
-        mma_commit(smem_u32(&bars.q_empty));
+        if (!ok) break;
+        mma_commit(smem_u32(&bars.o_full));
       }
       if (!ok) abort_flag = 1;
       // every MMA this thread issued has completed before TMEM is released
@@ -292,208 +312,244 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------- softmax + epilogue
-    const int s = (warp - 4) >> 2;          // slot
+    const int c = (warp - 4) >> 2;          // column quarter: keys 32c.. of each tile, value dims 32c.. of O
     const int q4 = warp & 3;                // TMEM lane quadrant
-    const int r = q4 * 32 + lane;           // row within the tile
-    const int i = m0 + r;                   // query position
+    const int r = q4 * 32 + lane;           // stacked row = TMEM lane
+    const int half = r >> 6;                // 0: first head of the pair, 1: second
+    const int i = m0 + (r & (BM - 1));      // query position
     const bool row_ok = i < L;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tO = tmem + lane_base + col_o(s);
-    int tc = 0;  // tiles processed by this slot (S buffer index / phase, PV count)
-    for (int p = 0; p < n_pairs; ++p) {
-      const int hl = 2 * p + s;
-      if (hl >= G1) break;
-      const int head = head_of(hl);
-      // RoPE of this row's rotary query part, in place in the swizzled Q tile
-      bool ok = mbar_wait(smem_u32(&bars.q_full[s]), p & 1, a.status, 221, &abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        abort_flag = 1;
-        break;
-      }
-      if (row_ok) {
-        uint8_t* rowp = q_sm[s] + 2 * (BM * 128) + r * 128;
+    const uint32_t tO = tmem + lane_base + kColO + CW * c;
+    const uint32_t tQ = tmem + lane_base + kColQ;
+    int tc = 0;                             // tiles processed over the whole CTA
+    bool failed = false;
+    for (int p = 0; p < n_pairs && !failed; ++p) {
+      const int hl = 2 * p + half;
+      // ---- Q of this row into TMEM: thread c moves dims 16c .. 16c+15 of each
+      // content chunk and rotates dims 8c .. 8c+7 with 32+8c .. 32+8c+7 of the rotary chunk
+      bool ok = true;
+      for (int k = 0; k < 3; ++k) {
+        const int qk = 3 * p + k, sl = qk & 1;
+        ok = mbar_wait(smem_u32(&bars.q_full[sl]), (qk >> 1) & 1, a.status, 221, &abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          failed = true;
+          break;
+        }
+        const uint8_t* rowp = qs_sm + sl * QS_BYTES + r * 128;
         const int sw = r & 7;
-        float x[64];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((c ^ sw) << 4));
-          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&v);
+        if (k < 2) {
+          uint32_t v[8];
+          const uint4 v0 = *reinterpret_cast<const uint4*>(rowp + (((2 * c) ^ sw) << 4));
+          const uint4 v1 = *reinterpret_cast<const uint4*>(rowp + (((2 * c + 1) ^ sw) << 4));
+          v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w;
+          v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+          tmem_st8(tQ + 32 * k + 8 * c, v);
+        } else {
+          const uint4 vl = *reinterpret_cast<const uint4*>(rowp + ((c ^ sw) << 4));
+          const uint4 vh = *reinterpret_cast<const uint4*>(rowp + (((4 + c) ^ sw) << 4));
+          const __nv_bfloat162* hl2 = reinterpret_cast<const __nv_bfloat162*>(&vl);
+          const __nv_bfloat162* hh2 = reinterpret_cast<const __nv_bfloat162*>(&vh);
+          const int pos = row_ok ? i : L - 1;  // rows past the end are discarded; any table row will do
+          const float* cs = a.cos_tab + (long)pos * (DR / 2) + 8 * c;
+          const float* sn = a.sin_tab + (long)pos * (DR / 2) + 8 * c;
+          uint32_t lo[4], hi[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(hv[e]);
-            x[c * 8 + 2 * e] = f.x;
-            x[c * 8 + 2 * e + 1] = f.y;
+            const float2 x = __bfloat1622float2(hl2[e]);
+            const float2 y = __bfloat1622float2(hh2[e]);
+            const float c0 = cs[2 * e], s0 = sn[2 * e], c1 = cs[2 * e + 1], s1 = sn[2 * e + 1];
+            lo[e] = pack_bf16x2(x.x * c0 - y.x * s0, x.y * c1 - y.y * s1);
+            hi[e] = pack_bf16x2(y.x * c0 + x.x * s0, y.y * c1 + x.y * s1);
           }
+          tmem_st4(tQ + 64 + 4 * c, lo);
+          tmem_st4(tQ + 64 + 16 + 4 * c, hi);
         }
-        const float* cs = a.cos_tab + (long)i * (DR / 2);
-        const float* sn = a.sin_tab + (long)i * (DR / 2);
-        float y[64];
-#pragma unroll
-        for (int k = 0; k < DR / 2; ++k) {
-          const float c0 = cs[k], s0 = sn[k];
-          y[k] = x[k] * c0 - x[k + DR / 2] * s0;
-          y[k + DR / 2] = x[k + DR / 2] * c0 + x[k] * s0;
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 v;
-          v.x = pack_bf16x2(y[c * 8 + 0], y[c * 8 + 1]);
-          v.y = pack_bf16x2(y[c * 8 + 2], y[c * 8 + 3]);
-          v.z = pack_bf16x2(y[c * 8 + 4], y[c * 8 + 5]);
-          v.w = pack_bf16x2(y[c * 8 + 6], y[c * 8 + 7]);
-          *reinterpret_cast<uint4*>(rowp + ((c ^ sw) << 4)) = v;
-        }
+        mbar_arrive(smem_u32(&bars.q_free[sl]));
       }
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&bars.q_ready[s]));
+      if (failed) break;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars.q_ready));
 
-      float m_ref = -INFINITY, l_sum = 0.f;
-      bool aborted = false;
+      // ---- online softmax over all key tiles, CW key columns per thread
+      float m_ref = -INFINITY, l_part = 0.f;
       for (int jj = 0; jj < n_tiles; ++jj, ++tc) {
-        const int buf = tc & 1;
-        ok = mbar_wait(smem_u32(&bars.s_full[s][buf]), (tc >> 1) & 1, a.status, 222, &abort_flag);
+        const int u = tc & 1;
+        ok = mbar_wait(smem_u32(&bars.s_full[u]), (tc >> 1) & 1, a.status, 222, &abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
-          aborted = true;
+          failed = true;
           break;
         }
         tc_fence_after();
-        const uint32_t tS = tmem + lane_base + col_s(s, buf);
-        uint32_t sr[64];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        const uint32_t tS = tmem + lane_base + col_s(u);
+        uint32_t sr[CW];
+        tmem_ld32(tS + CW * c, sr);
         tmem_wait_ld();
-        const int key0 = (j_lo + jj) * BN;
-        const bool full_vis = (key0 + BN - 1 <= m0) && (!a.sliding || key0 > m0 + BM - 1 - a.window);
+        const int key0 = (j_lo + jj) * BN + CW * c;
+        const bool full_vis = (key0 + CW - 1 <= m0) && (!a.sliding || key0 > m0 + BM - 1 - a.window);
         if (!full_vis) {
+          // key column e of this quarter is visible iff e_lo <= e <= e_hi
+          const int e_hi = i - key0;
+          const int e_lo = a.sliding ? i - a.window + 1 - key0 : INT_MIN;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int j = key0 + c;
-            // bitwise operators: a select per element, no branches
-            const bool vis = (j <= i) & ((a.sliding == 0) | (j > i - a.window));
-            sr[c] = vis ? sr[c] : __float_as_uint(-INFINITY);
-          }
+          for (int e = 0; e < CW; ++e)
+            sr[e] = ((e <= e_hi) & (e >= e_lo)) ? sr[e] : __float_as_uint(-INFINITY);
         }
-        float mr = -INFINITY;
+        float mq0 = __uint_as_float(sr[0]), mq1 = __uint_as_float(sr[1]);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mr = fmaxf(mr, __uint_as_float(sr[c]));
+        for (int e = 2; e < CW - 2; e += 4) {
+          mq0 = fmax3(mq0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+          mq1 = fmax3(mq1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+        }
+        const float pm = fmax3(fmaxf(mq0, mq1), __uint_as_float(sr[CW - 2]), __uint_as_float(sr[CW - 1]));
+        // the row maximum of the whole tile: exchange with the three threads holding the other columns
+        float* xs = xm + (tc & 1) * (NWG * ROWS);
+        xs[c * ROWS + r] = pm;
+        tc_fence_before();  // this thread's S loads are done before another quarter overwrites them with P
+        mbar_arrive(smem_u32(&bars.mx_ready));
+        ok = mbar_wait(smem_u32(&bars.mx_ready), tc & 1, a.status, 227, &abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        const float mr = fmaxf(fmaxf(xs[r], xs[ROWS + r]), fmaxf(xs[2 * ROWS + r], xs[3 * ROWS + r]));
         const float mx = mr * a.sl2;  // sl2 > 0: the maximum commutes with the scale
         const bool first = (jj == 0);
         const bool need = first || (mx > m_ref + kRescaleThreshold);
         float alpha = 1.f;
         if (need) {
           const float m_new = first ? mx : fmaxf(m_ref, mx);
-          if (!first) alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
-          l_sum *= alpha;
+          if (!first) alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_new);
+          l_part *= alpha;
           m_ref = m_new;
         }
+        uint32_t pk[CW / 2];
+                {
+          const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          const float2 sl2v = make_float2(a.sl2, a.sl2), nmv = make_float2(nm, nm);
+          float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < CW / 2; ++e) {
+            const float2 sv = make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
+            const float2 xv = ffma2(sv, sl2v, nmv);
+            const float2 pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
+            if (e & 1) rs1 = fadd2(rs1, pv);
+            else rs0 = fadd2(rs0, pv);
+            pk[e] = pack_bf16x2(pv.x, pv.y);
+          }
+          l_part += (rs0.x + rs0.y) + (rs1.x + rs1.y);
+        }
+        // P columns 16 c .. 16 c + 15 overwrite S columns that every quarter loaded before the exchange
+        tmem_st16(tS + (CW / 2) * c, pk);
         if (!first && __any_sync(0xffffffffu, need)) {
-          // O holds tiles < jj once this slot's previous PV has landed: PV
-          // number tc (1-based) -> completion parity (tc - 1) & 1
-          ok = mbar_wait(smem_u32(&bars.pv_done[s]), (uint32_t)(tc - 1) & 1, a.status, 226, &abort_flag);
+          // this quarter of O must hold every earlier tile before it is rescaled and PV(jj)
+          // adds to it: PV(jj-1) is the CTA's PV number tc - 1; PV(jj-2) preceded S(jj) in
+          // issue order, so the wait is within one phase
+          ok = mbar_wait(smem_u32(&bars.pv_done), (tc - 1) & 1, a.status, 226, &abort_flag);
           if (!__all_sync(0xffffffffu, ok)) {
-            aborted = true;
+            failed = true;
             break;
           }
           tc_fence_after();
-#pragma unroll 1
-          for (int ch = 0; ch < DV / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tO + ch * 32, o);
-            tmem_wait_ld();
+          uint32_t o[32];
+          tmem_ld32(tO, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tO + ch * 32, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO, o);
         }
-        const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        uint32_t pk[32];
-        float rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), a.sl2, nm));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), a.sl2, nm));
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        l_sum += rs;
-        tmem_st32(tS, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars.p_full[s][buf]));
+        mbar_arrive(smem_u32(&bars.p_full[u]));
       }
-      if (aborted) {
-        abort_flag = 1;
-        break;
-      }
+      if (failed) break;
+
       // ---------------------------------------------------------- epilogue
-      ok = mbar_wait(smem_u32(&bars.o_full[s]), p & 1, a.status, 223, &abort_flag);
+      ok = mbar_wait(smem_u32(&bars.o_full), p & 1, a.status, 223, &abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
-        abort_flag = 1;
+        failed = true;
         break;
       }
       tc_fence_after();
-      const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      // row sum: add the other quarters' partial sums (same running maximum everywhere).
+      // Slot tc & 1 was last read two tiles ago.
+      {
+        float* xs = xm + (tc & 1) * (NWG * ROWS);
+        xs[c * ROWS + r] = l_part;
+        mbar_arrive(smem_u32(&bars.ml_ready));
+        ok = mbar_wait(smem_u32(&bars.ml_ready), p & 1, a.status, 225, &abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          failed = true;
+          break;
+        }
+        l_part = (xs[r] + xs[ROWS + r]) + (xs[2 * ROWS + r] + xs[3 * ROWS + r]);
+      }
+      const float inv = l_part > 0.f ? 1.f / l_part : 0.f;
+      const int cbase = CW * c;          // this warpgroup finishes value columns [cbase, cbase + 32)
+      const bool real = hl < G1;         // the second half of a short last pair is discarded
+
       if (hl == 0) {
         // noise head: park the normalised H_N (bf16) for every signal head
 #pragma unroll 1
-        for (int ch = 0; ch < DV / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tO + ch * 32, o);
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t o[16];
+          tmem_ld16(tO + 16 * ch, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(hn_sm + hn_off(r, ch * 4 + q)) = v;
+          for (int q = 0; q < 2; ++q) {
+            uint4 pv;
+            pv.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+            pv.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+            pv.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+            pv.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+            *reinterpret_cast<uint4*>(hn_sm + hn_off(r & (BM - 1), (cbase + 16 * ch) / 8 + q)) = pv;
           }
         }
         mbar_arrive(smem_u32(&bars.hn_ready));
-      } else if (p == 0) {
+      } else if (real) {
+        // signal head: D = H_S - lambda H_N, Y = sigmoid(G) D
         ok = mbar_wait(smem_u32(&bars.hn_ready), 0, a.status, 224, &abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
-          abort_flag = 1;
+          failed = true;
           break;
         }
-      }
-      if (hl > 0) {
-        const int sh = head;  // signal head index
+        const int sh = head_of(hl);  // signal head index
         const long tok = (long)b * L + i;
         const float lam = row_ok ? sigmoidf_(a.lam[tok * n_S + sh]) : 0.f;
-        const __nv_bfloat16* gp = a.gate + (tok * n_S + sh) * DV;
-        __nv_bfloat16* op = a.out + (tok * n_S + sh) * DV;
+        const __nv_bfloat16* gp = a.gate + (tok * n_S + sh) * DV + cbase;
+        __nv_bfloat16* op = a.out + (tok * n_S + sh) * DV + cbase;
 #pragma unroll 1
-        for (int ch = 0; ch < DV / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(tO + ch * 32, o);
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t o[16];
+          tmem_ld16(tO + 16 * ch, o);
           tmem_wait_ld();
           if (row_ok) {
-            uint4 gv[4], hv[4];
+            uint4 gv[2], hv[2];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              gv[q] = reinterpret_cast<const uint4*>(gp + ch * 32)[q];
-              hv[q] = *reinterpret_cast<const uint4*>(hn_sm + hn_off(r, ch * 4 + q));
+            for (int q = 0; q < 2; ++q) {
+              gv[q] = reinterpret_cast<const uint4*>(gp + ch * 16)[q];
+              hv[q] = *reinterpret_cast<const uint4*>(hn_sm + hn_off(r & (BM - 1), (cbase + 16 * ch) / 8 + q));
             }
             const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(hv);
-            uint4 ov[4];
+            uint4 ov[2];
             uint32_t* ow = reinterpret_cast<uint32_t*>(ov);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float2 gf = __bfloat1622float2(g2[c]);
-              const float2 hf = __bfloat1622float2(h2[c]);
-              const float d0 = __uint_as_float(o[2 * c]) * inv - lam * hf.x;
-              const float d1 = __uint_as_float(o[2 * c + 1]) * inv - lam * hf.y;
-              ow[c] = pack_bf16x2(sigmoidf_(gf.x) * d0, sigmoidf_(gf.y) * d1);
+            for (int e = 0; e < 8; ++e) {
+              const float2 gf = __bfloat1622float2(g2[e]);
+              const float2 hf = __bfloat1622float2(h2[e]);
+              const float y0 = __uint_as_float(o[2 * e]) * inv;
+              const float y1 = __uint_as_float(o[2 * e + 1]) * inv;
+              ow[e] = pack_bf16x2(sigmoidf_(gf.x) * (y0 - lam * hf.x), sigmoidf_(gf.y) * (y1 - lam * hf.y));
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(op + ch * 32)[q] = ov[q];
+            for (int q = 0; q < 2; ++q) reinterpret_cast<uint4*>(op + ch * 16)[q] = ov[q];
           }
         }
       }
     }
+    if (failed) abort_flag = 1;
   }
   tc_fence_before();
   __syncthreads();
