@@ -127,6 +127,8 @@ PREFILL = {
                               B=1, L=128, d_c=64, d_R=16, n_kv=4, d_n=32, d_v=32, g=2, d_q=64, dtype="fp32"),
     "b4_l4k_g2": PrefillShape("bf16 prefill, causal, B=4 L=4096 g=2", B=4, L=4096, g=2),
     "b1_l32k_g3": PrefillShape("bf16 prefill, causal, B=1 L=32768 g=3", B=1, L=32768, g=3),
+    # the same kernel configuration at a size a full counter capture replays quickly
+    "b2_l8k_g3": PrefillShape("bf16 prefill, causal, B=2 L=8192 g=3", B=2, L=8192, g=3),
     "b2_l64k_swa4k": PrefillShape("bf16 prefill, sliding window W=4096, B=2 L=65536 g=2", B=2, L=65536, g=2,
                                   mask="sliding", window=4096),
 }
