@@ -8,8 +8,8 @@
 //   sum_j p_j (c_hat_j W_UV) = (sum_j p_j c_hat_j) W_UV (latent weighted sum)
 // Kernels: decode_absorb (q_abs = W_UK q_nope, RoPE of q_rope at position
 // seqlen-1), decode_split (split-KV online softmax over the cache, partial
-// results per split), decode_merge (log-sum-exp merge of the splits) and
-// decode_combine (W_UV, differential and gate epilogue).
+// results per split) and decode_combine (log-sum-exp merge of the splits, W_UV,
+// differential and gate epilogue).
 #include <math.h>
 
 #include "common.cuh"
@@ -17,61 +17,100 @@
 
 namespace gdla {
 
-// Rows per combine block: max(1, 12 / (g+1)) sequences times the g+1 heads of
-// a KV group; one W_UV slice is staged once per block for all of them.
-constexpr int MAX_ROWS = 12;  // rows (sequence, head of the group) per combine block
-// Absorb blocks: KV group x 64 latent rows x ABS_SEQ sequences.
-constexpr int ABS_ROWS = 64;
-constexpr int ABS_SEQ = 16;
+// Absorb blocks: KV group x 128 latent rows x (up to 48 query rows = sequences x heads of the group).
+constexpr int ABS_C = 128;   // latent rows per block: 32 threads x 4
+constexpr int ABS_R = 48;    // query rows per block: 8 warps x 6
+// Combine blocks: KV group x (up to 24 query rows); 32 threads x 4 value columns, 8 warps x 3 rows.
+constexpr int CMB_R = 24;
+constexpr int CMB_KC = 64;   // latent rows of W_UV staged per step
+
+__host__ __device__ inline int absorb_seqs(int g) { return max(1, ABS_R / (g + 1)); }
+__host__ __device__ inline int combine_seqs(int g) { return max(1, CMB_R / (g + 1)); }
 
 // q_abs[b, head, c] = sum_n W_UKV[c, h*(d_nope+d_v) + n] * q_nope[b, head, n] for the
 // g+1 heads of KV group h, and RoPE of their rotary parts at position seqlen-1.
-// Block (KV group h, 64 latent rows, up to 16 sequences): the W_UK rows and the
-// query rows are staged in shared memory with coalesced loads, then every
-// thread computes (latent row, query row) dot products from shared memory.
+// Block (KV group h, 128 latent rows, absorb_seqs(g) sequences): W_UK (transposed) and
+// the query rows are staged in shared memory; every thread accumulates a 4 (latent
+// rows) x 6 (query rows) tile, so each shared load feeds several FMAs.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
-  const int h = blockIdx.x, c0 = blockIdx.y * ABS_ROWS, b0 = blockIdx.z * ABS_SEQ;
-  const int nb = min(ABS_SEQ, p.B - b0);
+  const int h = blockIdx.x, c0 = blockIdx.y * ABS_C;
+  const int spb = absorb_seqs(p.g), b0 = blockIdx.z * spb;
+  const int nb = min(spb, p.B - b0);
   const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1;
   const int dqk = p.d_nope + p.d_rope, ncol = p.n_kv * (p.d_nope + p.d_v), DN = p.d_nope;
-  const int DNP = DN + 1;  // padded row (bank-conflict free column reads)
-  const int nrows = min(ABS_ROWS, p.d_c - c0);
+  const int nrows = min(ABS_C, p.d_c - c0);
   const T* q = reinterpret_cast<const T*>(p.q);
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   extern __shared__ float sm[];
-  float* ws = sm;                   // [ABS_ROWS][DNP]
-  float* qs = ws + ABS_ROWS * DNP;  // [R][DN]
-  constexpr int VEC = 16 / (int)sizeof(T);  // elements per 16-byte load
+  constexpr int WT = ABS_C + 4;          // padded row of the transposed W_UK tile
+  float* wt = sm;                        // [DN][WT]: wt[n][c] = W_UK[c0 + c][n]
+  float* qs = wt + DN * WT;              // [ABS_R][DN]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int VEC = 16 / (int)sizeof(T);
   const int vrow = DN / VEC;
-#pragma unroll 4
-  for (int e = threadIdx.x; e < nrows * vrow; e += blockDim.x) {
-    const int cr = e / vrow, v = e % vrow;
-    const uint4 x = *reinterpret_cast<const uint4*>(w + (long)(c0 + cr) * ncol + (long)h * (p.d_nope + p.d_v) + v * VEC);
-    const T* xe = reinterpret_cast<const T*>(&x);
+  for (int e = tid; e < ABS_C * vrow; e += blockDim.x) {
+    const int cr = e % ABS_C, v = e / ABS_C;  // consecutive threads: consecutive latent rows (conflict-free stores)
+    float f[VEC];
+    if (cr < nrows) {
+      const uint4 x = *reinterpret_cast<const uint4*>(w + (long)(c0 + cr) * ncol + (long)h * (p.d_nope + p.d_v) + v * VEC);
+      const T* xe = reinterpret_cast<const T*>(&x);
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) ws[cr * DNP + v * VEC + i] = to_f(xe[i]);
+      for (int i = 0; i < VEC; ++i) f[i] = to_f(xe[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) f[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) wt[(v * VEC + i) * WT + cr] = f[i];
   }
-#pragma unroll 4
-  for (int e = threadIdx.x; e < R * vrow; e += blockDim.x) {
-    const int r = e / vrow, v = e % vrow, bl = r / G1, u = r % G1;
-    const int head = u < p.g ? h * p.g + u : n_S + h;
-    const uint4 x = *reinterpret_cast<const uint4*>(q + ((long)(b0 + bl) * H_q + head) * dqk + v * VEC);
-    const T* xe = reinterpret_cast<const T*>(&x);
+  for (int e = tid; e < ABS_R * vrow; e += blockDim.x) {
+    const int r = e / vrow, v = e % vrow;
+    float f[VEC];
+    if (r < R) {
+      const int bl = r / G1, u = r % G1;
+      const int head = u < p.g ? h * p.g + u : n_S + h;
+      const uint4 x = *reinterpret_cast<const uint4*>(q + ((long)(b0 + bl) * H_q + head) * dqk + v * VEC);
+      const T* xe = reinterpret_cast<const T*>(&x);
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) qs[r * DN + v * VEC + i] = to_f(xe[i]);
+      for (int i = 0; i < VEC; ++i) f[i] = to_f(xe[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) f[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) qs[r * DN + v * VEC + i] = f[i];
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < nrows * R; e += blockDim.x) {
-    const int cr = e % nrows, r = e / nrows;  // consecutive threads: consecutive latent rows
-    const float* wr = ws + cr * DNP;
-    const float* qr = qs + r * DN;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < DN; ++k) acc = fmaf(wr[k], qr[k], acc);
-    const int bl = r / G1, u = r % G1;
-    const int head = u < p.g ? h * p.g + u : n_S + h;
-    p.q_abs[((long)(b0 + bl) * H_q + head) * p.d_c + c0 + cr] = acc;
+  // thread: latent rows 4*lane .. +3, query rows 6*warp .. +5
+  float acc[6][4];
+#pragma unroll
+  for (int i = 0; i < 6; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  const float* qw = qs + (6 * warp) * DN;
+#pragma unroll 4
+  for (int n = 0; n < DN; ++n) {
+    const float4 wv = *reinterpret_cast<const float4*>(wt + n * WT + 4 * lane);
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      const float qv = qw[i * DN + n];
+      acc[i][0] = fmaf(wv.x, qv, acc[i][0]);
+      acc[i][1] = fmaf(wv.y, qv, acc[i][1]);
+      acc[i][2] = fmaf(wv.z, qv, acc[i][2]);
+      acc[i][3] = fmaf(wv.w, qv, acc[i][3]);
+    }
+  }
+  if (4 * lane < nrows) {
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      const int r = 6 * warp + i;
+      if (r >= R) break;
+      const int bl = r / G1, u = r % G1;
+      const int head = u < p.g ? h * p.g + u : n_S + h;
+      *reinterpret_cast<float4*>(p.q_abs + ((long)(b0 + bl) * H_q + head) * p.d_c + c0 + 4 * lane) =
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    }
   }
   // RoPE of the rotary query parts at position seqlen-1 (once per block row 0)
   if (blockIdx.y != 0) return;
@@ -199,118 +238,125 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
   }
 }
 
-// Merge of the split partials of one (sequence, head): O_lat = sum_s w_s O_s with
-// w_s = exp2(m_s - M) / sum_s' exp2(m_s' - M) l_s'. One block per (sequence,
-// head); the result goes to o_lat [B, H_q, d_c] (the absorbed-query buffer,
-// which the split pass no longer needs).
-__global__ void __launch_bounds__(256) decode_merge_kernel(DecodeParams p) {
-  const int head = blockIdx.x, b = blockIdx.y;
-  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, NS = p.n_splits, d_c = p.d_c;
-  __shared__ float wgt[256];
-  __shared__ float red[2];
-  const int tid = threadIdx.x;
-  if (tid < 32) {
-    float M = -INFINITY;
-    for (int s = tid; s < NS; s += 32) M = fmaxf(M, p.part_ml[(((long)b * NS + s) * H_q + head) * 2]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float den = 0.f;
-    for (int s = tid; s < NS; s += 32) {
-      const float* ml = p.part_ml + (((long)b * NS + s) * H_q + head) * 2;
-      const float wv = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
-      wgt[s] = wv;
-      den += wv * ml[1];
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (tid == 0) red[0] = den > 0.f ? 1.f / den : 0.f;
-  }
-  __syncthreads();
-  const float inv = red[0];
-  const float* src = p.part_o + ((long)b * NS * H_q + head) * d_c;
-  for (int c = tid; c < d_c; c += blockDim.x) {
-    float acc = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < NS; ++s) acc = fmaf(wgt[s], src[(long)s * H_q * d_c + c], acc);
-    p.q_abs[((long)b * H_q + head) * d_c + c] = acc * inv;
-  }
-}
-
-// Rows (sequence, head of the group) per combine block and the W_UV slice
-// staged once per block: max(1, 12 / (g+1)) sequences x (g+1) heads.
-__host__ __device__ inline int combine_seqs(int g) { return max(1, 12 / (g + 1)); }
-
-// H = O_lat W_UV for the g+1 heads of KV group h, then D = H_S - sigmoid(lam) H_N
-// and Y = sigmoid(G) D. Block (KV group h, chunk of sequences).
+// Merge of the split partials and the output epilogue, for the g+1 heads of KV group h
+// and combine_seqs(g) sequences per block:
+//   O_lat = sum_s w_s O_s with w_s = exp2(m_s - M) / sum_s' exp2(m_s' - M) l_s'
+//   (log-sum-exp merge of the split-KV partials),
+//   H = O_lat W_UV, D = H_S - sigmoid(lam) H_N, Y = sigmoid(G) D.
+// W_UV is staged CMB_KC latent rows at a time; every thread accumulates a
+// 3 (query rows) x 4 (value columns) tile of H.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   const int spb = combine_seqs(p.g);
   const int h = blockIdx.x, b0 = blockIdx.y * spb;
   const int nb = min(spb, p.B - b0);
-  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1, RM = spb * G1;
+  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1, NS = p.n_splits;
   const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v);
   extern __shared__ float sm[];
-  float* olat = sm;                        // [R][d_c]
-  float* hv = olat + RM * d_c;             // [R][DV]
-  T* wsm = reinterpret_cast<T*>(hv + RM * DV);  // [d_c][DV] W_UV slice
+  float* olat = sm;                              // [CMB_R][d_c]
+  float* hsm = olat + CMB_R * d_c;               // [CMB_R][DV]
+  float* wgt = hsm + CMB_R * DV;                 // [CMB_R][NS] merge weights (scaled by 1 / denominator)
+  T* wch = reinterpret_cast<T*>(wgt + CMB_R * NS);  // [CMB_KC][DV] staged W_UV rows
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   const T* gate = reinterpret_cast<const T*>(p.gate);
   T* out = reinterpret_cast<T*>(p.out);
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  auto head_of_row = [&](int r) { const int u = r % G1; return u < p.g ? h * p.g + u : n_S + h; };
+
+  // ---- merge weights: one warp per query row
+  for (int r = warp; r < R; r += 8) {
+    const int b = b0 + r / G1, head = head_of_row(r);
+    const float* ml = p.part_ml + ((long)b * NS * H_q + head) * 2;
+    float M = -INFINITY;
+    for (int sp = lane; sp < NS; sp += 32) M = fmaxf(M, ml[(long)sp * H_q * 2]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+    for (int sp = lane; sp < NS; sp += 32) {
+      const float m = ml[(long)sp * H_q * 2], l = ml[(long)sp * H_q * 2 + 1];
+      const float wv = (m == -INFINITY) ? 0.f : exp2f(m - M);
+      wgt[r * NS + sp] = wv;
+      den += wv * l;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    __syncwarp();
+    for (int sp = lane; sp < NS; sp += 32) wgt[r * NS + sp] *= inv;
+  }
+  __syncthreads();
+  // ---- O_lat rows (float4 over the latent dimension)
+  const int c4 = d_c / 4;
+  for (int e = tid; e < R * c4; e += blockDim.x) {
+    const int r = e / c4, v = e % c4;
+    const int b = b0 + r / G1, head = head_of_row(r);
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + ((long)b * NS * H_q + head) * d_c) + v;
+    const long stride4 = (long)H_q * d_c / 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < NS; ++sp) {
+      const float wv = wgt[r * NS + sp];
+      const float4 x = src[sp * stride4];
+      acc.x = fmaf(wv, x.x, acc.x);
+      acc.y = fmaf(wv, x.y, acc.y);
+      acc.z = fmaf(wv, x.z, acc.z);
+      acc.w = fmaf(wv, x.w, acc.w);
+    }
+    reinterpret_cast<float4*>(olat + r * d_c)[v] = acc;
+  }
+  // ---- H = O_lat W_UV: thread rows 3*warp .. +2, value columns 4*lane .. +3
+  float acc[3][4];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
   constexpr int VEC = 16 / (int)sizeof(T);
   const int per_row = DV / VEC;
-#pragma unroll 8
-  for (int e = tid; e < d_c * per_row; e += blockDim.x) {
-    const int c = e / per_row, v = e % per_row;
-    *reinterpret_cast<uint4*>(wsm + c * DV + v * VEC) =
-        *reinterpret_cast<const uint4*>(w + (long)c * ncol + (long)h * (p.d_nope + DV) + p.d_nope + v * VEC);
-  }
+  const bool col_ok = 4 * lane < DV;
+  for (int k0 = 0; k0 < d_c; k0 += CMB_KC) {
+    __syncthreads();  // O_lat written (first step) / previous W_UV rows consumed
+    for (int e = tid; e < CMB_KC * per_row; e += blockDim.x) {
+      const int c = e / per_row, v = e % per_row;
+      *reinterpret_cast<uint4*>(wch + c * DV + v * VEC) = *reinterpret_cast<const uint4*>(
+          w + (long)(k0 + c) * ncol + (long)h * (p.d_nope + DV) + p.d_nope + v * VEC);
+    }
+    __syncthreads();
+    if (col_ok) {
 #pragma unroll 4
-  for (int e = tid; e < R * (d_c / 4); e += blockDim.x) {
-    const int r = e / (d_c / 4), v = e % (d_c / 4), u = r % G1;
-    const int head = u < p.g ? h * p.g + u : n_S + h;
-    reinterpret_cast<float4*>(olat + r * d_c)[v] =
-        reinterpret_cast<const float4*>(p.q_abs + ((long)(b0 + r / G1) * H_q + head) * d_c)[v];
-  }
-  __syncthreads();
-  // hv[r][n] = sum_c olat[r][c] W_UV[c][n]: thread column n, rows rg, rg+RG, ...
-  const int RG = blockDim.x / DV;
-  const int n = tid % DV, rg = tid / DV;
-  if (rg < RG) {
-    float acc[MAX_ROWS];
+      for (int c = 0; c < CMB_KC; ++c) {
+        float wv[4];
 #pragma unroll
-    for (int i = 0; i < MAX_ROWS; ++i) acc[i] = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < d_c; ++c) {
-      const float wv = to_f(wsm[c * DV + n]);
+        for (int j = 0; j < 4; ++j) wv[j] = to_f(wch[c * DV + 4 * lane + j]);
 #pragma unroll
-      for (int i = 0; i < MAX_ROWS; ++i) {
-        const int r = rg + i * RG;
-        if (r < R) acc[i] = fmaf(olat[r * d_c + c], wv, acc[i]);
+        for (int i = 0; i < 3; ++i) {
+          const float ov = olat[(3 * warp + i) * d_c + k0 + c];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ov, wv[j], acc[i][j]);
+        }
       }
     }
+  }
+  if (col_ok) {
 #pragma unroll
-    for (int i = 0; i < MAX_ROWS; ++i) {
-      const int r = rg + i * RG;
-      if (r < R) hv[r * DV + n] = acc[i];
-    }
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) hsm[(3 * warp + i) * DV + 4 * lane + j] = acc[i][j];
   }
   __syncthreads();
+  // ---- differential and gate
   for (int e = tid; e < nb * p.g * DV; e += blockDim.x) {
     const int bl = e / (p.g * DV), u = (e / DV) % p.g, nn = e % DV;
     const int b = b0 + bl, sh = h * p.g + u;
     const float lam = sigmoidf_(p.lam[(long)b * n_S + sh]);
     const long idx = ((long)b * n_S + sh) * DV + nn;
-    const float d = hv[(bl * G1 + u) * DV + nn] - lam * hv[(bl * G1 + p.g) * DV + nn];
+    const float d = hsm[(bl * G1 + u) * DV + nn] - lam * hsm[(bl * G1 + p.g) * DV + nn];
     out[idx] = from_f<T>(sigmoidf_(to_f(gate[idx])) * d);
   }
 }
 
 cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
-  dim3 grid((unsigned)p.n_kv, (unsigned)((p.d_c + ABS_ROWS - 1) / ABS_ROWS),
-            (unsigned)((p.B + ABS_SEQ - 1) / ABS_SEQ));
-  const size_t smem =
-      sizeof(float) * ((size_t)ABS_ROWS * (p.d_nope + 1) + (size_t)ABS_SEQ * (p.g + 1) * p.d_nope);
+  const int spb = absorb_seqs(p.g);
+  dim3 grid((unsigned)p.n_kv, (unsigned)((p.d_c + ABS_C - 1) / ABS_C), (unsigned)((p.B + spb - 1) / spb));
+  const size_t smem = sizeof(float) * ((size_t)p.d_nope * (ABS_C + 4) + (size_t)ABS_R * p.d_nope);
   cudaError_t e;
   if (dt == GDLA_BF16) {
     auto k = decode_absorb_kernel<__nv_bfloat16>;
@@ -364,14 +410,12 @@ cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaS
 }
 
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
-  decode_merge_kernel<<<dim3((unsigned)(p.n_kv * (p.g + 1)), (unsigned)p.B), 256, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const size_t esz = dt == GDLA_BF16 ? 2 : 4;
   const int spb = combine_seqs(p.g);
-  const size_t RM = (size_t)spb * (p.g + 1);
-  const size_t smem = sizeof(float) * (RM * p.d_c + RM * p.d_v) + esz * (size_t)p.d_c * p.d_v;
+  const size_t smem = sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * p.d_v + (size_t)CMB_R * p.n_splits) +
+                      esz * (size_t)CMB_KC * p.d_v;
   dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + spb - 1) / spb));
+  cudaError_t e;
   if (dt == GDLA_BF16) {
     auto k = decode_combine_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
