@@ -20,8 +20,9 @@ namespace gdla {
 // Absorb blocks: KV group x 128 latent rows x (up to 48 query rows = sequences x heads of the group).
 constexpr int ABS_C = 128;   // latent rows per block: 32 threads x 4
 constexpr int ABS_R = 48;    // query rows per block: 8 warps x 6
-// Combine blocks: KV group x (up to 24 query rows); 32 threads x 4 value columns, 8 warps x 3 rows.
-constexpr int CMB_R = 24;
+// Combine blocks: KV group x (up to 16 query rows); 32 threads x 4 value columns, 8 warps x 2 rows.
+constexpr int CMB_R = 16;
+constexpr int CMB_RPW = CMB_R / 8;  // query rows per warp
 constexpr int CMB_KC = 64;   // latent rows of W_UV staged per step
 
 __host__ __device__ inline int absorb_seqs(int g) { return max(1, ABS_R / (g + 1)); }
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
 //   (log-sum-exp merge of the split-KV partials),
 //   H = O_lat W_UV, D = H_S - sigmoid(lam) H_N, Y = sigmoid(G) D.
 // W_UV is staged CMB_KC latent rows at a time; every thread accumulates a
-// 3 (query rows) x 4 (value columns) tile of H.
+// CMB_RPW (query rows) x 4 (value columns) tile of H.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   const int spb = combine_seqs(p.g);
@@ -292,9 +293,25 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     const int b = b0 + r / G1, head = head_of_row(r);
     const float4* src = reinterpret_cast<const float4*>(p.part_o + ((long)b * NS * H_q + head) * d_c) + v;
     const long stride4 = (long)H_q * d_c / 4;
+    const float* wr = wgt + r * NS;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < NS; ++sp) {
-      const float wv = wgt[r * NS + sp];
+    int sp = 0;
+    // four splits' partials in flight at a time (the loads are independent)
+    for (; sp + 4 <= NS; sp += 4) {
+      float4 x[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) x[q] = src[(sp + q) * stride4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float wv = wr[sp + q];
+        acc.x = fmaf(wv, x[q].x, acc.x);
+        acc.y = fmaf(wv, x[q].y, acc.y);
+        acc.z = fmaf(wv, x[q].z, acc.z);
+        acc.w = fmaf(wv, x[q].w, acc.w);
+      }
+    }
+    for (; sp < NS; ++sp) {
+      const float wv = wr[sp];
       const float4 x = src[sp * stride4];
       acc.x = fmaf(wv, x.x, acc.x);
       acc.y = fmaf(wv, x.y, acc.y);
@@ -303,10 +320,10 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     }
     reinterpret_cast<float4*>(olat + r * d_c)[v] = acc;
   }
-  // ---- H = O_lat W_UV: thread rows 3*warp .. +2, value columns 4*lane .. +3
-  float acc[3][4];
+  // ---- H = O_lat W_UV: thread rows CMB_RPW*warp .., value columns 4*lane .. +3
+  float acc[CMB_RPW][4];
 #pragma unroll
-  for (int i = 0; i < 3; ++i)
+  for (int i = 0; i < CMB_RPW; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
   constexpr int VEC = 16 / (int)sizeof(T);
@@ -327,8 +344,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) wv[j] = to_f(wch[c * DV + 4 * lane + j]);
 #pragma unroll
-        for (int i = 0; i < 3; ++i) {
-          const float ov = olat[(3 * warp + i) * d_c + k0 + c];
+        for (int i = 0; i < CMB_RPW; ++i) {
+          const float ov = olat[(CMB_RPW * warp + i) * d_c + k0 + c];
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ov, wv[j], acc[i][j]);
         }
@@ -337,9 +354,9 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   }
   if (col_ok) {
 #pragma unroll
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < CMB_RPW; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) hsm[(3 * warp + i) * DV + 4 * lane + j] = acc[i][j];
+      for (int j = 0; j < 4; ++j) hsm[(CMB_RPW * warp + i) * DV + 4 * lane + j] = acc[i][j];
   }
   __syncthreads();
   // ---- differential and gate
