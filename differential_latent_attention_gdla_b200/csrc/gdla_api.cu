@@ -32,7 +32,6 @@ gdla_status common_dims(int B, int L, int d_c, int d_rope, int n_kv, int d_nope,
   if (dtype != GDLA_BF16 && dtype != GDLA_FP32) return GDLA_ERR_INVALID_ARG;
   if (n_noise != n_kv) return GDLA_ERR_UNSUPPORTED;
   if (g > 8 || !head_dims_ok(d_nope, d_rope, d_v) || !latent_ok(d_c)) return GDLA_ERR_UNSUPPORTED;
-  if ((long)n_kv * (g + 1) > 64) return GDLA_ERR_UNSUPPORTED;
   return GDLA_OK;
 }
 
@@ -130,6 +129,7 @@ gdla_status validate_decode(const gdla_decode_args* a) {
   gdla_status st = common_dims(a->B, a->T_max, a->d_c, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_noise,
                                a->g, a->dtype);
   if (st != GDLA_OK) return st;
+  if ((long)a->n_kv * (a->g + 1) > 64) return GDLA_ERR_UNSUPPORTED;  // query heads of one decode block
   if (a->mask != GDLA_MASK_CAUSAL && a->mask != GDLA_MASK_SLIDING) return GDLA_ERR_INVALID_ARG;
   if (a->mask == GDLA_MASK_SLIDING && a->window < 1) return GDLA_ERR_INVALID_ARG;
   if (a->rope_max_pos < a->T_max) return GDLA_ERR_INVALID_ARG;

@@ -61,8 +61,9 @@ typedef enum { GDLA_BF16 = 0, GDLA_FP32 = 1 } gdla_dtype;
  * floor(i/g) and subtracts noise head floor(i/g) (Repeat_g as
  * repeat-interleave). Supported head shapes (d_nope, d_rope, d_v):
  * (128, 64, 128), (64, 32, 64), (32, 16, 32); d_c in {64, 128, 256, 512};
- * 1 <= g <= 8 and n_kv * (g + 1) <= 64 query heads. Other sizes return
- * GDLA_ERR_UNSUPPORTED. The tensor-core kernels serve bf16: prefill with
+ * 1 <= g <= 8; decode additionally n_kv * (g + 1) <= 64 query heads (prefill
+ * takes any head count, e.g. the report's 16 KV heads with g = 4, 80 heads).
+ * Other sizes return GDLA_ERR_UNSUPPORTED. The tensor-core kernels serve bf16: prefill with
  * (128, 64, 128) heads, decode with d_c = 512, d_rope = 64 and at most 48
  * query heads; every other supported shape runs on the CUDA-core kernels. */
 

@@ -101,6 +101,14 @@ def test_prefill_validation_rejects_before_launch(lib):
     assert lib.gdla_prefill(None, None) == E
 
 
+def test_prefill_accepts_eighty_heads(lib):
+    # the report's attention shape (16 KV heads, g = 4: 64 signal + 16 noise heads) is a
+    # valid prefill; sizing needs no launch
+    a = good_prefill()
+    a.g = 4
+    assert lib.gdla_prefill_workspace_size(ctypes.byref(a)) > 0
+
+
 def test_prefill_workspace_size_is_monotone(lib):
     a = good_prefill()
     s1 = lib.gdla_prefill_workspace_size(ctypes.byref(a))
@@ -125,6 +133,7 @@ def test_decode_validation_rejects_before_launch(lib):
     for mut, want in ((lambda a: setattr(a, "B", 0), E), (lambda a: setattr(a, "c_cache", 0), E),
                       (lambda a: setattr(a, "workspace_bytes", 1024), E), (lambda a: setattr(a, "rope_max_pos", 10), E),
                       (lambda a: setattr(a, "n_noise", 4), U), (lambda a: setattr(a, "d_rope", 48), U),
+                      (lambda a: setattr(a, "g", 4), U),  # 16 x 5 = 80 query heads: prefill only
                       (lambda a: (setattr(a, "mask", 1), setattr(a, "window", -3)), E)):
         a = good()
         mut(a)

@@ -41,6 +41,9 @@ SMALL = [
     wl.PrefillShape("bf16 L=1", B=3, L=1, n_kv=2, g=2),
     wl.PrefillShape("bf16 d=64", B=1, L=257, d_c=256, d_R=32, n_kv=2, d_n=64, d_v=64, g=4),
     wl.PrefillShape("fp32 d=128 causal", B=1, L=150, n_kv=1, g=3, dtype="fp32"),
+    # the report's attention shape: 16 KV heads, g = 4 (80 query heads), full and 128-token window
+    wl.PrefillShape("bf16 80 heads g=4 causal", B=1, L=200, n_kv=16, g=4),
+    wl.PrefillShape("bf16 80 heads g=4 sliding W=128", B=1, L=400, n_kv=16, g=4, mask="sliding", window=128),
 ]
 
 
