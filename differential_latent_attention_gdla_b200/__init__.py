@@ -73,6 +73,33 @@ def rope_tables(max_pos: int, d_rope: int, base: float = 10000.0, device="cuda")
     return ang.cos().float().to(device), ang.sin().float().to(device)
 
 
+def yarn_rope_tables(max_pos: int, d_rope: int, factor: float, original_max_pos: int, base: float = 10000.0,
+                     beta_fast: float = 32.0, beta_slow: float = 1.0, device="cuda"):
+    """cos/sin tables [max_pos, d_rope/2] (fp32) of RoPE with YaRN frequency scaling
+    ("Context Extension via YaRN", page 1, section 2), for extending a model trained
+    on ``original_max_pos`` tokens by ``factor``: a frequency whose wavelength
+    2 pi / theta is below original_max_pos / beta_fast is kept, one above
+    original_max_pos / beta_slow is divided by ``factor``, and in between the
+    divisor moves linearly with the wavelength. Model set-up, like ``rope_tables``;
+    pair the tables with ``softmax_scale = yarn_mscale(factor)**2 / sqrt(d_qk)``."""
+    theta = base ** (-2.0 * torch.arange(d_rope // 2, dtype=torch.float64) / d_rope)
+    wavelength = 2.0 * math.pi / theta
+    short, long_ = original_max_pos / beta_fast, original_max_pos / beta_slow
+    if long_ > short:
+        ramp = ((wavelength - short) / (long_ - short)).clamp(0.0, 1.0)
+    else:
+        ramp = (wavelength > short).to(torch.float64)
+    theta = theta * ((1.0 - ramp) + ramp / factor)
+    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * theta[None, :]
+    return ang.cos().float().to(device), ang.sin().float().to(device)
+
+
+def yarn_mscale(factor: float) -> float:
+    """YaRN's attention temperature m = 1 + 0.1 ln(factor) (1 for factor <= 1); the
+    logits are multiplied by m^2, which the caller folds into softmax_scale."""
+    return 1.0 + 0.1 * math.log(factor) if factor > 1.0 else 1.0
+
+
 # ------------------------------------------------------------------- expansion
 def latent_expand(c_kv, gamma, k_rope, w_ukv, rope_cos, rope_sin, *, n_kv: int, d_nope: int, d_v: int,
                   rms_eps: float = 0.0, kv_out=None, k_rope_out=None, c_hat_out=None, stream=None):

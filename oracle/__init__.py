@@ -14,6 +14,7 @@ forms, invariants, brute force and independent numpy formulations.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 import threading
@@ -57,6 +58,7 @@ def _load():
                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp]
             lib.gdla_oracle_rope.argtypes = [_dp, ctypes.c_long, ctypes.c_int, ctypes.c_double, _dp]
             lib.gdla_oracle_rope_table.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_double, _dp, _dp]
+            lib.gdla_oracle_yarn_inv_freq.argtypes = [ctypes.c_int] + [ctypes.c_double] * 5 + [_dp]
             lib.gdla_oracle_attend_row.argtypes = [_dp, _dp, _dp, ctypes.c_long, _dp, ctypes.c_long, _dp,
                                                    ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_long, ctypes.c_int, ctypes.c_long, ctypes.c_double,
@@ -66,11 +68,11 @@ def _load():
             lib.gdla_oracle_prefill_rows.restype = ctypes.c_int
             lib.gdla_oracle_prefill_rows.argtypes = (
                 [ctypes.c_int, ctypes.c_long] + [ctypes.c_int] * 6 + [ctypes.c_int, ctypes.c_long]
-                + [ctypes.c_double] * 3 + [_dp] * 4 + [ctypes.c_long, _lp, _lp] + [_dp] * 3 + [_ip] + [_dp] * 2)
+                + [ctypes.c_double] * 3 + [_dp] * 5 + [ctypes.c_long, _lp, _lp] + [_dp] * 3 + [_ip] + [_dp] * 2)
             lib.gdla_oracle_decode_seq.restype = ctypes.c_int
             lib.gdla_oracle_decode_seq.argtypes = (
                 [ctypes.c_long] + [ctypes.c_int] * 6 + [ctypes.c_int, ctypes.c_long, ctypes.c_double,
-                                                       ctypes.c_double] + [_dp] * 6 + [_ip, _dp, _dp])
+                                                       ctypes.c_double] + [_dp] * 7 + [_ip, _dp, _dp])
             _lib = lib
     return _lib
 
@@ -131,6 +133,36 @@ def rope_table(max_pos: int, d_R: int, base: float = DEFAULT_ROPE_BASE):
     return c, s
 
 
+def rope_freqs(d_R: int, base: float = DEFAULT_ROPE_BASE) -> np.ndarray:
+    """The plain RoPE frequencies theta_k = base^(-2k/d_R), k < d_R/2 (fp64)."""
+    return base ** (-2.0 * np.arange(d_R // 2) / d_R)
+
+
+def yarn_inv_freq(d_R: int, factor: float, original_max_pos: float, base: float = DEFAULT_ROPE_BASE,
+                  beta_fast: float = 32.0, beta_slow: float = 1.0) -> np.ndarray:
+    """RoPE frequencies rescaled by YaRN ("Context Extension via YaRN", page 1,
+    section 2): kept where the wavelength is below original_max_pos/beta_fast,
+    divided by ``factor`` above original_max_pos/beta_slow, blended linearly in the
+    wavelength in between (computed by the C oracle)."""
+    out = np.empty(d_R // 2)
+    _load().gdla_oracle_yarn_inv_freq(d_R, base, factor, original_max_pos, beta_fast, beta_slow, _p(out))
+    return out
+
+
+def yarn_mscale(factor: float) -> float:
+    """YaRN's attention temperature: the factor 1 + 0.1 ln(s) by which the pages'
+    listing scales both rotated vectors, i.e. a factor m^2 on the logits (1 for
+    s <= 1). The pages' prose gives sqrt(1 + 0.1 ln s) instead; the listing's
+    value is the one used here (a reading)."""
+    return 1.0 + 0.1 * math.log(factor) if factor > 1.0 else 1.0
+
+
+def rope_table_freq(max_pos: int, inv_freq) -> tuple[np.ndarray, np.ndarray]:
+    """cos/sin tables [max_pos, d_R/2] for explicit frequencies (fp64)."""
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * _d(inv_freq)[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
 def attend_row(q_n, q_r_rot, k_n, k_r_rot, v, i: int, mask: int = MASK_CAUSAL, window: int = 0,
                scale: float | None = None, want_p: bool = False):
     """Steps 4-6 for one query row ``i`` of one head over keys/values [T, *].
@@ -163,10 +195,11 @@ def differential_gate(h_s, h_n, lam_logits, gate_logits, g: int) -> np.ndarray:
 def prefill_rows(*, c_kv, gamma, k_rope, w_ukv, q_rows, lam_rows, gate_rows, row_b, row_i, g: int,
                  d_n: int, d_v: int, mask: int = MASK_CAUSAL, window: int = 0, scale: float | None = None,
                  eps: float = DEFAULT_EPS, rope_base: float = DEFAULT_ROPE_BASE, want_heads: bool = False,
-                 kv_sel=None):
+                 kv_sel=None, inv_freq=None):
     """Output rows Y [nrows, n_S, d_v] of the prefill for query tokens (row_b, row_i).
     With ``kv_sel`` (a list of KV group indices) only those groups are computed
-    and the other groups' rows are NaN.
+    and the other groups' rows are NaN. ``inv_freq`` [d_R/2] replaces the RoPE
+    frequencies rope_base^(-2k/d_R) (e.g. with ``yarn_inv_freq``).
 
     c_kv [B, L, d_c], k_rope [B, L, d_R], w_ukv [d_c, n_kv*(d_n+d_v)], gamma [d_c]
     cover the whole batch; q_rows [nrows, n_S+n_N, d_n+d_R], lam_rows
@@ -192,8 +225,10 @@ def prefill_rows(*, c_kv, gamma, k_rope, w_ukv, q_rows, lam_rows, gate_rows, row
     if kv_sel is not None:
         sel = np.zeros(n_kv, dtype=np.int32)
         sel[np.asarray(kv_sel, dtype=np.int64)] = 1
+    inv = None if inv_freq is None else _d(inv_freq)
+    assert inv is None or inv.shape == (d_R // 2,)
     rc = _load().gdla_oracle_prefill_rows(
-        B, L, d_c, d_R, n_kv, d_n, d_v, g, mask, window, scale, eps, rope_base,
+        B, L, d_c, d_R, n_kv, d_n, d_v, g, mask, window, scale, eps, rope_base, _p(inv) if inv is not None else None,
         _p(c_kv), _p(gamma), _p(k_rope), _p(w_ukv), nrows, rb.ctypes.data_as(_lp), ri.ctypes.data_as(_lp),
         _p(q_rows), _p(lam_rows), _p(gate_rows), sel.ctypes.data_as(_ip) if sel is not None else None, _p(y),
         _p(heads) if want_heads else None)
@@ -208,12 +243,13 @@ def prefill_rows(*, c_kv, gamma, k_rope, w_ukv, q_rows, lam_rows, gate_rows, row
 
 def decode_seq(*, c_hat, k_r_rot, q, w_ukv, lam, gate, g: int, d_n: int, d_v: int, mask: int = MASK_CAUSAL,
                window: int = 0, scale: float | None = None, rope_base: float = DEFAULT_ROPE_BASE,
-               kv_sel=None, want_heads: bool = False):
+               kv_sel=None, want_heads: bool = False, inv_freq=None):
     """Decode of one token at position T-1 over one sequence's latent cache.
 
     c_hat [T, d_c] (normalised latent), k_r_rot [T, d_R] (rotated key),
     q [n_S+n_N, d_n+d_R] (rotary part pre-RoPE), lam [n_S], gate [n_S, d_v].
     Returns Y [n_S, d_v]; rows of KV groups excluded by ``kv_sel`` are NaN.
+    ``inv_freq`` [d_R/2] replaces the RoPE frequencies of the query rotation.
     """
     c_hat, k_r_rot, q, w_ukv, lam, gate = map(_d, (c_hat, k_r_rot, q, w_ukv, lam, gate))
     T, d_c = c_hat.shape
@@ -228,8 +264,11 @@ def decode_seq(*, c_hat, k_r_rot, q, w_ukv, lam, gate, g: int, d_n: int, d_v: in
     if kv_sel is not None:
         sel = np.zeros(n_kv, dtype=np.int32)
         sel[np.asarray(kv_sel, dtype=np.int64)] = 1
+    inv = None if inv_freq is None else _d(inv_freq)
+    assert inv is None or inv.shape == (d_R // 2,)
     rc = _load().gdla_oracle_decode_seq(
-        T, d_c, d_R, n_kv, d_n, d_v, g, mask, window, scale, rope_base, _p(c_hat), _p(k_r_rot), _p(q),
+        T, d_c, d_R, n_kv, d_n, d_v, g, mask, window, scale, rope_base, _p(inv) if inv is not None else None,
+        _p(c_hat), _p(k_r_rot), _p(q),
         _p(w_ukv), _p(lam), _p(gate), sel.ctypes.data_as(_ip) if sel is not None else None, _p(y),
         _p(heads) if want_heads else None)
     if rc != 0:

@@ -110,15 +110,46 @@ void gdla_oracle_expand_head(const double* c_hat, const double* w_ukv, long T, i
  * theta_k = base^(-2k/d_R), k = 0 .. d_R/2-1; the pair (x[k], x[k+d_R/2]) is
  * rotated by the angle pos*theta_k.
  */
-void gdla_oracle_rope(const double* x, long pos, int d_R, double base, double* y) {
+static void rope_apply(const double* x, long pos, int d_R, double base, const double* inv_freq, double* y) {
   const int half = d_R / 2;
   for (int k = 0; k < half; ++k) {
-    double theta = pow(base, -2.0 * k / (double)d_R);
+    /* the frequencies come from the base, or are given (a rescaled RoPE such as YaRN) */
+    double theta = inv_freq ? inv_freq[k] : pow(base, -2.0 * k / (double)d_R);
     double a = (double)pos * theta;
     double c = cos(a), s = sin(a);
     double x1 = x[k], x2 = x[k + half];
     y[k] = x1 * c - x2 * s;
     y[k + half] = x2 * c + x1 * s;
+  }
+}
+
+void gdla_oracle_rope(const double* x, long pos, int d_R, double base, double* y) {
+  rope_apply(x, pos, d_R, base, 0, y);
+}
+
+/* ---- YaRN frequency scaling ("Context Extension via YaRN", page 1, section 2) ----
+ * Extending the context by a factor s = L_new / L_native: with the wavelength of
+ * frequency k, lambda_k = 2 pi / theta_k, frequencies whose wavelength is below
+ * orig/beta_fast are kept (scale 1), those above orig/beta_slow are interpolated
+ * (scale 1/s), and in between the scale moves linearly with the wavelength:
+ *   alpha_k = clamp((lambda_k - orig/beta_fast) / (orig/beta_slow - orig/beta_fast), 0, 1)
+ *   theta'_k = theta_k * ((1 - alpha_k) + alpha_k / s).
+ * The logit temperature is a separate factor (see the Python wrapper). */
+void gdla_oracle_yarn_inv_freq(int d_R, double base, double factor, double orig_max_pos, double beta_fast,
+                               double beta_slow, double* inv_freq) {
+  const int half = d_R / 2;
+  const double lam_fast = orig_max_pos / beta_fast, lam_slow = orig_max_pos / beta_slow;
+  for (int k = 0; k < half; ++k) {
+    const double theta = pow(base, -2.0 * k / (double)d_R);
+    const double lam = 2.0 * acos(-1.0) / theta;  /* 2 pi / theta */
+    double alpha;
+    if (lam_slow > lam_fast) {
+      alpha = (lam - lam_fast) / (lam_slow - lam_fast);
+      alpha = alpha < 0.0 ? 0.0 : (alpha > 1.0 ? 1.0 : alpha);
+    } else {
+      alpha = lam > lam_fast ? 1.0 : 0.0;
+    }
+    inv_freq[k] = theta * ((1.0 - alpha) + alpha / factor);
   }
 }
 
@@ -216,7 +247,7 @@ void gdla_oracle_differential_gate(const double* h_s, const double* h_nz, const 
  */
 int gdla_oracle_prefill_rows(int B, long L, int d_c, int d_R, int n_kv, int d_n, int d_v,
                              int g, int mask, long window, double scale, double eps,
-                             double rope_base, const double* c_kv, const double* gamma,
+                             double rope_base, const double* inv_freq, const double* c_kv, const double* gamma,
                              const double* k_rope, const double* w_ukv, long nrows,
                              const long* row_b, const long* row_i, const double* q_rows,
                              const double* lam_rows, const double* gate_rows, const int* kv_sel,
@@ -252,7 +283,7 @@ int gdla_oracle_prefill_rows(int B, long L, int d_c, int d_R, int n_kv, int d_n,
     /* step 1 (the whole latent) and step 3 for the shared rotary key */
     gdla_oracle_latent_norm(c_kv + (long)b * L * d_c, gamma, T, d_c, eps, c_hat);
     for (long j = 0; j < T; ++j)
-      gdla_oracle_rope(k_rope + ((long)b * L + j) * d_R, j, d_R, rope_base, k_r_rot + j * d_R);
+      rope_apply(k_rope + ((long)b * L + j) * d_R, j, d_R, rope_base, inv_freq, k_r_rot + j * d_R);
 
     for (int h = 0; h < n_kv; ++h) {
       if (kv_sel && !kv_sel[h]) continue;
@@ -274,7 +305,7 @@ int gdla_oracle_prefill_rows(int B, long L, int d_c, int d_R, int n_kv, int d_n,
         long i = row_i[r];
         const double* qh = q_rows + ((long)r * H_q + head) * d_qk;
         double q_r[512];
-        gdla_oracle_rope(qh + d_n, i, d_R, rope_base, q_r);
+        rope_apply(qh + d_n, i, d_R, rope_base, inv_freq, q_r);
         gdla_oracle_attend_row(qh, q_r, k_n, d_n, k_r_rot, d_R, v, d_v, d_n, d_R, d_v, i, mask,
                                window, scale, heads + ((long)r * H_q + head) * d_v, NULL);
       }
@@ -306,7 +337,7 @@ int gdla_oracle_prefill_rows(int B, long L, int d_c, int d_R, int n_kv, int d_n,
  * the other groups are left untouched.
  */
 int gdla_oracle_decode_seq(long T, int d_c, int d_R, int n_kv, int d_n, int d_v, int g,
-                           int mask, long window, double scale, double rope_base,
+                           int mask, long window, double scale, double rope_base, const double* inv_freq,
                            const double* c_hat, const double* k_r_rot, const double* q,
                            const double* w_ukv, const double* lam, const double* gate,
                            const int* kv_sel, double* y, double* heads_out) {
@@ -326,7 +357,7 @@ int gdla_oracle_decode_seq(long T, int d_c, int d_R, int n_kv, int d_n, int d_v,
       int head = (which < g) ? h * g + which : n_S + h;
       const double* qh = q + (long)head * d_qk;
       double q_r[512];
-      gdla_oracle_rope(qh + d_n, i, d_R, rope_base, q_r);
+      rope_apply(qh + d_n, i, d_R, rope_base, inv_freq, q_r);
       gdla_oracle_attend_row(qh, q_r, k_n, d_n, k_r_rot, d_R, v, d_v, d_n, d_R, d_v, i, mask,
                              window, scale, heads + (long)head * d_v, NULL);
     }

@@ -19,11 +19,12 @@ RNG = np.random.default_rng(1234)
 
 
 # ------------------------------------------------------------------ independent forms
-def np_rope_complex(x, pos, base=10000.0):
+def np_rope_complex(x, pos, base=10000.0, theta=None):
     """RoPE as multiplication of (x_k + i x_{k+d/2}) by exp(i pos theta_k)."""
     d = x.shape[-1]
     h = d // 2
-    theta = base ** (-2.0 * np.arange(h) / d)
+    if theta is None:
+        theta = base ** (-2.0 * np.arange(h) / d)
     z = (x[..., :h] + 1j * x[..., h:]) * np.exp(1j * pos * theta)
     return np.concatenate([z.real, z.imag], axis=-1)
 
@@ -44,7 +45,8 @@ def np_attention_matrix(Q, K, V, scale, mask, window):
     return P @ V, P
 
 
-def np_gdla_prefill(c, gamma, k_rope, q, w, lam, gate, g, d_n, d_v, mask, window, eps=1e-6, base=10000.0):
+def np_gdla_prefill(c, gamma, k_rope, q, w, lam, gate, g, d_n, d_v, mask, window, eps=1e-6, base=10000.0,
+                    theta=None, scale=None):
     """The whole layer in numpy matrix form (one sequence): normalise, expand,
     rotate (complex form), attend per head, differential, gate."""
     L, d_c = c.shape
@@ -54,13 +56,14 @@ def np_gdla_prefill(c, gamma, k_rope, q, w, lam, gate, g, d_n, d_v, mask, window
     chat = gamma * c / np.sqrt((c * c).mean(axis=1, keepdims=True) + eps)
     KV = (chat @ w).reshape(L, n_kv, d_n + d_v)
     pos = np.arange(L)[:, None]
-    kr = np_rope_complex(k_rope, pos, base)
+    kr = np_rope_complex(k_rope, pos, base, theta)
     H = np.zeros((L, n_S + n_kv, d_v))
-    scale = 1.0 / math.sqrt(d_n + d_R)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_n + d_R)
     for head in range(n_S + n_kv):
         kvh = head // g if head < n_S else head - n_S
         qn = q[:, head, :d_n]
-        qr = np_rope_complex(q[:, head, d_n:], pos, base)
+        qr = np_rope_complex(q[:, head, d_n:], pos, base, theta)
         Qf = np.concatenate([qn, qr], axis=1)
         Kf = np.concatenate([KV[:, kvh, :d_n], kr], axis=1)
         H[:, head], _ = np_attention_matrix(Qf, Kf, KV[:, kvh, d_n:], scale, mask, window)
@@ -434,3 +437,64 @@ def test_prefill_group_selection_matches_full():
                                row_b=rb, row_i=ri, g=2, d_n=inp["d_n"], d_v=inp["d_v"], kv_sel=[1]).reshape(full.shape)
     np.testing.assert_array_equal(part[:, :, 2:4], full[:, :, 2:4])
     assert np.isnan(part[:, :, :2]).all() and np.isnan(part[:, :, 4:]).all()
+
+
+# ------------------------------------------------------------------ YaRN (context extension)
+# "Open-Source Frontier Models: Architecture and Benchmarks of Rnj-1 and Motif-2",
+# section 2 (Context Extension via YaRN): per-frequency scale 1 (short wavelengths),
+# 1/s (long wavelengths), linear ramp in between; logit temperature from ln s.
+def test_yarn_factor_one_is_plain_rope():
+    for d_R in (16, 64):
+        np.testing.assert_allclose(oracle.yarn_inv_freq(d_R, 1.0, 4096.0), oracle.rope_freqs(d_R), rtol=1e-15, atol=0)
+
+
+@pytest.mark.parametrize("factor,orig", [(32.0, 4096.0), (64.0, 4096.0), (16.0, 64.0)])
+def test_yarn_frequency_regimes(factor, orig):
+    d_R = 64
+    base = oracle.rope_freqs(d_R)
+    ratio = oracle.yarn_inv_freq(d_R, factor, orig) / base
+    wavelength = 2 * math.pi / base
+    short, long_ = orig / 32.0, orig / 1.0
+    hi, lo = wavelength < short, wavelength > long_
+    assert lo.any() and (hi.any() or wavelength.min() >= short)        # (short wavelength 2: no kept band)
+    np.testing.assert_allclose(ratio[hi], 1.0, rtol=1e-15)            # high frequencies kept
+    np.testing.assert_allclose(ratio[lo], 1.0 / factor, rtol=1e-15)   # low frequencies divided by s
+    mid = ~hi & ~lo
+    assert ((ratio[mid] < 1.0) & (ratio[mid] > 1.0 / factor)).all()
+    assert (np.diff(ratio) <= 1e-15).all()                            # monotone in the wavelength
+    # the ramp is linear in the wavelength: alpha = (lambda - short) / (long - short)
+    alpha = (wavelength[mid] - short) / (long_ - short)
+    np.testing.assert_allclose(ratio[mid], (1 - alpha) + alpha / factor, rtol=1e-14)
+
+
+def test_yarn_interpolated_frequencies_map_positions_back():
+    # for a fully interpolated frequency the angle at position s*p equals the native angle at p
+    d_R, factor = 64, 32.0
+    f = oracle.yarn_inv_freq(d_R, factor, 4096.0)
+    base = oracle.rope_freqs(d_R)
+    lo = f < base
+    k = np.flatnonzero(np.isclose(f, base / factor, rtol=1e-15))
+    assert len(k) > 0 and lo.any()
+    for p in (1, 7, 4095):
+        np.testing.assert_allclose(factor * p * f[k], p * base[k], rtol=1e-14)
+
+
+def test_yarn_mscale_closed_form():
+    assert oracle.yarn_mscale(1.0) == 1.0 and oracle.yarn_mscale(0.5) == 1.0
+    assert abs(oracle.yarn_mscale(math.exp(10.0)) - 2.0) < 1e-15
+    assert abs(oracle.yarn_mscale(64.0) - (1 + 0.1 * math.log(64.0))) < 1e-15
+
+
+def test_prefill_explicit_frequencies_match_base_and_matrix_form():
+    inp = tiny_inputs(d_R=8)
+    plain = run_all_rows(inp)
+    np.testing.assert_array_equal(run_all_rows(inp, inv_freq=oracle.rope_freqs(8)), plain)
+    theta = oracle.yarn_inv_freq(8, 4.0, 8.0, beta_fast=4.0, beta_slow=1.0)
+    scale = oracle.yarn_mscale(4.0) ** 2 / math.sqrt(inp["d_n"] + 8)
+    y = run_all_rows(inp, inv_freq=theta, scale=scale)
+    assert not np.allclose(y, plain)
+    for b in range(inp["c_kv"].shape[0]):
+        ey, _ = np_gdla_prefill(inp["c_kv"][b], inp["gamma"], inp["k_rope"][b], inp["q"][b], inp["w_ukv"],
+                                inp["lam"][b], inp["gate"][b], inp["g"], inp["d_n"], inp["d_v"], oracle.MASK_CAUSAL, 0,
+                                theta=theta, scale=scale)
+        np.testing.assert_allclose(y[b], ey, rtol=1e-11, atol=1e-12)

@@ -189,3 +189,56 @@ def test_decode_peaked_softmax_rescale_path(scale):
     # exponents by ~|s| 2^-9, so only the RMS bar applies (a wrong rescale
     # would be an O(1) error)
     assert_parity(f64(y), ref, torch.bfloat16, f"decode peaked x{scale}", elementwise=False)
+
+
+# ------------------------------------------------------------------ YaRN context extension
+# Rescaled RoPE tables and the YaRN logit temperature are inputs of the same kernels
+# ("Open-Source Frontier Models: Architecture and Benchmarks of Rnj-1 and Motif-2",
+# section 2); positions far beyond the native length exercise the interpolated band.
+YARN = dict(factor=16.0, orig=64)
+
+
+def yarn_scale(d_qk):
+    return gdla.yarn_mscale(YARN["factor"]) ** 2 / float(np.sqrt(d_qk))
+
+
+def test_prefill_yarn_every_element():
+    shape = wl.PrefillShape("bf16 YaRN x16 from 64 tokens, g=3", B=1, L=300, n_kv=2, g=3)
+    inp = wl.make_prefill_inputs(shape, seed=31, device=DEV, act="unit")
+    cos, sin = gdla.yarn_rope_tables(shape.L, shape.d_R, YARN["factor"], YARN["orig"], device=DEV)
+    scale = yarn_scale(shape.d_n + shape.d_R)
+    y = gdla.prefill(inp["c_kv"], inp["gamma"], inp["k_rope"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                     inp["gate_logits"], g=shape.g, softmax_scale=scale)
+    torch.cuda.synchronize()
+    rows = all_rows(shape)
+    rb = torch.tensor([r[0] for r in rows], device=DEV)
+    ri = torch.tensor([r[1] for r in rows], device=DEV)
+    ref = oracle.prefill_rows(
+        c_kv=f64(inp["c_kv"]), gamma=f64(inp["gamma"]), k_rope=f64(inp["k_rope"]), w_ukv=f64(inp["w_ukv"]),
+        q_rows=f64(inp["q"][rb, ri]), lam_rows=f64(inp["lam_logits"][rb, ri]), gate_rows=f64(inp["gate_logits"][rb, ri]),
+        row_b=rb.cpu().numpy(), row_i=ri.cpu().numpy(), g=shape.g, d_n=shape.d_n, d_v=shape.d_v, scale=scale,
+        inv_freq=oracle.yarn_inv_freq(shape.d_R, YARN["factor"], YARN["orig"]))
+    assert_parity(f64(y).reshape(ref.shape), ref, torch.bfloat16, shape.name)
+    # the rescaled tables change the result (the check above is not vacuous)
+    plain = oracle.prefill_rows(
+        c_kv=f64(inp["c_kv"]), gamma=f64(inp["gamma"]), k_rope=f64(inp["k_rope"]), w_ukv=f64(inp["w_ukv"]),
+        q_rows=f64(inp["q"][rb, ri]), lam_rows=f64(inp["lam_logits"][rb, ri]), gate_rows=f64(inp["gate_logits"][rb, ri]),
+        row_b=rb.cpu().numpy(), row_i=ri.cpu().numpy(), g=shape.g, d_n=shape.d_n, d_v=shape.d_v)
+    assert np.sqrt(np.mean((plain - ref) ** 2)) > 0.1 * np.sqrt(np.mean(ref ** 2))
+
+
+def test_decode_yarn_every_element():
+    shape = wl.DecodeShape("bf16 YaRN decode B=3 T=300", B=3, T=300, n_kv=2, g=2)
+    inp = wl.make_decode_inputs(shape, seed=33, device=DEV, act="unit", seqlens=[300, 190, 64])
+    cos, sin = gdla.yarn_rope_tables(shape.T, shape.d_R, YARN["factor"], YARN["orig"], device=DEV)
+    scale = yarn_scale(shape.d_n + shape.d_R)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g, softmax_scale=scale)
+    torch.cuda.synchronize()
+    theta = oracle.yarn_inv_freq(shape.d_R, YARN["factor"], YARN["orig"])
+    ref = np.stack([oracle.decode_seq(
+        c_hat=f64(inp["c_cache"][b, :T]), k_r_rot=f64(inp["kr_cache"][b, :T]), q=f64(inp["q"][b]),
+        w_ukv=f64(inp["w_ukv"]), lam=f64(inp["lam_logits"][b]), gate=f64(inp["gate_logits"][b]), g=shape.g,
+        d_n=shape.d_n, d_v=shape.d_v, scale=scale, inv_freq=theta)
+        for b, T in enumerate(int(t) for t in inp["seqlens"])])
+    assert_parity(f64(y), ref, torch.bfloat16, shape.name)
