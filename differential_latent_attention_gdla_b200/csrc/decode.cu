@@ -24,6 +24,7 @@ constexpr int ABS_R = 48;    // query rows per block: 8 warps x 6
 constexpr int CMB_R = 16;
 constexpr int CMB_RPW = CMB_R / 8;  // query rows per warp
 constexpr int CMB_KC = 64;   // latent rows of W_UV staged per step
+constexpr int kMergeBatch = 12;  // split partials loaded together by one thread
 
 __host__ __device__ inline int absorb_seqs(int g) { return max(1, ABS_R / (g + 1)); }
 __host__ __device__ inline int combine_seqs(int g) { return max(1, CMB_R / (g + 1)); }
@@ -257,12 +258,38 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   float* olat = sm;                              // [CMB_R][d_c]
   float* hsm = olat + CMB_R * d_c;               // [CMB_R][DV]
   float* wgt = hsm + CMB_R * DV;                 // [CMB_R][NS] merge weights (scaled by 1 / denominator)
-  T* wch = reinterpret_cast<T*>(wgt + CMB_R * NS);  // [CMB_KC][DV] staged W_UV rows
+  T* wch = reinterpret_cast<T*>(wgt + CMB_R * NS);  // 2 x [CMB_KC][DV] staged W_UV rows
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   const T* gate = reinterpret_cast<const T*>(p.gate);
   T* out = reinterpret_cast<T*>(p.out);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   auto head_of_row = [&](int r) { const int u = r % G1; return u < p.g ? h * p.g + u : n_S + h; };
+  // W_UV rows [k0, k0 + CMB_KC) of this KV group: register-staged, so that the loads of
+  // the next rows overlap the products on the current ones
+  constexpr int VEC = 16 / (int)sizeof(T);
+  const int per_row = DV / VEC;
+  const int n_w = CMB_KC * per_row;  // 16-byte pieces per staged block
+  constexpr int kWPT = 8;            // pieces per thread (n_w <= 256 * kWPT for every supported width)
+  uint4 wreg[kWPT];
+  auto load_w = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < kWPT; ++q) {
+      const int e = tid + q * 256;
+      if (e < n_w) {
+        const int c = e / per_row, v = e % per_row;
+        wreg[q] = *reinterpret_cast<const uint4*>(w + (long)(k0 + c) * ncol + (long)h * (p.d_nope + DV) + p.d_nope +
+                                                  v * VEC);
+      }
+    }
+  };
+  auto store_w = [&](T* dst) {
+#pragma unroll
+    for (int q = 0; q < kWPT; ++q) {
+      const int e = tid + q * 256;
+      if (e < n_w) *reinterpret_cast<uint4*>(dst + (e / per_row) * DV + (e % per_row) * VEC) = wreg[q];
+    }
+  };
+  load_w(0);
 
   // ---- merge weights: one warp per query row
   for (int r = warp; r < R; r += 8) {
@@ -295,28 +322,20 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     const long stride4 = (long)H_q * d_c / 4;
     const float* wr = wgt + r * NS;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int sp = 0;
-    // four splits' partials in flight at a time (the loads are independent)
-    for (; sp + 4 <= NS; sp += 4) {
-      float4 x[4];
+    // up to kMergeBatch splits' partials in flight at a time (the loads are independent)
+    for (int sp0 = 0; sp0 < NS; sp0 += kMergeBatch) {
+      float4 x[kMergeBatch];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) x[q] = src[(sp + q) * stride4];
+      for (int q = 0; q < kMergeBatch; ++q)
+        x[q] = sp0 + q < NS ? src[(sp0 + q) * stride4] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float wv = wr[sp + q];
+      for (int q = 0; q < kMergeBatch; ++q) {
+        const float wv = sp0 + q < NS ? wr[sp0 + q] : 0.f;
         acc.x = fmaf(wv, x[q].x, acc.x);
         acc.y = fmaf(wv, x[q].y, acc.y);
         acc.z = fmaf(wv, x[q].z, acc.z);
         acc.w = fmaf(wv, x[q].w, acc.w);
       }
-    }
-    for (; sp < NS; ++sp) {
-      const float wv = wr[sp];
-      const float4 x = src[sp * stride4];
-      acc.x = fmaf(wv, x.x, acc.x);
-      acc.y = fmaf(wv, x.y, acc.y);
-      acc.z = fmaf(wv, x.z, acc.z);
-      acc.w = fmaf(wv, x.w, acc.w);
     }
     reinterpret_cast<float4*>(olat + r * d_c)[v] = acc;
   }
@@ -326,23 +345,18 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   for (int i = 0; i < CMB_RPW; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  constexpr int VEC = 16 / (int)sizeof(T);
-  const int per_row = DV / VEC;
   const bool col_ok = 4 * lane < DV;
-  for (int k0 = 0; k0 < d_c; k0 += CMB_KC) {
-    __syncthreads();  // O_lat written (first step) / previous W_UV rows consumed
-    for (int e = tid; e < CMB_KC * per_row; e += blockDim.x) {
-      const int c = e / per_row, v = e % per_row;
-      *reinterpret_cast<uint4*>(wch + c * DV + v * VEC) = *reinterpret_cast<const uint4*>(
-          w + (long)(k0 + c) * ncol + (long)h * (p.d_nope + DV) + p.d_nope + v * VEC);
-    }
-    __syncthreads();
+  store_w(wch);
+  __syncthreads();  // O_lat and the first W_UV rows are in shared memory
+  for (int k0 = 0, it = 0; k0 < d_c; k0 += CMB_KC, ++it) {
+    const T* wcur = wch + (it & 1) * (CMB_KC * DV);
+    if (k0 + CMB_KC < d_c) load_w(k0 + CMB_KC);
     if (col_ok) {
 #pragma unroll 4
       for (int c = 0; c < CMB_KC; ++c) {
         float wv[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) wv[j] = to_f(wch[c * DV + 4 * lane + j]);
+        for (int j = 0; j < 4; ++j) wv[j] = to_f(wcur[c * DV + 4 * lane + j]);
 #pragma unroll
         for (int i = 0; i < CMB_RPW; ++i) {
           const float ov = olat[(CMB_RPW * warp + i) * d_c + k0 + c];
@@ -351,6 +365,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
         }
       }
     }
+    if (k0 + CMB_KC < d_c) store_w(wch + ((it + 1) & 1) * (CMB_KC * DV));
+    __syncthreads();  // next rows staged; the buffer just read may be refilled
   }
   if (col_ok) {
 #pragma unroll
@@ -430,7 +446,7 @@ cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStre
   const size_t esz = dt == GDLA_BF16 ? 2 : 4;
   const int spb = combine_seqs(p.g);
   const size_t smem = sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * p.d_v + (size_t)CMB_R * p.n_splits) +
-                      esz * (size_t)CMB_KC * p.d_v;
+                      esz * 2 * (size_t)CMB_KC * p.d_v;
   dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + spb - 1) / spb));
   cudaError_t e;
   if (dt == GDLA_BF16) {
