@@ -253,7 +253,7 @@ def run_ours(a):
         gdla.decode(din["c_cache"], din["kr_cache"], din["q"], din["w_ukv"], cos, sin, din["lam_logits"],
                     din["gate_logits"], din["seqlens"], g=D.g, out=yd, workspace=dws, stream=stream)
 
-    launches_per_step = 2 + 1 + 4  # norm+rope, expansion GEMM | attention | absorb, split-KV, merge, combine
+    launches_per_step = 2 + 1 + 3  # norm+rope, expansion GEMM | attention | absorb, split-KV, combine
     for _ in range(a.warmup):
         expand()
         attend()
