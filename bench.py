@@ -63,7 +63,7 @@ def measured_traffic(kernel: str, workload: str):
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
@@ -174,7 +174,7 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", str(index)], stdout=self.f, stderr=subprocess.DEVNULL)
+                                          "-lms", "50", "-i", str(index)], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
