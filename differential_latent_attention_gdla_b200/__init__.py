@@ -20,8 +20,9 @@ import torch
 from . import _abi
 from ._abi import GDLA_BF16, GDLA_FP32, GDLA_MASK_CAUSAL, GDLA_MASK_SLIDING, GdlaError  # noqa: F401
 
-__all__ = ["prefill", "attend", "decode", "decode_noalloc", "latent_expand", "rope_tables", "prefill_workspace_size", "decode_workspace_size",
-           "workspace_status", "build_info", "GdlaError"]
+__all__ = ["prefill", "attend", "decode", "decode_noalloc", "latent_expand", "rope_tables", "yarn_rope_tables",
+           "yarn_mscale", "prefill_workspace_size", "decode_workspace_size", "workspace_status", "diag_wait_timeout",
+           "build_info", "GdlaError"]
 
 _DT = {torch.bfloat16: GDLA_BF16, torch.float32: GDLA_FP32}
 
@@ -260,6 +261,13 @@ def decode_noalloc(c_cache, kr_cache, q, w_ukv, rope_cos, rope_sin, lam_logits, 
                      mask, window, softmax_scale, None)
     _abi.check(_lib().gdla_decode_noalloc(ctypes.byref(a), _stream(stream)), "gdla_decode_noalloc")
     return out
+
+
+def diag_wait_timeout(status_word, stream=None) -> None:
+    """Diagnostic: run one device wait that can never complete; it ends at its
+    limit and records GDLA_ERR_TIMEOUT in ``status_word`` (a 256-byte uint8 CUDA
+    tensor), readable with ``workspace_status``."""
+    _abi.check(_lib().gdla_diag_wait_timeout(_ptr(status_word), _stream(stream)), "gdla_diag_wait_timeout")
 
 
 def workspace_status(workspace, stream=None) -> int:

@@ -57,7 +57,8 @@ class DecodeArgs(ctypes.Structure):
 
 # Every symbol include/gdla.h declares.
 EXPORTED = ("gdla_latent_expand", "gdla_prefill_workspace_size", "gdla_prefill", "gdla_attend", "gdla_decode_workspace_size",
-            "gdla_decode", "gdla_decode_noalloc", "gdla_status_string", "gdla_workspace_status", "gdla_build_info")
+            "gdla_decode", "gdla_decode_noalloc", "gdla_status_string", "gdla_workspace_status", "gdla_build_info",
+            "gdla_diag_wait_timeout")
 
 _lock = threading.Lock()
 _lib = None
@@ -91,6 +92,8 @@ def load(path: str = LIB_PATH):
         lib.gdla_status_string.argtypes = [ctypes.c_int]
         lib.gdla_status_string.restype = ctypes.c_char_p
         lib.gdla_workspace_status.argtypes = [_vp, _vp]
+        lib.gdla_diag_wait_timeout.argtypes = [_vp, _vp]
+        lib.gdla_diag_wait_timeout.restype = ctypes.c_int
         lib.gdla_workspace_status.restype = ctypes.c_int
         lib.gdla_build_info.argtypes = []
         lib.gdla_build_info.restype = ctypes.c_char_p

@@ -289,6 +289,14 @@ gdla_status gdla_decode(const gdla_decode_args* a, void* stream) {
   return cuda_status(e);
 }
 
+gdla_status gdla_diag_wait_timeout(void* status_word, void* stream) {
+  if (!status_word || ((uintptr_t)status_word & 255) != 0) return GDLA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(status_word, 0, kStatusBytes, s);
+  if (e == cudaSuccess) e = launch_diag_wait(reinterpret_cast<int*>(status_word), s);
+  return cuda_status(e);
+}
+
 gdla_status gdla_workspace_status(const void* workspace, void* stream) {
   if (!workspace) return GDLA_ERR_INVALID_ARG;
   int code = 0;

@@ -72,4 +72,8 @@ cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStre
 bool decode_tc_supported(const DecodeParams& p, gdla_dtype dt);
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
 
+// ---- diagnostic: a device wait that can never complete ends at its limit and
+// records GDLA_ERR_TIMEOUT in the status word.
+cudaError_t launch_diag_wait(int* status, cudaStream_t s);
+
 }  // namespace gdla

@@ -226,6 +226,17 @@ const char* gdla_status_string(gdla_status s);
  * wait of the last call hit its cap. The word is cleared by every call. */
 gdla_status gdla_workspace_status(const void* workspace, void* stream);
 
+/* Diagnostic (the report has no counterpart): launches one CTA whose device-side
+ * wait can never complete (an mbarrier that nothing arrives on). The wait gives
+ * up after its limit, the same ~1 s bound every wait in the kernels has, and
+ * records GDLA_ERR_TIMEOUT in the status word at `status_word` (a 256-byte,
+ * 256-aligned device buffer owned by the caller, cleared here first), so that a
+ * caller can check, without faulting the GPU, that a stalled kernel ends and is
+ * reported through gdla_workspace_status. Returns GDLA_ERR_INVALID_ARG for a NULL
+ * or misaligned buffer, GDLA_ERR_CUDA if the launch fails, else GDLA_OK; the
+ * kernel runs asynchronously on `stream`. */
+gdla_status gdla_diag_wait_timeout(void* status_word, void* stream);
+
 /* Build information, for checks that the native library is the one loaded. */
 const char* gdla_build_info(void);
 
