@@ -12,6 +12,9 @@ in HBM:
 over the visible pairs, all ranks' work over the slowest rank's time);
 `decode` carries the decode's algorithmic GB/s (the cache read once). Inputs are
 larger than L2 (q alone is 805 MB), so no flush is needed between steps.
+`e2e` is the same prefill through gdla_prefill_host: the activations start in
+page-locked host memory and Y ends there, and the call overlaps the chunked
+copies with the kernels.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 With --impl reference the fp64 CPU oracle is timed on a bounded sample of the
@@ -40,8 +43,8 @@ CSRC = os.path.join(ROOT, "differential_latent_attention_gdla_b200", "csrc")
 # were taken on: once a kernel changes, its figure no longer applies and the bench
 # reports null.
 MEASURED_TRAFFIC = {
-    ("attn_tc_kernel", "b1_l32k_g3"): (2.165e9, ("attn_tc.cu", "sm100.cuh"), "4492c1bf09296e71"),
-    ("decode_tc_kernel", "b64_t32k"): (2.468e9, ("decode_tc.cu", "sm100.cuh"), "4e1c44c8fbc70fef"),
+    ("attn_tc_kernel", "b1_l32k_g3"): (2.164e9, ("attn_tc.cu", "sm100.cuh"), "79c179dd071b6bbd"),
+    ("decode_tc_kernel", "b64_t32k"): (2.468e9, ("decode_tc.cu", "sm100.cuh"), "fd915ee4fbe041b2"),
 }
 
 
@@ -69,6 +72,7 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-chunk", type=int, default=0, help="tokens per host-copy chunk (0: library default)")
     ap.add_argument("--prefill", default=PREFILL_NAME, help="prefill workload name (profiling uses smaller ones)")
     ap.add_argument("--decode", default=DECODE_NAME, help="decode workload name")
     return ap.parse_args()
@@ -295,23 +299,22 @@ def run_ours(a):
     att_tflops = f_att / (t_att * 1e-3) / 1e12
     dec_gbs = weak_scaling_value(db, world, t_dec * 1e-3) / 1e9
 
-    # end to end through the public call with host buffers (pinned), copies inside the timed region
+    # end to end through the public host-buffer call (gdla_prefill_host): the activations
+    # start in page-locked host memory and Y ends there; every copy is inside the timed region
     e2e = None
     if a.e2e_steps > 0:
         keys = ["c_kv", "k_rope", "q", "lam_logits", "gate_logits"]
         host = {k: pin[k].cpu().pin_memory() for k in keys}
         yh = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-        ws = torch.empty(gdla.prefill_workspace_size(B=P.B, L=P.L, d_c=P.d_c, d_rope=P.d_R, n_kv=P.n_kv,
-                                                     d_nope=P.d_n, d_v=P.d_v, g=P.g), dtype=torch.uint8, device=dev)
-        dev_in = {k: torch.empty_like(pin[k]) for k in keys}
+        ws = torch.empty(gdla.prefill_host_workspace_size(B=P.B, L=P.L, d_c=P.d_c, d_rope=P.d_R, n_kv=P.n_kv,
+                                                          d_nope=P.d_n, d_v=P.d_v, g=P.g,
+                                                          chunk_tokens=a.e2e_chunk),
+                         dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            for k in keys:
-                dev_in[k].copy_(host[k], non_blocking=True)
-            gdla.prefill(dev_in["c_kv"], pin["gamma"], dev_in["k_rope"], dev_in["q"], pin["w_ukv"], cos, sin,
-                         dev_in["lam_logits"], dev_in["gate_logits"], g=P.g, mask=P.mask, window=P.window, out=y,
-                         workspace=ws, stream=stream)
-            yh.copy_(y, non_blocking=True)
+            gdla.prefill_host(host["c_kv"], pin["gamma"], host["k_rope"], host["q"], pin["w_ukv"], cos, sin,
+                              host["lam_logits"], host["gate_logits"], g=P.g, mask=P.mask, window=P.window,
+                              chunk_tokens=a.e2e_chunk, out=yh, workspace=ws, stream=stream)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -326,7 +329,10 @@ def run_ours(a):
         h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
         e2e = {"value": weak_scaling_value(pf, world, t * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": yh.numel() * yh.element_size(), "ms_per_step": t}
-        del ws, dev_in, host
+        if int(gdla.workspace_status(ws)) != 0:
+            raise RuntimeError("device status word reports a failed wait (host-buffer prefill)")
+        e2e["chunk_tokens"] = a.e2e_chunk if a.e2e_chunk > 0 else "library default"
+        del ws, host
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:

@@ -20,7 +20,7 @@ import torch
 from . import _abi
 from ._abi import GDLA_BF16, GDLA_FP32, GDLA_MASK_CAUSAL, GDLA_MASK_SLIDING, GdlaError  # noqa: F401
 
-__all__ = ["prefill", "attend", "decode", "decode_noalloc", "latent_expand", "rope_tables", "yarn_rope_tables",
+__all__ = ["prefill", "prefill_host", "prefill_host_workspace_size", "attend", "decode", "decode_noalloc", "latent_expand", "rope_tables", "yarn_rope_tables",
            "yarn_mscale", "prefill_workspace_size", "decode_workspace_size", "workspace_status", "diag_wait_timeout",
            "build_info", "GdlaError"]
 
@@ -40,6 +40,14 @@ def _ptr(t) -> int | None:
         return None
     if not t.is_cuda:
         raise ValueError("GDLA tensors must be CUDA device tensors")
+    if not t.is_contiguous():
+        raise ValueError("GDLA tensors must be contiguous (row-major)")
+    return t.data_ptr()
+
+
+def _host_ptr(t) -> int:
+    if t.is_cuda:
+        raise ValueError("prefill_host takes its activations as CPU tensors (page-locked for copy overlap)")
     if not t.is_contiguous():
         raise ValueError("GDLA tensors must be contiguous (row-major)")
     return t.data_ptr()
@@ -123,7 +131,7 @@ def latent_expand(c_kv, gamma, k_rope, w_ukv, rope_cos, rope_sin, *, n_kv: int, 
 
 # --------------------------------------------------------------------- prefill
 def _prefill_args(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, out, g, mask, window,
-                  softmax_scale, rms_eps, cache_c_hat, cache_k_rope, workspace):
+                  softmax_scale, rms_eps, cache_c_hat, cache_k_rope, workspace, act_ptr=_ptr):
     B, L, d_c = c_kv.shape
     d_rope = k_rope.shape[-1]
     H_q, d_qk = q.shape[2], q.shape[3]
@@ -136,9 +144,9 @@ def _prefill_args(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits,
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     return _abi.PrefillArgs(B, L, d_c, d_rope, n_noise, d_nope, d_v, n_noise, g, _mask(mask), int(window),
                             float(softmax_scale), float(rms_eps), _dtype(c_kv), rope_cos.shape[0],
-                            _ptr(c_kv), _ptr(gamma), _ptr(k_rope), _ptr(q), _ptr(w_ukv), _ptr(rope_cos),
-                            _ptr(rope_sin), _ptr(lam_logits), _ptr(gate_logits), _ptr(out), _ptr(cache_c_hat),
-                            _ptr(cache_k_rope), ws_ptr, ws_bytes)
+                            act_ptr(c_kv), _ptr(gamma), act_ptr(k_rope), act_ptr(q), _ptr(w_ukv), _ptr(rope_cos),
+                            _ptr(rope_sin), act_ptr(lam_logits), act_ptr(gate_logits), act_ptr(out),
+                            _ptr(cache_c_hat), _ptr(cache_k_rope), ws_ptr, ws_bytes)
 
 
 def prefill_workspace_size(*, B, L, d_c, d_rope, n_kv, d_nope, d_v, g, dtype=torch.bfloat16) -> int:
@@ -173,24 +181,58 @@ def prefill(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_
     return out
 
 
+def prefill_host_workspace_size(*, B, L, d_c, d_rope, n_kv, d_nope, d_v, g, chunk_tokens=0,
+                                dtype=torch.bfloat16) -> int:
+    a = _abi.PrefillArgs()
+    a.B, a.L, a.d_c, a.d_rope, a.n_kv, a.d_nope, a.d_v, a.n_noise, a.g = B, L, d_c, d_rope, n_kv, d_nope, d_v, n_kv, g
+    a.dtype = _DT[dtype]
+    return int(_lib().gdla_prefill_host_workspace_size(ctypes.byref(a), int(chunk_tokens)))
+
+
+def prefill_host(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, *, g: int,
+                 mask: str = "causal", window: int = 0, softmax_scale: float = 0.0, rms_eps: float = 0.0,
+                 chunk_tokens: int = 0, out=None, workspace=None, cache_c_hat=None, cache_k_rope=None, stream=None):
+    """prefill() for activations in host memory: c_kv, k_rope, q, lam_logits,
+    gate_logits and the returned Y are CPU tensors (page-locked ones let the
+    copies overlap the kernels); gamma, w_ukv, the RoPE tables, the workspace
+    and the optional decode-cache outputs are CUDA tensors. The inputs travel
+    to the GPU in chunks of ``chunk_tokens`` tokens (0 = the library default)
+    while earlier chunks compute. Asynchronous like every call: synchronise
+    ``stream`` before reading Y."""
+    B, L = c_kv.shape[:2]
+    n_signal, d_v_guess = lam_logits.shape[-1], gate_logits.shape[-1]
+    if out is None:
+        out = torch.empty((B, L, n_signal, d_v_guess), dtype=c_kv.dtype, pin_memory=True)
+    a = _prefill_args(c_kv, gamma, k_rope, q, w_ukv, rope_cos, rope_sin, lam_logits, gate_logits, out, g, mask,
+                      window, softmax_scale, rms_eps, cache_c_hat, cache_k_rope, workspace, act_ptr=_host_ptr)
+    if workspace is None:
+        need = int(_lib().gdla_prefill_host_workspace_size(ctypes.byref(a), int(chunk_tokens)))
+        workspace = torch.empty(need, dtype=torch.uint8, device=gamma.device)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), need
+    _abi.check(_lib().gdla_prefill_host(ctypes.byref(a), int(chunk_tokens), _stream(stream)), "gdla_prefill_host")
+    return out
+
+
 def attend(q, kv, k_rope_rot, rope_cos, rope_sin, lam_logits, gate_logits, *, g: int, mask: str = "causal",
-           window: int = 0, softmax_scale: float = 0.0, out=None, status=None, stream=None):
+           window: int = 0, softmax_scale: float = 0.0, q_start: int = 0, out=None, status=None, stream=None):
     """Steps 3-8 over an expanded latent (the output of latent_expand); returns
-    Y [B, L, n_signal, d_v]. ``status`` is an optional 256-byte uint8 CUDA
-    tensor that receives the device status word."""
-    B, L, H_q, d_qk = q.shape
-    n_kv, dkv = kv.shape[2], kv.shape[3]
+    Y [B, q_len, n_signal, d_v]. The query side (q, lam_logits, gate_logits)
+    holds q_len = q.shape[1] rows per sequence at positions q_start ..
+    q_start + q_len - 1; kv and k_rope_rot hold all L key positions. ``status``
+    is an optional 256-byte uint8 CUDA tensor that receives the device status word."""
+    B, q_len, H_q, d_qk = q.shape
+    L, n_kv, dkv = kv.shape[1], kv.shape[2], kv.shape[3]
     d_rope = k_rope_rot.shape[-1]
     d_nope = d_qk - d_rope
     d_v = dkv - d_nope
     if out is None:
-        out = torch.empty((B, L, lam_logits.shape[-1], d_v), dtype=q.dtype, device=q.device)
+        out = torch.empty((B, q_len, lam_logits.shape[-1], d_v), dtype=q.dtype, device=q.device)
     if status is None:
         status = torch.empty(256, dtype=torch.uint8, device=q.device)
     a = _abi.AttendArgs(B, L, d_rope, n_kv, d_nope, d_v, H_q // (g + 1), g, _mask(mask), int(window),
                         float(softmax_scale), _dtype(q), rope_cos.shape[0], _ptr(q), _ptr(kv), _ptr(k_rope_rot),
                         _ptr(rope_cos), _ptr(rope_sin), _ptr(lam_logits), _ptr(gate_logits), _ptr(out), _ptr(status),
-                        status.numel())
+                        status.numel(), int(q_len), int(q_start))
     _abi.check(_lib().gdla_attend(ctypes.byref(a), _stream(stream)), "gdla_attend")
     return out
 

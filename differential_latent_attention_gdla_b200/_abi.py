@@ -43,7 +43,8 @@ class AttendArgs(ctypes.Structure):
         ("mask", ctypes.c_int), ("window", ctypes.c_int), ("softmax_scale", ctypes.c_float),
         ("dtype", ctypes.c_int), ("rope_max_pos", ctypes.c_int),
         ("q", _vp), ("kv", _vp), ("k_rope_rot", _vp), ("rope_cos", _vp), ("rope_sin", _vp), ("lam_logits", _vp),
-        ("gate_logits", _vp), ("out", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+        ("gate_logits", _vp), ("out", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+        ("q_len", ctypes.c_int), ("q_start", ctypes.c_int)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -56,9 +57,9 @@ class DecodeArgs(ctypes.Structure):
 
 
 # Every symbol include/gdla.h declares.
-EXPORTED = ("gdla_latent_expand", "gdla_prefill_workspace_size", "gdla_prefill", "gdla_attend", "gdla_decode_workspace_size",
-            "gdla_decode", "gdla_decode_noalloc", "gdla_status_string", "gdla_workspace_status", "gdla_build_info",
-            "gdla_diag_wait_timeout")
+EXPORTED = ("gdla_latent_expand", "gdla_prefill_workspace_size", "gdla_prefill", "gdla_prefill_host_workspace_size",
+            "gdla_prefill_host", "gdla_attend", "gdla_decode_workspace_size", "gdla_decode", "gdla_decode_noalloc",
+            "gdla_status_string", "gdla_workspace_status", "gdla_build_info", "gdla_diag_wait_timeout")
 
 _lock = threading.Lock()
 _lib = None
@@ -81,6 +82,10 @@ def load(path: str = LIB_PATH):
         lib.gdla_prefill_workspace_size.restype = ctypes.c_size_t
         lib.gdla_prefill.argtypes = [ctypes.POINTER(PrefillArgs), _vp]
         lib.gdla_prefill.restype = ctypes.c_int
+        lib.gdla_prefill_host_workspace_size.argtypes = [ctypes.POINTER(PrefillArgs), ctypes.c_int]
+        lib.gdla_prefill_host_workspace_size.restype = ctypes.c_size_t
+        lib.gdla_prefill_host.argtypes = [ctypes.POINTER(PrefillArgs), ctypes.c_int, _vp]
+        lib.gdla_prefill_host.restype = ctypes.c_int
         lib.gdla_attend.argtypes = [ctypes.POINTER(AttendArgs), _vp]
         lib.gdla_attend.restype = ctypes.c_int
         lib.gdla_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]

@@ -46,14 +46,15 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(AttnParams p) {
 
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
-  const int m0 = blockIdx.x * BM;
+  const int Lq = p.q_len, q_end = p.q_start + p.q_len;
+  const int m0 = p.q_start + blockIdx.x * BM;  // position of the block's first query row
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv;
   const int L = p.L;
   const float sl2 = p.scale * kLog2e;
 
-  const int last_row = min(L - 1, m0 + BM - 1);
+  const int last_row = min(q_end - 1, m0 + BM - 1);
   const int key_lo = p.sliding ? max(0, m0 - p.window + 1) : 0;
   const int t_lo = (key_lo / BN) * BN;
 
@@ -68,8 +69,8 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(AttnParams p) {
       const int r = e / DQK, k = e % DQK;
       const int i = m0 + r;
       float val = 0.f;
-      if (i < L) {
-        const T* qr = q + (((long)b * L + i) * H_q + head) * DQK;
+      if (i < q_end) {
+        const T* qr = q + (((long)b * Lq + (i - p.q_start)) * H_q + head) * DQK;
         if (k < DN) {
           val = to_f(qr[k]);
         } else {
@@ -198,8 +199,8 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(AttnParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int row = m0 + ty * 4 + i;
-        if (row >= L) continue;
-        const long tok = (long)b * L + row;
+        if (row >= q_end) continue;
+        const long tok = (long)b * Lq + (row - p.q_start);
         const float lam = sigmoidf_(p.lam[tok * n_S + sh]);
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
@@ -221,7 +222,7 @@ static cudaError_t launch_one(const AttnParams& p, cudaStream_t s) {
   auto k = attn_simt_kernel<T, DN, DR, DV>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((p.L + BM - 1) / BM), (unsigned)p.n_kv, (unsigned)p.B);
+  dim3 grid((unsigned)((p.q_len + BM - 1) / BM), (unsigned)p.n_kv, (unsigned)p.B);
   k<<<grid, NT, smem, s>>>(p);
   return cudaGetLastError();
 }

@@ -84,6 +84,7 @@ __device__ __forceinline__ uint32_t hn_off(int r, int c) { return (uint32_t)(r *
 
 struct AttnTcArgs {
   int B, L, n_kv, g, sliding, window, rope_max_pos, n_qtiles;
+  int q_len, q_start;  // query rows: positions q_start .. q_start+q_len-1; keys: 0 .. L-1
   float sl2;  // tau * log2(e)
   const float* cos_tab;
   const float* sin_tab;
@@ -125,9 +126,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int m_idx = a.n_qtiles - 1 - t % a.n_qtiles;
   const int h = (t / a.n_qtiles) % a.n_kv;
   const int b = t / (a.n_qtiles * a.n_kv);
-  const int m0 = m_idx * BM;
-  const int L = a.L;
-  const int last_row = min(L - 1, m0 + BM - 1);
+  const int m_loc = m_idx * BM;           // first query row of the block within the q/Y tensors
+  const int m0 = a.q_start + m_loc;       // its position in the sequence
+  const int q_end = a.q_start + a.q_len;  // one past the last query position
+  const int last_row = min(q_end - 1, m0 + BM - 1);
   const int key_lo = a.sliding ? max(0, m0 - a.window + 1) : 0;
   const int j_lo = key_lo / BN;
   const int n_tiles = last_row / BN - j_lo + 1;
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t bar = smem_u32(&bars.q_full[sl]);
         mbar_expect_tx(bar, QS_BYTES);
         for (int s = 0; s < 2; ++s)
-          tma_load_4d(smem_u32(qs_sm + sl * QS_BYTES + s * (BM * 128)), &tmQ, bar, k * 64, head_in(p, s), m0, b);
+          tma_load_4d(smem_u32(qs_sm + sl * QS_BYTES + s * (BM * 128)), &tmQ, bar, k * 64, head_in(p, s), m_loc, b);
         ++qk;
         return true;
       };
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int r = q4 * 32 + lane;           // stacked row = TMEM lane
     const int half = r >> 6;                // 0: first head of the pair, 1: second
     const int i = m0 + (r & (BM - 1));      // query position
-    const bool row_ok = i < L;
+    const bool row_ok = i < q_end;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const uint32_t tO = tmem + lane_base + kColO + CW * c;
     const uint32_t tQ = tmem + lane_base + kColQ;
@@ -349,7 +351,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint4 vh = *reinterpret_cast<const uint4*>(rowp + (((4 + c) ^ sw) << 4));
           const __nv_bfloat162* hl2 = reinterpret_cast<const __nv_bfloat162*>(&vl);
           const __nv_bfloat162* hh2 = reinterpret_cast<const __nv_bfloat162*>(&vh);
-          const int pos = row_ok ? i : L - 1;  // rows past the end are discarded; any table row will do
+          const int pos = row_ok ? i : q_end - 1;  // rows past the end are discarded; any table row will do
           const float* cs = a.cos_tab + (long)pos * (DR / 2) + 8 * c;
           const float* sn = a.sin_tab + (long)pos * (DR / 2) + 8 * c;
           uint32_t lo[4], hi[4];
@@ -515,7 +517,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           break;
         }
         const int sh = head_of(hl);  // signal head index
-        const long tok = (long)b * L + i;
+        const long tok = (long)b * a.q_len + (i - a.q_start);
         const float lam = row_ok ? sigmoidf_(a.lam[tok * n_S + sh]) : 0.f;
         const __nv_bfloat16* gp = a.gate + (tok * n_S + sh) * DV + cbase;
         __nv_bfloat16* op = a.out + (tok * n_S + sh) * DV + cbase;
@@ -566,9 +568,9 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   const int H_q = p.n_kv * (p.g + 1);
   CUtensorMap tq, tkv, tkr;
   {
-    const uint64_t dims[4] = {(uint64_t)(DN + DR), (uint64_t)H_q, (uint64_t)p.L, (uint64_t)p.B};
+    const uint64_t dims[4] = {(uint64_t)(DN + DR), (uint64_t)H_q, (uint64_t)p.q_len, (uint64_t)p.B};
     const uint64_t str[3] = {(uint64_t)(DN + DR) * 2, (uint64_t)H_q * (DN + DR) * 2,
-                             (uint64_t)p.L * H_q * (DN + DR) * 2};
+                             (uint64_t)p.q_len * H_q * (DN + DR) * 2};
     const uint32_t box[4] = {64, 1, BM, 1};
     if (!make_tmap_bf16(&tq, p.q, 4, dims, str, box)) return cudaErrorInvalidValue;
   }
@@ -587,7 +589,8 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   }
   AttnTcArgs a{};
   a.B = p.B; a.L = p.L; a.n_kv = p.n_kv; a.g = p.g; a.sliding = p.sliding; a.window = p.window;
-  a.rope_max_pos = p.rope_max_pos; a.n_qtiles = (p.L + BM - 1) / BM; a.sl2 = p.scale * kLog2e;
+  a.rope_max_pos = p.rope_max_pos; a.n_qtiles = (p.q_len + BM - 1) / BM;
+  a.q_len = p.q_len; a.q_start = p.q_start; a.sl2 = p.scale * kLog2e;
   a.cos_tab = p.cos_tab; a.sin_tab = p.sin_tab; a.lam = p.lam;
   a.gate = reinterpret_cast<const __nv_bfloat16*>(p.gate);
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);

@@ -97,8 +97,13 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   __shared__ float lsum[NQ];
   __shared__ float alpha_s[NQ];
   __shared__ volatile int abort_flag;
+  __shared__ int skip_cta;
 
-  if (sm100::earlier_failure(a.status)) return;  // an earlier CTA of this call timed out
+  // an earlier CTA of this call timed out: this one does no work (decided once for the CTA,
+  // so no thread is left waiting at a barrier that the others have skipped)
+  if (threadIdx.x == 0) skip_cta = sm100::earlier_failure(a.status) ? 1 : 0;
+  __syncthreads();
+  if (skip_cta) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.x, b = blockIdx.y;
   const int H_q = a.H_q;

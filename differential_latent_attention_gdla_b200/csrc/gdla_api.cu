@@ -55,6 +55,44 @@ PrefillLayout prefill_layout(const gdla_prefill_args* a) {
   return l;
 }
 
+// gdla_prefill_host: the prefill workspace, device copies of the whole batch's
+// latent inputs (c_kv, k_rope: 1152 bytes a token at the report's sizes, ~5% of
+// the per-token activations), then kHostSlots staging slots, one query chunk of
+// `chunk` tokens each, for q, lambda, gate and Y.
+constexpr int kHostSlots = 8;
+constexpr int kDefaultChunk = 2048;
+
+struct HostLayout {
+  PrefillLayout base;
+  int chunk;
+  size_t c_kv, k_rope;                // [B, L, d_c], [B, L, d_rope]
+  size_t q, lam, gate, out;           // slot 0; slot i at + i * the stride
+  size_t q_st, lam_st, gate_st, out_st;
+  size_t total;
+};
+
+HostLayout host_layout(const gdla_prefill_args* a, int chunk_tokens) {
+  HostLayout l;
+  l.base = prefill_layout(a);
+  l.chunk = chunk_tokens > 0 ? chunk_tokens : kDefaultChunk;
+  if (l.chunk > a->L) l.chunk = a->L;
+  const size_t es = esize(a->dtype), n = (size_t)l.chunk, n_S = (size_t)a->g * a->n_noise;
+  const size_t H_q = n_S + a->n_noise, tok = (size_t)a->B * (size_t)a->L;
+  l.q_st = align256(n * H_q * (a->d_nope + a->d_rope) * es);
+  l.lam_st = align256(n * n_S * sizeof(float));
+  l.gate_st = align256(n * n_S * a->d_v * es);
+  l.out_st = l.gate_st;
+  size_t off = l.base.total;
+  l.c_kv = off; off = align256(off + tok * a->d_c * es);
+  l.k_rope = off; off = align256(off + tok * a->d_rope * es);
+  l.q = off; off += kHostSlots * l.q_st;
+  l.lam = off; off += kHostSlots * l.lam_st;
+  l.gate = off; off += kHostSlots * l.gate_st;
+  l.out = off; off += kHostSlots * l.out_st;
+  l.total = off;
+  return l;
+}
+
 struct DecodeLayout {
   size_t status, q_abs, q_rot, part_o, part_ml, total;
   int n_splits, split_len;
@@ -167,7 +205,23 @@ const char* gdla_build_info(void) {
   return "libgdla sm_100a (tcgen05/TMA attention + expansion, split-KV decode); built " __DATE__ " " __TIME__;
 }
 
-gdla_status gdla_latent_expand(const gdla_expand_args* a, void* stream) {
+// Expansion of `tokens` consecutive tokens whose positions are pos0 + (t mod L);
+// every pointer already points at the first of them. The RoPE tables are shifted
+// by pos0 rows, so the norm/RoPE kernel sees positions t mod L.
+static cudaError_t expand_rows(const gdla_expand_args* a, long tokens, int L, int pos0, int* status,
+                               cudaStream_t s) {
+  const long half = a->d_rope / 2;
+  NormRopeParams np{tokens, L, a->d_c, a->d_rope, a->rope_max_pos - pos0,
+                    a->rms_eps > 0.f ? a->rms_eps : 1e-6f, a->c_kv, a->gamma, a->k_rope,
+                    a->rope_cos + pos0 * half, a->rope_sin + pos0 * half, a->c_hat_out, a->k_rope_out};
+  cudaError_t e = launch_norm_rope(np, a->dtype, s);
+  if (e != cudaSuccess) return e;
+  GemmParams gp{tokens, a->n_kv * (a->d_nope + a->d_v), a->d_c, a->c_hat_out, a->w_ukv, a->kv_out};
+  if (a->dtype == GDLA_BF16 && gemm_tc_supported(gp)) return launch_gemm_tc(gp, status, s);
+  return launch_gemm_simt(gp, a->dtype, s);
+}
+
+static gdla_status validate_expand(const gdla_expand_args* a) {
   if (!a) return GDLA_ERR_INVALID_ARG;
   gdla_status st = common_dims(a->B, a->L, a->d_c, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_kv, 1, a->dtype);
   if (st != GDLA_OK) return st;
@@ -176,24 +230,20 @@ gdla_status gdla_latent_expand(const gdla_expand_args* a, void* stream) {
                        a->kv_out, a->k_rope_out, a->c_hat_out};
   for (const void* p : req)
     if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
-  cudaStream_t s = (cudaStream_t)stream;
-  NormRopeParams np{(long)a->B * a->L, a->L, a->d_c, a->d_rope, a->rope_max_pos,
-                    a->rms_eps > 0.f ? a->rms_eps : 1e-6f, a->c_kv, a->gamma, a->k_rope,
-                    a->rope_cos, a->rope_sin, a->c_hat_out, a->k_rope_out};
-  cudaError_t e = launch_norm_rope(np, a->dtype, s);
-  if (e != cudaSuccess) return cuda_status(e);
-  GemmParams gp{(long)a->B * a->L, a->n_kv * (a->d_nope + a->d_v), a->d_c, a->c_hat_out, a->w_ukv, a->kv_out};
-  if (a->dtype == GDLA_BF16 && gemm_tc_supported(gp))
-    e = launch_gemm_tc(gp, nullptr, s);
-  else
-    e = launch_gemm_simt(gp, a->dtype, s);
-  return cuda_status(e);
+  return GDLA_OK;
+}
+
+gdla_status gdla_latent_expand(const gdla_expand_args* a, void* stream) {
+  gdla_status st = validate_expand(a);
+  if (st != GDLA_OK) return st;
+  return cuda_status(expand_rows(a, (long)a->B * a->L, a->L, 0, nullptr, (cudaStream_t)stream));
 }
 
 static gdla_status attend_impl(const gdla_attend_args* a, cudaStream_t s, bool clear_status) {
   AttnParams ap{};
   ap.B = a->B; ap.L = a->L; ap.n_kv = a->n_kv; ap.g = a->g; ap.d_nope = a->d_nope; ap.d_rope = a->d_rope;
   ap.d_v = a->d_v; ap.sliding = a->mask == GDLA_MASK_SLIDING; ap.window = ap.sliding ? a->window : 0;
+  ap.q_len = a->q_len > 0 ? a->q_len : a->L; ap.q_start = a->q_len > 0 ? a->q_start : 0;
   ap.rope_max_pos = a->rope_max_pos; ap.scale = default_scale(a->softmax_scale, a->d_nope, a->d_rope);
   ap.q = a->q; ap.kv = a->kv; ap.kr = a->k_rope_rot; ap.cos_tab = a->rope_cos; ap.sin_tab = a->rope_sin;
   ap.lam = a->lam_logits; ap.gate = a->gate_logits; ap.out = a->out; ap.status = (int*)a->workspace;
@@ -214,6 +264,9 @@ gdla_status gdla_attend(const gdla_attend_args* a, void* stream) {
   if (a->mask != GDLA_MASK_CAUSAL && a->mask != GDLA_MASK_SLIDING) return GDLA_ERR_INVALID_ARG;
   if (a->mask == GDLA_MASK_SLIDING && a->window < 1) return GDLA_ERR_INVALID_ARG;
   if (a->rope_max_pos < a->L) return GDLA_ERR_INVALID_ARG;
+  if (a->q_len < 0 || a->q_start < 0 || (a->q_len == 0 && a->q_start != 0) ||
+      (long)a->q_start + a->q_len > a->L)
+    return GDLA_ERR_INVALID_ARG;
   const void* req[] = {a->q, a->kv, a->k_rope_rot, a->rope_cos, a->rope_sin, a->lam_logits, a->gate_logits,
                        a->out, a->workspace};
   for (const void* p : req)
@@ -246,8 +299,8 @@ gdla_status gdla_prefill(const gdla_prefill_args* a, void* stream) {
   ea.rope_max_pos = a->rope_max_pos; ea.c_kv = a->c_kv; ea.gamma = a->gamma; ea.k_rope = a->k_rope;
   ea.w_ukv = a->w_ukv; ea.rope_cos = a->rope_cos; ea.rope_sin = a->rope_sin;
   ea.kv_out = kv; ea.k_rope_out = k_rot; ea.c_hat_out = c_hat;
-  st = gdla_latent_expand(&ea, stream);
-  if (st != GDLA_OK) return st;
+  e = expand_rows(&ea, (long)a->B * a->L, a->L, 0, status, s);
+  if (e != cudaSuccess) return cuda_status(e);
 
   gdla_attend_args aa{};
   aa.B = a->B; aa.L = a->L; aa.d_rope = a->d_rope; aa.n_kv = a->n_kv; aa.d_nope = a->d_nope; aa.d_v = a->d_v;
@@ -257,6 +310,157 @@ gdla_status gdla_prefill(const gdla_prefill_args* a, void* stream) {
   aa.lam_logits = a->lam_logits; aa.gate_logits = a->gate_logits; aa.out = a->out;
   aa.workspace = status; aa.workspace_bytes = kStatusBytes;
   return attend_impl(&aa, s, /*clear_status=*/false);
+}
+
+size_t gdla_prefill_host_workspace_size(const gdla_prefill_args* a, int chunk_tokens) {
+  if (!a || a->B < 1 || a->L < 1 || a->g < 1 || a->n_noise < 1) return 0;
+  return host_layout(a, chunk_tokens).total;
+}
+
+gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void* stream) {
+  if (!a) return GDLA_ERR_INVALID_ARG;
+  gdla_status st = common_dims(a->B, a->L, a->d_c, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_noise, a->g,
+                               a->dtype);
+  if (st != GDLA_OK) return st;
+  if (a->mask != GDLA_MASK_CAUSAL && a->mask != GDLA_MASK_SLIDING) return GDLA_ERR_INVALID_ARG;
+  if (a->mask == GDLA_MASK_SLIDING && a->window < 1) return GDLA_ERR_INVALID_ARG;
+  if (a->rope_max_pos < a->L) return GDLA_ERR_INVALID_ARG;
+  const void* dev[] = {a->gamma, a->w_ukv, a->rope_cos, a->rope_sin, a->workspace};
+  for (const void* p : dev)
+    if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  if (!opt_aligned16(a->cache_c_hat) || !opt_aligned16(a->cache_k_rope)) return GDLA_ERR_INVALID_ARG;
+  const void* host[] = {a->c_kv, a->k_rope, a->q, a->lam_logits, a->gate_logits, a->out};
+  for (const void* p : host)
+    if (!p) return GDLA_ERR_INVALID_ARG;
+  if (((uintptr_t)a->workspace & 255) != 0) return GDLA_ERR_INVALID_ARG;
+  const HostLayout lay = host_layout(a, chunk_tokens);
+  if (a->workspace_bytes < lay.total) return GDLA_ERR_INVALID_ARG;
+
+  cudaStream_t s = (cudaStream_t)stream;
+  char* ws = (char*)a->workspace;
+  int* status = (int*)(ws + lay.base.status);
+  char* c_hat = a->cache_c_hat ? (char*)a->cache_c_hat : ws + lay.base.c_hat;
+  char* k_rot = a->cache_k_rope ? (char*)a->cache_k_rope : ws + lay.base.k_rot;
+  char* kv = ws + lay.base.kv;
+  const size_t es = esize(a->dtype);
+  const int n_S = a->g * a->n_noise, H_q = n_S + a->n_noise;
+  // bytes per token of every per-token tensor
+  const size_t b_ckv = (size_t)a->d_c * es, b_kr = (size_t)a->d_rope * es;
+  const size_t b_q = (size_t)H_q * (a->d_nope + a->d_rope) * es, b_lam = (size_t)n_S * sizeof(float);
+  const size_t b_gate = (size_t)n_S * a->d_v * es, b_kv = (size_t)a->n_kv * (a->d_nope + a->d_v) * es;
+
+  // two copy streams; events: start, latent inputs landed, one per slot for inputs
+  // landed / compute done / output copied, and the end of each copy stream
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_kv = nullptr, ev_end = nullptr;
+  cudaEvent_t ev_in[kHostSlots] = {}, ev_comp[kHostSlots] = {}, ev_out[kHostSlots] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_kv, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_end, cudaEventDisableTiming);
+  for (int i = 0; i < kHostSlots && e == cudaSuccess; ++i) {
+    e = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_comp[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming);
+  }
+  bool forked = false;
+  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, kStatusBytes, s);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_start, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_start, 0);
+  forked = (e == cudaSuccess);
+
+  // 1. the latent inputs of the whole batch, then steps 1-3 for every token at once
+  //    (the same launch as gdla_prefill's expansion)
+  const size_t tok = (size_t)a->B * a->L;
+  char* d_ckv = ws + lay.c_kv;
+  char* d_kr = ws + lay.k_rope;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_ckv, a->c_kv, tok * b_ckv, cudaMemcpyDefault, s_in);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_kr, a->k_rope, tok * b_kr, cudaMemcpyDefault, s_in);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_kv, s_in);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_kv, 0);
+  if (e == cudaSuccess) {
+    gdla_expand_args ea{};
+    ea.B = a->B; ea.L = a->L; ea.d_c = a->d_c; ea.d_rope = a->d_rope; ea.n_kv = a->n_kv;
+    ea.d_nope = a->d_nope; ea.d_v = a->d_v; ea.dtype = a->dtype; ea.rms_eps = a->rms_eps;
+    ea.rope_max_pos = a->rope_max_pos; ea.gamma = a->gamma; ea.w_ukv = a->w_ukv;
+    ea.rope_cos = a->rope_cos; ea.rope_sin = a->rope_sin;
+    ea.c_kv = d_ckv; ea.k_rope = d_kr; ea.c_hat_out = c_hat; ea.k_rope_out = k_rot; ea.kv_out = kv;
+    e = expand_rows(&ea, (long)tok, a->L, 0, status, s);
+  }
+
+  // 2. query chunks, latest positions first: under the causal mask they see the
+  //    most keys, so the cheapest chunks are the last ones, whose kernels and
+  //    copy-back run after the final host-to-device copy
+  gdla_attend_args aa{};
+  aa.B = 1; aa.d_rope = a->d_rope; aa.n_kv = a->n_kv; aa.d_nope = a->d_nope; aa.d_v = a->d_v;
+  aa.n_noise = a->n_noise; aa.g = a->g; aa.mask = a->mask; aa.window = a->window;
+  aa.softmax_scale = a->softmax_scale; aa.dtype = a->dtype; aa.rope_max_pos = a->rope_max_pos;
+  aa.rope_cos = a->rope_cos; aa.rope_sin = a->rope_sin;
+  aa.workspace = status; aa.workspace_bytes = kStatusBytes;
+  const int n_chunks = (a->L + lay.chunk - 1) / lay.chunk;
+  long k = 0;  // chunks issued so far; chunk k uses slot k mod kHostSlots
+  for (int c = n_chunks - 1; c >= 0 && e == cudaSuccess; --c) {
+    for (int b = 0; b < a->B && e == cudaSuccess; ++b, ++k) {
+      const int t0 = c * lay.chunk;
+      const int n = a->L - t0 < lay.chunk ? a->L - t0 : lay.chunk;
+      const int sl = (int)(k % kHostSlots);
+      const size_t row = (size_t)b * a->L + t0;  // first token of the chunk in the [B, L] tensors
+      char* d_q = ws + lay.q + sl * lay.q_st;
+      char* d_lam = ws + lay.lam + sl * lay.lam_st;
+      char* d_gate = ws + lay.gate + sl * lay.gate_st;
+      char* d_out = ws + lay.out + sl * lay.out_st;
+      // inputs of chunk k, once chunk k - kHostSlots has finished reading the slot
+      if (k >= kHostSlots) e = cudaStreamWaitEvent(s_in, ev_comp[sl], 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(d_q, (const char*)a->q + row * b_q, n * b_q, cudaMemcpyDefault, s_in);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(d_lam, (const char*)a->lam_logits + row * b_lam, n * b_lam, cudaMemcpyDefault, s_in);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(d_gate, (const char*)a->gate_logits + row * b_gate, n * b_gate, cudaMemcpyDefault,
+                            s_in);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_in[sl], s_in);
+      // its attention, once the inputs landed and the slot's previous Y was copied out
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in[sl], 0);
+      if (e == cudaSuccess && k >= kHostSlots) e = cudaStreamWaitEvent(s, ev_out[sl], 0);
+      if (e == cudaSuccess) {
+        // the chunk's queries against the keys of positions 0 .. t0 + n - 1 of sequence b
+        aa.L = t0 + n; aa.q_len = n; aa.q_start = t0;
+        aa.q = d_q; aa.lam_logits = (const float*)d_lam; aa.gate_logits = d_gate; aa.out = d_out;
+        aa.kv = kv + (size_t)b * a->L * b_kv; aa.k_rope_rot = k_rot + (size_t)b * a->L * b_kr;
+        const gdla_status as = attend_impl(&aa, s, /*clear_status=*/false);
+        if (as != GDLA_OK) e = cudaErrorLaunchFailure;
+      }
+      if (e == cudaSuccess) e = cudaEventRecord(ev_comp[sl], s);
+      // Y rows of chunk k back to the host
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp[sl], 0);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync((char*)a->out + row * b_gate, d_out, n * b_gate, cudaMemcpyDefault, s_out);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_out[sl], s_out);
+    }
+  }
+  // join both copy streams into `stream`, also after a failure, so that the
+  // caller's later work (and a synchronise of `stream`) covers every copy
+  if (forked) {
+    cudaError_t j = cudaEventRecord(ev_end, s_in);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ev_end, 0);
+    if (j == cudaSuccess) j = cudaEventRecord(ev_end, s_out);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ev_end, 0);
+    if (e == cudaSuccess) e = j;
+  }
+  // released by the runtime once their pending work completes
+  for (int i = 0; i < kHostSlots; ++i) {
+    if (ev_in[i]) cudaEventDestroy(ev_in[i]);
+    if (ev_comp[i]) cudaEventDestroy(ev_comp[i]);
+    if (ev_out[i]) cudaEventDestroy(ev_out[i]);
+  }
+  if (ev_start) cudaEventDestroy(ev_start);
+  if (ev_kv) cudaEventDestroy(ev_kv);
+  if (ev_end) cudaEventDestroy(ev_end);
+  if (s_in) cudaStreamDestroy(s_in);
+  if (s_out) cudaStreamDestroy(s_out);
+  return cuda_status(e);
 }
 
 size_t gdla_decode_workspace_size(const gdla_decode_args* a) {

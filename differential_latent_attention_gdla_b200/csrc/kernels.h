@@ -32,17 +32,21 @@ bool gemm_tc_supported(const GemmParams& p);
 cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s);
 
 // ---- steps 3-8: attention of every head of a KV group + differential + gate.
+// The query side covers the block of positions q_start .. q_start+q_len-1 of every
+// sequence (q_len = L, q_start = 0 for a whole prefill); the key side covers
+// positions 0 .. L-1, and q_start + q_len <= L.
 struct AttnParams {
   int B, L, n_kv, g, d_nope, d_rope, d_v;
+  int q_len, q_start;
   int sliding, window, rope_max_pos;
   float scale;          // tau
-  const void* q;        // [B, L, H_q, d_nope+d_rope]
+  const void* q;        // [B, q_len, H_q, d_nope+d_rope]
   const void* kv;       // [B, L, n_kv, d_nope+d_v]
   const void* kr;       // [B, L, d_rope] rotated
   const float* cos_tab; const float* sin_tab;
-  const float* lam;     // [B, L, n_S]
-  const void* gate;     // [B, L, n_S, d_v]
-  void* out;            // [B, L, n_S, d_v]
+  const float* lam;     // [B, q_len, n_S]
+  const void* gate;     // [B, q_len, n_S, d_v]
+  void* out;            // [B, q_len, n_S, d_v]
   int* status;
 };
 cudaError_t launch_attn_simt(const AttnParams& p, gdla_dtype dt, cudaStream_t s);

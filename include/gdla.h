@@ -139,7 +139,18 @@ gdla_status gdla_prefill(const gdla_prefill_args* args, void* stream);
  * under the mask, differential subtraction and sigmoid gate, exactly as in
  * gdla_prefill. `kv` and `k_rope_rot` are the outputs of gdla_latent_expand
  * for the same batch. The workspace only carries the status word
- * (>= 256 bytes, 256-byte aligned). */
+ * (>= 256 bytes, 256-byte aligned).
+ *
+ * Query block (chunked prefill; the report has no counterpart, it is the same
+ * attention restricted to some query rows): with q_len > 0 only the queries at
+ * positions q_start .. q_start+q_len-1 of every sequence are computed. q,
+ * lam_logits, gate_logits and out then hold q_len rows per sequence
+ * ([B, q_len, ...]; row r is position q_start + r, which sets its RoPE angle
+ * and its mask), while kv and k_rope_rot keep their L rows (positions 0..L-1).
+ * Requires q_start >= 0 and q_start + q_len <= L, else GDLA_ERR_INVALID_ARG.
+ * q_len == 0 (a zero-initialised struct) selects all L rows, and then q_start
+ * must be 0. Every row's result is bit-identical to the whole-sequence call
+ * when q_start is a multiple of 64. */
 typedef struct {
   int B, L, d_rope, n_kv, d_nope, d_v, n_noise, g;
   gdla_mask mask;
@@ -157,9 +168,50 @@ typedef struct {
   void* out;                 /* [B, L, n_signal, d_v] */
   void* workspace;           /* status word */
   size_t workspace_bytes;
+  int q_len;                 /* query rows per sequence; 0 = L (see above) */
+  int q_start;               /* position of the first query row */
 } gdla_attend_args;
 
 gdla_status gdla_attend(const gdla_attend_args* args, void* stream);
+
+/* ------------------------------------------------------- prefill, host buffers
+ * The forward of gdla_prefill for activations held in host memory (the report
+ * has no counterpart; the arithmetic is gdla_prefill's, row for row). The layer's
+ * parameters stay on the GPU: gamma, w_ukv, rope_cos, rope_sin, and the optional
+ * cache_c_hat / cache_k_rope outputs are DEVICE pointers as in gdla_prefill. The
+ * activations are HOST pointers, in gdla_prefill's layouts:
+ *   inputs  c_kv, k_rope, q, lam_logits, gate_logits
+ *   output  out
+ * Page-locked host memory (cudaHostAlloc / cudaHostRegister) lets the copies
+ * overlap the kernels; pageable memory gives the same result without the overlap.
+ *
+ * The call first copies the latent inputs (c_kv, k_rope) of the whole batch
+ * and expands every token, as gdla_prefill does. Then every sequence's queries
+ * are cut into chunks of `chunk_tokens` tokens (<= 0 selects 2048; the last
+ * chunk of a sequence may be shorter). Each chunk's q, lambda and gate rows are
+ * copied to the device on a copy stream, attended (the query-block form of
+ * gdla_attend) on `stream`, and its rows of Y are copied back on a second copy
+ * stream, so the transfers of one chunk overlap the kernels of its neighbours.
+ * Chunks go latest positions first: under the causal mask they see the most
+ * keys, so the cheapest chunks come last, after the final host-to-device copy.
+ * With chunks of a multiple of 64 tokens the result is bit-identical to
+ * gdla_prefill's.
+ *
+ * The device workspace (>= gdla_prefill_host_workspace_size(args,
+ * chunk_tokens) bytes, 256-byte aligned) holds gdla_prefill's workspace, device
+ * copies of c_kv and k_rope, and eight chunk-sized staging slots per query-side
+ * tensor (q, lambda, gate, Y) that the chunks take in turn.
+ *
+ * Per call, the library creates two non-blocking copy streams and a few events.
+ * They are released once their work completes. All work is ordered after
+ * earlier work on `stream`, and later work on `stream` waits for all of it.
+ * Like every entry point, the call returns without synchronising, so `out` is
+ * valid only after `stream` has been synchronised, and the host inputs must
+ * stay unchanged until then. Errors as for gdla_prefill. A CUDA failure after
+ * the first copy was enqueued still joins the copy streams into `stream`
+ * before GDLA_ERR_CUDA is returned. */
+size_t gdla_prefill_host_workspace_size(const gdla_prefill_args* args, int chunk_tokens);
+gdla_status gdla_prefill_host(const gdla_prefill_args* args, int chunk_tokens, void* stream);
 
 /* --------------------------------------------------------------------- decode
  * One new token per sequence over the compact latent cache ("Motif 3:

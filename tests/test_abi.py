@@ -146,3 +146,59 @@ def test_expand_validation(lib):
     assert lib.gdla_latent_expand(ctypes.byref(a), None) == _abi.GDLA_ERR_INVALID_ARG  # table too short
     a.rope_max_pos = 10
     assert lib.gdla_latent_expand(ctypes.byref(a), None) == _abi.GDLA_ERR_INVALID_ARG  # NULL pointers
+
+
+def good_attend():
+    a = _abi.AttendArgs(2, 300, 64, 16, 128, 128, 16, 3, _abi.GDLA_MASK_CAUSAL, 0, 0.0, _abi.GDLA_BF16, 300)
+    base = 0x10000000
+    for i, f in enumerate(("q", "kv", "k_rope_rot", "rope_cos", "rope_sin", "lam_logits", "gate_logits", "out",
+                           "workspace")):
+        setattr(a, f, base + i * 0x1000000)
+    a.workspace_bytes = 256
+    return a
+
+
+def test_attend_query_block_validation(lib):
+    # the query block must lie inside the L key positions; q_len == 0 means all rows
+    E = _abi.GDLA_ERR_INVALID_ARG
+    for q_len, q_start in ((-1, 0), (10, -1), (0, 5), (301, 0), (200, 101), (1, 300)):
+        a = good_attend()
+        a.q_len, a.q_start = q_len, q_start
+        assert lib.gdla_attend(ctypes.byref(a), None) == E, (q_len, q_start)
+
+
+def test_prefill_host_validation_rejects_before_launch(lib):
+    def st(mut, chunk=256):
+        a = good_prefill()
+        a.workspace_bytes = lib.gdla_prefill_host_workspace_size(ctypes.byref(a), chunk)
+        mut(a)
+        return lib.gdla_prefill_host(ctypes.byref(a), chunk, None)
+
+    E, U = _abi.GDLA_ERR_INVALID_ARG, _abi.GDLA_ERR_UNSUPPORTED
+    assert st(lambda a: setattr(a, "q", 0)) == E                       # host input NULL
+    assert st(lambda a: setattr(a, "out", 0)) == E                     # host output NULL
+    assert st(lambda a: setattr(a, "gamma", 0x10000004)) == E          # device parameter misaligned
+    assert st(lambda a: setattr(a, "workspace", a.workspace + 16)) == E
+    assert st(lambda a: setattr(a, "workspace_bytes", a.workspace_bytes - 1)) == E
+    assert st(lambda a: setattr(a, "rope_max_pos", 99)) == E
+    assert st(lambda a: setattr(a, "g", 9)) == U
+    assert lib.gdla_prefill_host(None, 0, None) == E
+
+
+def test_prefill_host_workspace_size(lib):
+    # the prefill workspace, device copies of c_kv and k_rope, and eight chunk-sized
+    # staging slots for q, lambda, gate and Y
+    a = good_prefill()  # B=2, L=100, 16 KV heads, g=3: 64 query heads
+    base = lib.gdla_prefill_workspace_size(ctypes.byref(a))
+    latent = 2 * 100 * (512 + 64) * 2
+    s64 = lib.gdla_prefill_host_workspace_size(ctypes.byref(a), 64)
+    per_tok = 64 * 192 * 2 + 48 * 4 + 2 * 48 * 128 * 2  # q, lambda, gate + Y
+    assert s64 >= base + latent + 8 * 64 * per_tok
+    assert s64 <= base + latent + 2 * 256 + 8 * (64 * per_tok + 4 * 256)
+    assert s64 % 256 == 0
+    # chunks longer than the sequence (and the default) clamp to L
+    s_full = lib.gdla_prefill_host_workspace_size(ctypes.byref(a), 100)
+    assert lib.gdla_prefill_host_workspace_size(ctypes.byref(a), 5000) == s_full
+    assert lib.gdla_prefill_host_workspace_size(ctypes.byref(a), 0) == s_full
+    assert s_full > s64
+    assert lib.gdla_prefill_host_workspace_size(None, 64) == 0
