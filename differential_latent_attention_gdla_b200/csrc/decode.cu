@@ -20,9 +20,10 @@ namespace gdla {
 // Absorb blocks: KV group x 128 latent rows x (up to 48 query rows = sequences x heads of the group).
 constexpr int ABS_C = 128;   // latent rows per block: 32 threads x 4
 constexpr int ABS_R = 48;    // query rows per block: 8 warps x 6
-// Combine blocks: KV group x (up to 16 query rows); 32 threads x 4 value columns, 8 warps x 2 rows.
+// Combine blocks: KV group x (up to 16 query rows). The W_UV product gives each thread
+// 4 query rows x one 16-byte vector of value columns over one K-slice of every staged
+// block of latent rows; the slices' partial sums are added in a fixed order.
 constexpr int CMB_R = 16;
-constexpr int CMB_RPW = CMB_R / 8;  // query rows per warp
 constexpr int CMB_KC = 64;   // latent rows of W_UV staged per step
 constexpr int kMergeBatch = 12;  // split partials loaded together by one thread
 
@@ -245,8 +246,8 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
 //   O_lat = sum_s w_s O_s with w_s = exp2(m_s - M) / sum_s' exp2(m_s' - M) l_s'
 //   (log-sum-exp merge of the split-KV partials),
 //   H = O_lat W_UV, D = H_S - sigmoid(lam) H_N, Y = sigmoid(G) D.
-// W_UV is staged CMB_KC latent rows at a time; every thread accumulates a
-// CMB_RPW (query rows) x 4 (value columns) tile of H.
+// W_UV is staged CMB_KC latent rows at a time; every thread accumulates a 4 (query
+// rows) x 16-byte-vector (value columns) tile of H over one K-slice of each block.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   const int spb = combine_seqs(p.g);
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   float* hsm = olat + CMB_R * d_c;               // [CMB_R][DV]
   float* wgt = hsm + CMB_R * DV;                 // [CMB_R][NS] merge weights (scaled by 1 / denominator)
   T* wch = reinterpret_cast<T*>(wgt + CMB_R * NS);  // 2 x [CMB_KC][DV] staged W_UV rows
+  float* red = reinterpret_cast<float*>(wch + 2 * CMB_KC * DV);  // [K-slices][CMB_R][DV] partial products
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   const T* gate = reinterpret_cast<const T*>(p.gate);
   T* out = reinterpret_cast<T*>(p.out);
@@ -313,8 +315,9 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     for (int sp = lane; sp < NS; sp += 32) wgt[r * NS + sp] *= inv;
   }
   __syncthreads();
-  // ---- O_lat rows (float4 over the latent dimension)
+  // ---- O_lat rows (float4 over the latent dimension); rows R .. CMB_R-1 are zero
   const int c4 = d_c / 4;
+  for (int e = R * c4 + tid; e < CMB_R * c4; e += blockDim.x) reinterpret_cast<float4*>(olat)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = tid; e < R * c4; e += blockDim.x) {
     const int r = e / c4, v = e % c4;
     const int b = b0 + r / G1, head = head_of_row(r);
@@ -339,40 +342,58 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     }
     reinterpret_cast<float4*>(olat + r * d_c)[v] = acc;
   }
-  // ---- H = O_lat W_UV: thread rows CMB_RPW*warp .., value columns 4*lane .. +3
-  float acc[CMB_RPW][4];
+  // ---- H = O_lat W_UV. Thread (K-slice sl, rows 4 rg .. 4 rg + 3, columns VEC cg ..):
+  // per step it reads four W_UV rows as 16-byte vectors and O_lat as float4 along the
+  // latent dimension, so each shared load feeds 4 x VEC (or 4 x 4) FMAs
+  const int groups = DV / VEC;              // 16-byte column vectors per W_UV row
+  const int tps = groups * (CMB_R / 4);     // threads per K-slice
+  const int n_sl = 256 / tps;               // K-slices (2 .. 16 over the supported widths)
+  const int ks = CMB_KC / n_sl;             // latent rows per slice and staged block (multiple of 4)
+  const int sl = tid / tps, rg = (tid % tps) / groups, cg = tid % groups;
+  float acc[4][VEC];
 #pragma unroll
-  for (int i = 0; i < CMB_RPW; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  const bool col_ok = 4 * lane < DV;
+    for (int j = 0; j < VEC; ++j) acc[i][j] = 0.f;
   store_w(wch);
   __syncthreads();  // O_lat and the first W_UV rows are in shared memory
   for (int k0 = 0, it = 0; k0 < d_c; k0 += CMB_KC, ++it) {
     const T* wcur = wch + (it & 1) * (CMB_KC * DV);
     if (k0 + CMB_KC < d_c) load_w(k0 + CMB_KC);
-    if (col_ok) {
-#pragma unroll 4
-      for (int c = 0; c < CMB_KC; ++c) {
-        float wv[4];
+    for (int kk = 0; kk < ks; kk += 4) {
+      const int kr = sl * ks + kk;  // row of the staged block
+      float wv[4][VEC];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) wv[j] = to_f(wcur[c * DV + 4 * lane + j]);
+      for (int q = 0; q < 4; ++q) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(wcur + (kr + q) * DV + cg * VEC);
+        const T* xe = reinterpret_cast<const T*>(&raw);
 #pragma unroll
-        for (int i = 0; i < CMB_RPW; ++i) {
-          const float ov = olat[(CMB_RPW * warp + i) * d_c + k0 + c];
+        for (int j = 0; j < VEC; ++j) wv[q][j] = to_f(xe[j]);
+      }
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ov, wv[j], acc[i][j]);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const float4 ov = *reinterpret_cast<const float4*>(olat + (4 * rg + i) * d_c + k0 + kr);
+#pragma unroll
+        for (int j = 0; j < VEC; ++j)
+          acc[i][j] = fmaf(ov.w, wv[3][j], fmaf(ov.z, wv[2][j], fmaf(ov.y, wv[1][j], fmaf(ov.x, wv[0][j], acc[i][j]))));
       }
     }
     if (k0 + CMB_KC < d_c) store_w(wch + ((it + 1) & 1) * (CMB_KC * DV));
     __syncthreads();  // next rows staged; the buffer just read may be refilled
   }
-  if (col_ok) {
 #pragma unroll
-    for (int i = 0; i < CMB_RPW; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) hsm[(CMB_RPW * warp + i) * DV + 4 * lane + j] = acc[i][j];
+    for (int j = 0; j < VEC; j += 4)
+      *reinterpret_cast<float4*>(red + (sl * CMB_R + 4 * rg + i) * DV + cg * VEC + j) =
+          make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
+  __syncthreads();
+  // the slices' partial products, added in slice order (deterministic)
+  for (int e = tid; e < R * DV; e += blockDim.x) {
+    const int r = e / DV, c = e % DV;
+    float v = 0.f;
+    for (int q = 0; q < n_sl; ++q) v += red[(q * CMB_R + r) * DV + c];
+    hsm[r * DV + c] = v;
   }
   __syncthreads();
   // ---- differential and gate
@@ -445,8 +466,10 @@ cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaS
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
   const size_t esz = dt == GDLA_BF16 ? 2 : 4;
   const int spb = combine_seqs(p.g);
+  // O_lat, H, merge weights, two staged W_UV blocks, and the K-slices' partial products
+  // (n_slices x CMB_R x d_v = 1024 x (16 / esz) floats)
   const size_t smem = sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * p.d_v + (size_t)CMB_R * p.n_splits) +
-                      esz * 2 * (size_t)CMB_KC * p.d_v;
+                      esz * 2 * (size_t)CMB_KC * p.d_v + sizeof(float) * 1024 * (16 / esz);
   dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + spb - 1) / spb));
   cudaError_t e;
   if (dt == GDLA_BF16) {

@@ -137,6 +137,13 @@ DECODE_SMALL = [
     (wl.DecodeShape("decode sliding", B=2, T=700, n_kv=1, g=3), [700, 200], "sliding", 128),
     (wl.DecodeShape("decode d=32 fp32", B=2, T=150, d_c=64, d_R=16, n_kv=4, d_n=32, d_v=32, g=2, dtype="fp32"),
      [150, 77], "causal", 0),
+    # 40 sequences: the split heuristic gives splits of three 128-token tiles, so one block
+    # walks several tiles (ring reuse, both S^T / P^T buffers, the O^T rescale) and the
+    # lengths 1000 .. 103 leave ragged tails and short last splits
+    (wl.DecodeShape("decode multi-tile splits", B=40, T=1000, n_kv=16, g=2), [1000 - 23 * i for i in range(40)],
+     "causal", 0),
+    (wl.DecodeShape("decode multi-tile sliding W=300", B=40, T=1000, n_kv=16, g=2),
+     [1000 - 23 * i for i in range(40)], "sliding", 300),
 ]
 
 
@@ -189,6 +196,21 @@ def test_decode_peaked_softmax_rescale_path(scale):
     # exponents by ~|s| 2^-9, so only the RMS bar applies (a wrong rescale
     # would be an O(1) error)
     assert_parity(f64(y), ref, torch.bfloat16, f"decode peaked x{scale}", elementwise=False)
+
+
+def test_decode_peaked_multi_tile_splits():
+    """Peaked attention with several tiles per split block: the running maximum
+    jumps between tiles of one block, so O^T is rescaled in TMEM between value
+    passes (the path a one-tile split never takes)."""
+    shape = wl.DecodeShape("decode peaked multi-tile", B=40, T=1000, n_kv=16, g=2)
+    inp = wl.make_decode_inputs(shape, seed=13, device=DEV, act="unit", seqlens=[1000 - 17 * i for i in range(40)])
+    inp["q"] = (inp["q"].float() * 20.0).to(torch.bfloat16)
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g)
+    torch.cuda.synchronize()
+    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
+    assert_parity(f64(y), ref, torch.bfloat16, "decode peaked multi-tile", elementwise=False)
 
 
 # ------------------------------------------------------------------ YaRN context extension
