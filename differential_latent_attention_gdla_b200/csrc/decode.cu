@@ -19,26 +19,38 @@ namespace gdla {
 
 // Absorb blocks: KV group x 128 latent rows x (up to 48 query rows = sequences x heads of the group).
 constexpr int ABS_C = 128;   // latent rows per block: 32 threads x 4
-constexpr int ABS_R = 48;    // query rows per block: 8 warps x 6
+constexpr int ABS_R = 48;    // query rows per block at most: 8 warps x ABS_RPW
+constexpr int ABS_RPW = ABS_R / 8;
 // Combine blocks: KV group x (up to 16 query rows). The W_UV product gives each thread
 // 4 query rows x one 16-byte vector of value columns over one K-slice of every staged
 // block of latent rows; the slices' partial sums are added in a fixed order.
-constexpr int CMB_R = 16;
+constexpr int CMB_R = 16;   // query rows per block at most
 constexpr int CMB_KC = 64;   // latent rows of W_UV staged per step
 constexpr int kMergeBatch = 12;  // split partials loaded together by one thread
 
-__host__ __device__ inline int absorb_seqs(int g) { return max(1, ABS_R / (g + 1)); }
-__host__ __device__ inline int combine_seqs(int g) { return max(1, CMB_R / (g + 1)); }
+constexpr int kMinBlocks = 128;  // about one block per SM
+// Sequences per absorb / combine block: as many as the row tile holds (they share the
+// block's W_UK / W_UV reads), but few enough for about kMinBlocks blocks when the batch
+// is small. On B = 16 x 32768 tokens, 128 blocks each made the decode call 8 % faster
+// than 64; on B = 64 the tile limit decides (256 and 208 blocks).
+__host__ __device__ inline int absorb_seqs(const DecodeParams& p) {
+  const int fill = max(1, p.B * p.n_kv * ((p.d_c + ABS_C - 1) / ABS_C) / kMinBlocks);
+  return min(max(1, ABS_R / (p.g + 1)), fill);
+}
+__host__ __device__ inline int combine_seqs(const DecodeParams& p) {
+  const int fill = max(1, p.B * p.n_kv / kMinBlocks);
+  return min(max(1, CMB_R / (p.g + 1)), fill);
+}
 
 // q_abs[b, head, c] = sum_n W_UKV[c, h*(d_nope+d_v) + n] * q_nope[b, head, n] for the
 // g+1 heads of KV group h, and RoPE of their rotary parts at position seqlen-1.
-// Block (KV group h, 128 latent rows, absorb_seqs(g) sequences): W_UK (transposed) and
+// Block (KV group h, 128 latent rows, absorb_seqs(p) sequences): W_UK (transposed) and
 // the query rows are staged in shared memory; every thread accumulates a 4 (latent
-// rows) x 6 (query rows) tile, so each shared load feeds several FMAs.
+// rows) x ABS_RPW (query rows) tile, so each shared load feeds several FMAs.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
   const int h = blockIdx.x, c0 = blockIdx.y * ABS_C;
-  const int spb = absorb_seqs(p.g), b0 = blockIdx.z * spb;
+  const int spb = absorb_seqs(p), b0 = blockIdx.z * spb;
   const int nb = min(spb, p.B - b0);
   const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1;
   const int dqk = p.d_nope + p.d_rope, ncol = p.n_kv * (p.d_nope + p.d_v), DN = p.d_nope;
@@ -86,17 +98,18 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
   }
   __syncthreads();
   // thread: latent rows 4*lane .. +3, query rows 6*warp .. +5
-  float acc[6][4];
+  float acc[ABS_RPW][4];
 #pragma unroll
-  for (int i = 0; i < 6; ++i)
+  for (int i = 0; i < ABS_RPW; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  const float* qw = qs + (6 * warp) * DN;
+  const float* qw = qs + (ABS_RPW * warp) * DN;
+  const int n_end = ABS_RPW * warp < R ? DN : 0;  // warps whose rows are all padding skip the product
 #pragma unroll 4
-  for (int n = 0; n < DN; ++n) {
+  for (int n = 0; n < n_end; ++n) {
     const float4 wv = *reinterpret_cast<const float4*>(wt + n * WT + 4 * lane);
 #pragma unroll
-    for (int i = 0; i < 6; ++i) {
+    for (int i = 0; i < ABS_RPW; ++i) {
       const float qv = qw[i * DN + n];
       acc[i][0] = fmaf(wv.x, qv, acc[i][0]);
       acc[i][1] = fmaf(wv.y, qv, acc[i][1]);
@@ -106,8 +119,8 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
   }
   if (4 * lane < nrows) {
 #pragma unroll
-    for (int i = 0; i < 6; ++i) {
-      const int r = 6 * warp + i;
+    for (int i = 0; i < ABS_RPW; ++i) {
+      const int r = ABS_RPW * warp + i;
       if (r >= R) break;
       const int bl = r / G1, u = r % G1;
       const int head = u < p.g ? h * p.g + u : n_S + h;
@@ -242,7 +255,7 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
 }
 
 // Merge of the split partials and the output epilogue, for the g+1 heads of KV group h
-// and combine_seqs(g) sequences per block:
+// and combine_seqs(p) sequences per block:
 //   O_lat = sum_s w_s O_s with w_s = exp2(m_s - M) / sum_s' exp2(m_s' - M) l_s'
 //   (log-sum-exp merge of the split-KV partials),
 //   H = O_lat W_UV, D = H_S - sigmoid(lam) H_N, Y = sigmoid(G) D.
@@ -250,7 +263,7 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
 // rows) x 16-byte-vector (value columns) tile of H over one K-slice of each block.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
-  const int spb = combine_seqs(p.g);
+  const int spb = combine_seqs(p);
   const int h = blockIdx.x, b0 = blockIdx.y * spb;
   const int nb = min(spb, p.B - b0);
   const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1, NS = p.n_splits;
@@ -317,7 +330,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   __syncthreads();
   // ---- O_lat rows (float4 over the latent dimension); rows R .. CMB_R-1 are zero
   const int c4 = d_c / 4;
-  for (int e = R * c4 + tid; e < CMB_R * c4; e += blockDim.x) reinterpret_cast<float4*>(olat)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int e = R * c4 + tid; e < CMB_R * c4; e += blockDim.x)
+    reinterpret_cast<float4*>(olat)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = tid; e < R * c4; e += blockDim.x) {
     const int r = e / c4, v = e % c4;
     const int b = b0 + r / G1, head = head_of_row(r);
@@ -346,9 +360,12 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   // per step it reads four W_UV rows as 16-byte vectors and O_lat as float4 along the
   // latent dimension, so each shared load feeds 4 x VEC (or 4 x 4) FMAs
   const int groups = DV / VEC;              // 16-byte column vectors per W_UV row
-  const int tps = groups * (CMB_R / 4);     // threads per K-slice
-  const int n_sl = 256 / tps;               // K-slices (2 .. 16 over the supported widths)
+  const int rgc = R <= 4 ? 1 : (R <= 8 ? 2 : 4);  // groups of 4 rows covering the R query rows
+  const int RT = 4 * rgc;                   // rows of the tile (R rounded up)
+  const int tps = groups * rgc;             // threads per K-slice
+  const int n_sl = min(256 / tps, CMB_KC / 4);  // K-slices (each at least 4 latent rows per block)
   const int ks = CMB_KC / n_sl;             // latent rows per slice and staged block (multiple of 4)
+  const bool active = tid < n_sl * tps;
   const int sl = tid / tps, rg = (tid % tps) / groups, cg = tid % groups;
   float acc[4][VEC];
 #pragma unroll
@@ -360,7 +377,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
   for (int k0 = 0, it = 0; k0 < d_c; k0 += CMB_KC, ++it) {
     const T* wcur = wch + (it & 1) * (CMB_KC * DV);
     if (k0 + CMB_KC < d_c) load_w(k0 + CMB_KC);
-    for (int kk = 0; kk < ks; kk += 4) {
+    for (int kk = 0; active && kk < ks; kk += 4) {
       const int kr = sl * ks + kk;  // row of the staged block
       float wv[4][VEC];
 #pragma unroll
@@ -381,18 +398,20 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     if (k0 + CMB_KC < d_c) store_w(wch + ((it + 1) & 1) * (CMB_KC * DV));
     __syncthreads();  // next rows staged; the buffer just read may be refilled
   }
+  if (active) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < VEC; j += 4)
-      *reinterpret_cast<float4*>(red + (sl * CMB_R + 4 * rg + i) * DV + cg * VEC + j) =
-          make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
+      for (int j = 0; j < VEC; j += 4)
+        *reinterpret_cast<float4*>(red + (sl * RT + 4 * rg + i) * DV + cg * VEC + j) =
+            make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
+  }
   __syncthreads();
   // the slices' partial products, added in slice order (deterministic)
   for (int e = tid; e < R * DV; e += blockDim.x) {
     const int r = e / DV, c = e % DV;
     float v = 0.f;
-    for (int q = 0; q < n_sl; ++q) v += red[(q * CMB_R + r) * DV + c];
+    for (int q = 0; q < n_sl; ++q) v += red[(q * RT + r) * DV + c];
     hsm[r * DV + c] = v;
   }
   __syncthreads();
@@ -408,7 +427,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
 }
 
 cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
-  const int spb = absorb_seqs(p.g);
+  const int spb = absorb_seqs(p);
   dim3 grid((unsigned)p.n_kv, (unsigned)((p.d_c + ABS_C - 1) / ABS_C), (unsigned)((p.B + spb - 1) / spb));
   const size_t smem = sizeof(float) * ((size_t)p.d_nope * (ABS_C + 4) + (size_t)ABS_R * p.d_nope);
   cudaError_t e;
@@ -465,7 +484,7 @@ cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaS
 
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
   const size_t esz = dt == GDLA_BF16 ? 2 : 4;
-  const int spb = combine_seqs(p.g);
+  const int spb = combine_seqs(p);
   // O_lat, H, merge weights, two staged W_UV blocks, and the K-slices' partial products
   // (n_slices x CMB_R x d_v = 1024 x (16 / esz) floats)
   const size_t smem = sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * p.d_v + (size_t)CMB_R * p.n_splits) +

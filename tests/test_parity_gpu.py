@@ -198,6 +198,21 @@ def test_decode_peaked_softmax_rescale_path(scale):
     assert_parity(f64(y), ref, torch.bfloat16, f"decode peaked x{scale}", elementwise=False)
 
 
+@pytest.mark.parametrize("g", [1, 5, 8])
+def test_decode_group_sizes_every_element(g):
+    """g + 1 heads per KV group from 2 to 9: the combine blocks hold 8, 6 and 9 query
+    rows (one, two or four row groups of its W_UV tile) and the split kernel's padded
+    head columns vary."""
+    shape = wl.DecodeShape(f"decode g={g}", B=5, T=400, n_kv=2, g=g)
+    inp = wl.make_decode_inputs(shape, seed=14 + g, device=DEV, act="fan_in", seqlens=[400, 333, 129, 64, 1])
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g)
+    torch.cuda.synchronize()
+    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
+    assert_parity(f64(y), ref, torch.bfloat16, shape.name)
+
+
 def test_decode_peaked_multi_tile_splits():
     """Peaked attention with several tiles per split block: the running maximum
     jumps between tiles of one block, so O^T is rescaled in TMEM between value
