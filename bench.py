@@ -131,8 +131,8 @@ def oracle_sample(shape, inp_cpu, n_rows: int, kv_groups):
     G = len(kv_groups)
     flops = 2.0 * T * shape.d_c * G * (shape.d_n + shape.d_v)
     flops += sum(2.0 * (shape.d_qk + shape.d_v) * (i + 1) * G * (shape.g + 1) for _, i in rows)
-    desc = (f"{n_rows} query rows evenly spread over [0, {L}) of the B=1 L=32768 g=3 causal prefill, "
-            f"{G} of 16 KV groups ({G * (shape.g + 1)} heads), expansion of the {T} visible tokens")
+    desc = (f"{n_rows} query rows evenly spread over [0, {L}) of the B={shape.B} L={L} g={shape.g} {shape.mask} "
+            f"prefill, {G} of {shape.n_kv} KV groups ({G * (shape.g + 1)} heads), expansion of the {T} visible tokens")
     return dt, flops, desc, oracle.num_threads()
 
 
