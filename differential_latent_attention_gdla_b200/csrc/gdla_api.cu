@@ -61,6 +61,10 @@ PrefillLayout prefill_layout(const gdla_prefill_args* a) {
 // `chunk` tokens each, for q, lambda, gate and Y.
 constexpr int kHostSlots = 8;
 constexpr int kDefaultChunk = 2048;
+// query chunks alternate over this many compute streams: once the latent is
+// expanded the chunks are independent, and the blocks of one chunk's attention
+// fill the last, partly empty wave of its neighbour's
+constexpr int kComputeStreams = 2;
 
 struct HostLayout {
   PrefillLayout base;
@@ -349,15 +353,19 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
   const size_t b_q = (size_t)H_q * (a->d_nope + a->d_rope) * es, b_lam = (size_t)n_S * sizeof(float);
   const size_t b_gate = (size_t)n_S * a->d_v * es, b_kv = (size_t)a->n_kv * (a->d_nope + a->d_v) * es;
 
-  // two copy streams; events: start, latent inputs landed, one per slot for inputs
-  // landed / compute done / output copied, and the end of each copy stream
-  cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_kv = nullptr, ev_end = nullptr;
+  // two copy streams and the compute streams; events: start, latent inputs landed,
+  // latent expanded, one per slot for inputs landed / compute done / output copied,
+  // and the end of each side stream
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_c[kComputeStreams] = {};
+  cudaEvent_t ev_start = nullptr, ev_kv = nullptr, ev_exp = nullptr, ev_end = nullptr;
   cudaEvent_t ev_in[kHostSlots] = {}, ev_comp[kHostSlots] = {}, ev_out[kHostSlots] = {};
   cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+  for (int i = 0; i < kComputeStreams && e == cudaSuccess; ++i)
+    e = cudaStreamCreateWithFlags(&s_c[i], cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_kv, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_exp, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_end, cudaEventDisableTiming);
   for (int i = 0; i < kHostSlots && e == cudaSuccess; ++i) {
     e = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
@@ -369,6 +377,7 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
   if (e == cudaSuccess) e = cudaEventRecord(ev_start, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_start, 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_start, 0);
+  for (int i = 0; i < kComputeStreams && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(s_c[i], ev_start, 0);
   forked = (e == cudaSuccess);
 
   // 1. the latent inputs of the whole batch, then steps 1-3 for every token at once
@@ -389,6 +398,8 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
     ea.c_kv = d_ckv; ea.k_rope = d_kr; ea.c_hat_out = c_hat; ea.k_rope_out = k_rot; ea.kv_out = kv;
     e = expand_rows(&ea, (long)tok, a->L, 0, status, s);
   }
+  if (e == cudaSuccess) e = cudaEventRecord(ev_exp, s);
+  for (int i = 0; i < kComputeStreams && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(s_c[i], ev_exp, 0);
 
   // 2. query chunks, latest positions first: under the causal mask they see the
   //    most keys, so the cheapest chunks are the last ones, whose kernels and
@@ -399,13 +410,37 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
   aa.softmax_scale = a->softmax_scale; aa.dtype = a->dtype; aa.rope_max_pos = a->rope_max_pos;
   aa.rope_cos = a->rope_cos; aa.rope_sin = a->rope_sin;
   aa.workspace = status; aa.workspace_bytes = kStatusBytes;
-  const int n_chunks = (a->L + lay.chunk - 1) / lay.chunk;
-  long k = 0;  // chunks issued so far; chunk k uses slot k mod kHostSlots
-  for (int c = n_chunks - 1; c >= 0 && e == cudaSuccess; --c) {
+  // Pieces of a sequence, latest first: the chunk grid 0, chunk, 2 chunk, ..., with
+  // the topmost grid chunk cut at chunk/2 and 3 chunk/4 (multiples of 64). The first
+  // piece is then a quarter chunk: its copy, which no attention can overlap, is
+  // short. Every boundary stays a multiple of 64 when the chunk is one.
+  const int t_last = ((a->L - 1) / lay.chunk) * lay.chunk;  // start of the topmost grid chunk
+  int top_cut[4] = {t_last, 0, 0, 0}, n_top = 1;            // cuts of [t_last, L), ascending
+  {
+    const int h = (lay.chunk / 2) / 64 * 64, qc = (lay.chunk / 4) / 64 * 64;
+    if (qc >= 64) {
+      if (t_last + h < a->L) top_cut[n_top++] = t_last + h;
+      if (t_last + h + qc < a->L) top_cut[n_top++] = t_last + h + qc;
+    }
+    top_cut[n_top] = a->L;
+  }
+  const long n_pieces = n_top + t_last / lay.chunk;
+  auto piece = [&](long c, int& t0, int& n) {
+    if (c < n_top) {  // the topmost grid chunk, last cut first
+      t0 = top_cut[n_top - 1 - c];
+      n = top_cut[n_top - c] - t0;
+    } else {          // the full grid chunks below it, descending
+      t0 = t_last - (int)(c - n_top + 1) * lay.chunk;
+      n = lay.chunk;
+    }
+  };
+  long k = 0;  // pieces issued so far; piece k uses slot k mod kHostSlots
+  for (long c = 0; c < n_pieces && e == cudaSuccess; ++c) {
     for (int b = 0; b < a->B && e == cudaSuccess; ++b, ++k) {
-      const int t0 = c * lay.chunk;
-      const int n = a->L - t0 < lay.chunk ? a->L - t0 : lay.chunk;
+      int t0 = 0, n = 0;
+      piece(c, t0, n);
       const int sl = (int)(k % kHostSlots);
+      cudaStream_t cs = s_c[k % kComputeStreams];
       const size_t row = (size_t)b * a->L + t0;  // first token of the chunk in the [B, L] tensors
       char* d_q = ws + lay.q + sl * lay.q_st;
       char* d_lam = ws + lay.lam + sl * lay.lam_st;
@@ -422,17 +457,17 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
                             s_in);
       if (e == cudaSuccess) e = cudaEventRecord(ev_in[sl], s_in);
       // its attention, once the inputs landed and the slot's previous Y was copied out
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in[sl], 0);
-      if (e == cudaSuccess && k >= kHostSlots) e = cudaStreamWaitEvent(s, ev_out[sl], 0);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev_in[sl], 0);
+      if (e == cudaSuccess && k >= kHostSlots) e = cudaStreamWaitEvent(cs, ev_out[sl], 0);
       if (e == cudaSuccess) {
         // the chunk's queries against the keys of positions 0 .. t0 + n - 1 of sequence b
         aa.L = t0 + n; aa.q_len = n; aa.q_start = t0;
         aa.q = d_q; aa.lam_logits = (const float*)d_lam; aa.gate_logits = d_gate; aa.out = d_out;
         aa.kv = kv + (size_t)b * a->L * b_kv; aa.k_rope_rot = k_rot + (size_t)b * a->L * b_kr;
-        const gdla_status as = attend_impl(&aa, s, /*clear_status=*/false);
+        const gdla_status as = attend_impl(&aa, cs, /*clear_status=*/false);
         if (as != GDLA_OK) e = cudaErrorLaunchFailure;
       }
-      if (e == cudaSuccess) e = cudaEventRecord(ev_comp[sl], s);
+      if (e == cudaSuccess) e = cudaEventRecord(ev_comp[sl], cs);
       // Y rows of chunk k back to the host
       if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp[sl], 0);
       if (e == cudaSuccess)
@@ -440,13 +475,16 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
       if (e == cudaSuccess) e = cudaEventRecord(ev_out[sl], s_out);
     }
   }
-  // join both copy streams into `stream`, also after a failure, so that the
-  // caller's later work (and a synchronise of `stream`) covers every copy
+  // join every side stream into `stream`, also after a failure, so that the
+  // caller's later work (and a synchronise of `stream`) covers every copy and kernel
   if (forked) {
-    cudaError_t j = cudaEventRecord(ev_end, s_in);
-    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ev_end, 0);
-    if (j == cudaSuccess) j = cudaEventRecord(ev_end, s_out);
-    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ev_end, 0);
+    cudaStream_t side[2 + kComputeStreams] = {s_in, s_out};
+    for (int i = 0; i < kComputeStreams; ++i) side[2 + i] = s_c[i];
+    cudaError_t j = cudaSuccess;
+    for (cudaStream_t x : side) {
+      if (j == cudaSuccess) j = cudaEventRecord(ev_end, x);
+      if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ev_end, 0);
+    }
     if (e == cudaSuccess) e = j;
   }
   // released by the runtime once their pending work completes
@@ -457,9 +495,12 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
   }
   if (ev_start) cudaEventDestroy(ev_start);
   if (ev_kv) cudaEventDestroy(ev_kv);
+  if (ev_exp) cudaEventDestroy(ev_exp);
   if (ev_end) cudaEventDestroy(ev_end);
   if (s_in) cudaStreamDestroy(s_in);
   if (s_out) cudaStreamDestroy(s_out);
+  for (int i = 0; i < kComputeStreams; ++i)
+    if (s_c[i]) cudaStreamDestroy(s_c[i]);
   return cuda_status(e);
 }
 

@@ -194,15 +194,19 @@ gdla_status gdla_attend(const gdla_attend_args* args, void* stream);
  * stream, so the transfers of one chunk overlap the kernels of its neighbours.
  * Chunks go latest positions first: under the causal mask they see the most
  * keys, so the cheapest chunks come last, after the final host-to-device copy.
- * With chunks of a multiple of 64 tokens the result is bit-identical to
- * gdla_prefill's.
+ * The topmost chunk of a sequence is cut at its half and three-quarter marks
+ * (rounded down to 64 tokens), so the first copy, which no kernel overlaps, is
+ * a quarter chunk. The chunks' attention alternates over two internal compute
+ * streams. With chunks of a multiple of 64 tokens the result is bit-identical
+ * to gdla_prefill's.
  *
  * The device workspace (>= gdla_prefill_host_workspace_size(args,
  * chunk_tokens) bytes, 256-byte aligned) holds gdla_prefill's workspace, device
  * copies of c_kv and k_rope, and eight chunk-sized staging slots per query-side
  * tensor (q, lambda, gate, Y) that the chunks take in turn.
  *
- * Per call, the library creates two non-blocking copy streams and a few events.
+ * Per call, the library creates two non-blocking copy streams, two compute
+ * streams and a few events.
  * They are released once their work completes. All work is ordered after
  * earlier work on `stream`, and later work on `stream` waits for all of it.
  * Like every entry point, the call returns without synchronising, so `out` is
