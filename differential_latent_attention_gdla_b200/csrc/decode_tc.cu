@@ -113,6 +113,25 @@ __global__ void __launch_bounds__(DTHREADS, 1)
   const int jt0 = (t0 / TT) * TT;
   const int n_tiles = (t1 > t0) ? (t1 - jt0 + TT - 1) / TT : 0;
 
+  // the TMA loads of cache tile k into stage k % DSTAGES, and its L2 prefetch
+  auto load_tile = [&](int k) {
+    const int st = k % DSTAGES;
+    const uint32_t bar = smem_u32(&bars.full[st]);
+    const uint32_t dst = smem_u32(tiles + st * TILE_BYTES);
+    const int j0 = jt0 + k * TT;
+    mbar_expect_tx(bar, TILE_BYTES);
+    for (int bx = 0; bx < NBOX - 1; ++bx) tma_load_3d(dst + bx * (TT * 128), &tmC, bar, bx * 64, j0, b);
+    tma_load_3d(dst + (NBOX - 1) * (TT * 128), &tmR, bar, 0, j0, b);
+  };
+  auto prefetch_tile = [&](int q) {
+    const int j = jt0 + q * TT;
+    for (int bx = 0; bx < NBOX - 1; ++bx) tma_prefetch_3d(&tmC, bx * 64, j, b);
+    tma_prefetch_3d(&tmR, 0, j, b);
+  };
+  // thread 0 (the producer lane) loads the first tiles right after initialising the
+  // barriers, so that their HBM latency overlaps the staging of the query below
+  const int n_early = min(DSTAGES, n_tiles);
+
   if (threadIdx.x == 0) {
     for (int i = 0; i < DSTAGES; ++i) {
       mbar_init(smem_u32(&bars.full[i]), 1);
@@ -129,6 +148,8 @@ __global__ void __launch_bounds__(DTHREADS, 1)
     abort_flag = 0;
     prefetch_tmap(&tmC);
     prefetch_tmap(&tmR);
+    for (int k = 0; k < n_early; ++k) load_tile(k);
+    for (int q = max(n_early, kPf); q < n_early + kPf && q < n_tiles; ++q) prefetch_tile(q);
   }
   // Qcat^T in bf16, pre-scaled by tau*log2(e), K-major with the 128-byte swizzle
   for (int e = threadIdx.x; e < NQ * NBOX * 8; e += DTHREADS) {
@@ -168,13 +189,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
       // tile's value MMAs finish, so two slots alone keep too few bytes in flight
       // to cover the HBM latency. One tile ahead measured best (7 % on B=64 x 32768
       // tokens); two to four tiles ahead were slower.
-      auto prefetch_tile = [&](int q) {
-        const int j = jt0 + q * TT;
-        for (int bx = 0; bx < NBOX - 1; ++bx) tma_prefetch_3d(&tmC, bx * 64, j, b);
-        tma_prefetch_3d(&tmR, 0, j, b);
-      };
-      for (int q = DSTAGES; q < kPf && q < n_tiles; ++q) prefetch_tile(q);
-      int k = 0;
+      int k = n_early;  // tiles 0 .. n_early-1 were issued during the set-up
       for (; k < n_tiles && !abort_flag; ++k) {
         const int st = k % DSTAGES;
         if (k + kPf < n_tiles) prefetch_tile(k + kPf);
@@ -183,12 +198,7 @@ __global__ void __launch_bounds__(DTHREADS, 1)
           abort_flag = 1;
           break;
         }
-        const uint32_t bar = smem_u32(&bars.full[st]);
-        const uint32_t dst = smem_u32(tiles + st * TILE_BYTES);
-        const int j0 = jt0 + k * TT;
-        mbar_expect_tx(bar, TILE_BYTES);
-        for (int bx = 0; bx < NBOX - 1; ++bx) tma_load_3d(dst + bx * (TT * 128), &tmC, bar, bx * 64, j0, b);
-        tma_load_3d(dst + (NBOX - 1) * (TT * 128), &tmR, bar, 0, j0, b);
+        load_tile(k);
       }
       if (abort_flag)
         for (int q = (k > DSTAGES ? k - DSTAGES : 0); q < k; ++q)
