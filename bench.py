@@ -44,7 +44,7 @@ CSRC = os.path.join(ROOT, "differential_latent_attention_gdla_b200", "csrc")
 # reports null.
 MEASURED_TRAFFIC = {
     ("attn_tc_kernel", "b1_l32k_g3"): (2.165e9, ("attn_tc.cu", "sm100.cuh"), "79c179dd071b6bbd"),
-    ("decode_tc_kernel", "b64_t32k"): (2.473e9, ("decode_tc.cu", "sm100.cuh"), "1ebe5864269158f6"),
+    ("decode_tc_kernel", "b64_t32k"): (2.474e9, ("decode_tc.cu", "sm100.cuh"), "5de5419009465d0a"),
 }
 
 
