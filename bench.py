@@ -170,8 +170,10 @@ def run_reference(a):
 class ClockSampler:
     def __init__(self, index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else f"/tmp/gdla_clocks_{os.getpid()}.csv"
+        # raw samples go to $GDLA_CLOCKS_DIR/clocks_rank<i>.csv when set (to keep them), else to /tmp
+        out_dir = os.environ.get("GDLA_CLOCKS_DIR")
+        self.path = (os.path.join(out_dir, f"clocks_rank{index}.csv") if out_dir
+                     else f"/tmp/gdla_clocks_{os.getpid()}_{index}.csv")
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
