@@ -54,6 +54,7 @@ def _load():
             lib = ctypes.CDLL(_LIB)
             lib.gdla_oracle_num_threads.restype = ctypes.c_int
             lib.gdla_oracle_latent_norm.argtypes = [_dp, _dp, ctypes.c_long, ctypes.c_int, ctypes.c_double, _dp]
+            lib.gdla_oracle_project.argtypes = [_dp, ctypes.c_long, ctypes.c_int, _dp, ctypes.c_int, _dp]
             lib.gdla_oracle_expand_head.argtypes = [_dp, _dp, ctypes.c_long, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp]
             lib.gdla_oracle_rope.argtypes = [_dp, ctypes.c_long, ctypes.c_int, ctypes.c_double, _dp]
@@ -104,6 +105,31 @@ def latent_norm(c, gamma, eps: float = DEFAULT_EPS) -> np.ndarray:
     out = np.empty_like(c)
     _load().gdla_oracle_latent_norm(_p(c), _p(gamma), T, d_c, eps, _p(out))
     return out
+
+
+def project(a, w) -> np.ndarray:
+    """out [T, N] = a [T, K] @ w [K, N], summed in increasing k (plain loops)."""
+    a = _d(a)
+    w = _d(w)
+    T, K = a.shape
+    N = w.shape[1]
+    out = np.empty((T, N))
+    _load().gdla_oracle_project(_p(a), T, K, _p(w), N, _p(out))
+    return out
+
+
+def gate_logits(c_q, gamma_q, w_g, eps: float = DEFAULT_EPS) -> np.ndarray:
+    """Gate logits G [T, n_S * d_v] from the query latent c_q [T, d_q]: the latent is
+    RMS-normalised (the same normalisation as step 1, with its own gain gamma_q) and
+    projected by W_G [d_q, n_S * d_v] ("Motif 3: Technical Report", section
+    "Architecture": the gate is computed from the normalised query latent)."""
+    return project(latent_norm(c_q, gamma_q, eps), w_g)
+
+
+def lambda_logits(x, w_lam) -> np.ndarray:
+    """lambda logits [T, n_S] = x [T, d_x] @ W_lambda [d_x, n_S] ("Motif 3: Technical
+    Report", section "Architecture": lambda_t = sigmoid(x_t W_lambda))."""
+    return project(x, w_lam)
 
 
 def expand_head(c_hat, w_ukv, n_kv: int, d_n: int, d_v: int, h: int):

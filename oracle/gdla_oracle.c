@@ -76,6 +76,22 @@ void gdla_oracle_latent_norm(const double* c, const double* gamma, long T, int d
   }
 }
 
+/* The inputs of the differential epilogue from the layer's activations ("Motif 3:
+ * Technical Report", section "Architecture": lambda_t = sigmoid(x_t W_lambda), and
+ * an element-wise sigmoid gate computed from the normalised query latent, i.e.
+ * G_t = c_hat_Q,t W_G): a plain row-by-matrix product
+ *   out[t, n] = sum_{k=0}^{K-1} a[t, k] * w[k, n],
+ * summed in increasing k. The query latent is normalised with
+ * gdla_oracle_latent_norm before it is projected. */
+void gdla_oracle_project(const double* a, long T, int K, const double* w, int N, double* out) {
+  for (long t = 0; t < T; ++t)
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += a[t * K + k] * w[(long)k * N + n];
+      out[t * N + n] = acc;
+    }
+}
+
 /* One token of step 2: out[n] = sum_{k=0}^{d_c-1} c_hat[k] * W[k, col0+n], summed in
  * increasing k for every n (the loop over n is innermost only for memory order). */
 static void expand_token(const double* c_hat_t, const double* w_ukv, int d_c, long ncol, long col0,

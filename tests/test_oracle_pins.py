@@ -498,3 +498,55 @@ def test_prefill_explicit_frequencies_match_base_and_matrix_form():
                                 inp["lam"][b], inp["gate"][b], inp["g"], inp["d_n"], inp["d_v"], oracle.MASK_CAUSAL, 0,
                                 theta=theta, scale=scale)
         np.testing.assert_allclose(y[b], ey, rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------------------------------ gate and lambda logits
+# "Motif 3: Technical Report", section "Architecture": lambda_t = sigmoid(x_t W_lambda),
+# and the sigmoid gate is computed from the normalised query latent (G = c_hat_Q W_G).
+def test_project_exact_on_small_integers():
+    # integer entries: every product and sum is exact in fp64, so the oracle must equal
+    # the sum of products computed with Python integers
+    a = RNG.integers(-9, 10, size=(4, 7))
+    w = RNG.integers(-9, 10, size=(7, 5))
+    want = [[sum(int(a[t, k]) * int(w[k, n]) for k in range(7)) for n in range(5)] for t in range(4)]
+    assert np.array_equal(oracle.project(a.astype(float), w.astype(float)), np.array(want, dtype=float))
+
+
+def test_project_one_hot_rows_pick_weight_rows():
+    w = RNG.standard_normal((6, 3))
+    a = np.eye(6)[[4, 0, 5]]
+    assert np.array_equal(oracle.project(a, w), w[[4, 0, 5]])
+
+
+def test_lambda_logits_are_linear_in_x():
+    w = RNG.standard_normal((16, 5))
+    x1, x2 = RNG.standard_normal((3, 16)), RNG.standard_normal((3, 16))
+    lhs = oracle.lambda_logits(2.0 * x1 - 3.0 * x2, w)
+    rhs = 2.0 * oracle.lambda_logits(x1, w) - 3.0 * oracle.lambda_logits(x2, w)
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+
+
+def test_gate_logits_of_a_constant_latent_row():
+    # c_Q = a * ones: its RMS is |a|, so (eps = 0) c_hat = sign(a) gamma_q and G = sign(a) gamma_q @ W_G
+    d_q, n = 8, 6
+    gam = 1.0 + 0.1 * RNG.standard_normal(d_q)
+    w = RNG.standard_normal((d_q, n))
+    c = np.array([[3.0] * d_q, [-0.25] * d_q])
+    got = oracle.gate_logits(c, gam, w, eps=0.0)
+    assert np.allclose(got[0], gam @ w, rtol=1e-13, atol=1e-13)
+    assert np.allclose(got[1], -(gam @ w), rtol=1e-13, atol=1e-13)
+
+
+def test_gate_logits_normalise_before_projecting():
+    # scale invariance of the normalised latent (eps = 0), and with W_G = I the gate
+    # logits are the normalised latent itself, whose mean square is gamma-weighted 1
+    d_q = 12
+    gam = np.ones(d_q)
+    c = RNG.standard_normal((5, d_q))
+    g1 = oracle.gate_logits(c, gam, np.eye(d_q), eps=0.0)
+    g2 = oracle.gate_logits(7.5 * c, gam, np.eye(d_q), eps=0.0)
+    assert np.allclose(g1, g2, rtol=1e-13, atol=1e-13)
+    assert np.allclose((g1 ** 2).mean(axis=1), 1.0, rtol=1e-13)
+    # the gain multiplies latent column k, i.e. row k of W_G
+    gam2 = np.arange(1.0, d_q + 1)
+    assert np.allclose(oracle.gate_logits(c, gam2, np.eye(d_q), eps=0.0), g1 * gam2, rtol=1e-13)
