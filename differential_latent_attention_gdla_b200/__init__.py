@@ -20,7 +20,7 @@ import torch
 from . import _abi
 from ._abi import GDLA_BF16, GDLA_FP32, GDLA_MASK_CAUSAL, GDLA_MASK_SLIDING, GdlaError  # noqa: F401
 
-__all__ = ["prefill", "prefill_host", "prefill_host_workspace_size", "attend", "decode", "decode_noalloc", "latent_expand", "rope_tables", "yarn_rope_tables",
+__all__ = ["prefill", "prefill_host", "prefill_host_workspace_size", "gates", "attend", "decode", "decode_noalloc", "latent_expand", "rope_tables", "yarn_rope_tables",
            "yarn_mscale", "prefill_workspace_size", "decode_workspace_size", "workspace_status", "diag_wait_timeout",
            "build_info", "GdlaError"]
 
@@ -235,6 +235,39 @@ def attend(q, kv, k_rope_rot, rope_cos, rope_sin, lam_logits, gate_logits, *, g:
                         status.numel(), int(q_len), int(q_start))
     _abi.check(_lib().gdla_attend(ctypes.byref(a), _stream(stream)), "gdla_attend")
     return out
+
+
+# ----------------------------------------------------------------------- gates
+def gates(c_q=None, gamma_q=None, w_g=None, x=None, w_lambda=None, *, n_signal: int, d_v: int = 0,
+          rms_eps: float = 0.0, gate_out=None, lam_out=None, workspace=None, stream=None):
+    """Gate and lambda logits from the layer's activations: gate_logits =
+    RMSNorm(c_q; gamma_q) @ w_g as [*, n_signal, d_v] (dtype of c_q) and
+    lam_logits = x @ w_lambda as [*, n_signal] fp32, where * is the leading
+    [B, L] (or [B]) of c_q / x. Pass only (c_q, gamma_q, w_g) or only
+    (x, w_lambda) to compute one of them. Returns (gate_logits, lam_logits),
+    None for the half not computed."""
+    if c_q is None and x is None:
+        raise ValueError("gates needs c_q (gate) and/or x (lambda)")
+    ref = c_q if c_q is not None else x
+    lead = tuple(ref.shape[:-1])
+    B, L = (lead[0], lead[1]) if len(lead) == 2 else (lead[0], 1)
+    d_q = c_q.shape[-1] if c_q is not None else 0
+    d_x = x.shape[-1] if x is not None else 0
+    if c_q is not None:
+        if d_v <= 0:
+            d_v = w_g.shape[1] // n_signal
+        if gate_out is None:
+            gate_out = torch.empty(lead + (n_signal, d_v), dtype=c_q.dtype, device=c_q.device)
+    if x is not None and lam_out is None:
+        lam_out = torch.empty(lead + (n_signal,), dtype=torch.float32, device=x.device)
+    a = _abi.GatesArgs(B, L, d_q, d_x, n_signal, d_v, _dtype(ref), float(rms_eps), _ptr(c_q), _ptr(gamma_q),
+                       _ptr(w_g), _ptr(x), _ptr(w_lambda), _ptr(gate_out), _ptr(lam_out), None, 0)
+    need = int(_lib().gdla_gates_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=ref.device)
+    a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel()
+    _abi.check(_lib().gdla_gates(ctypes.byref(a), _stream(stream)), "gdla_gates")
+    return (gate_out if c_q is not None else None), (lam_out if x is not None else None)
 
 
 # ---------------------------------------------------------------------- decode

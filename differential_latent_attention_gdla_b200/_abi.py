@@ -56,10 +56,18 @@ class DecodeArgs(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t)]
 
 
+class GatesArgs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "L", "d_q", "d_x", "n_signal", "d_v")] + [
+        ("dtype", ctypes.c_int), ("rms_eps", ctypes.c_float),
+        ("c_q", _vp), ("gamma_q", _vp), ("w_g", _vp), ("x", _vp), ("w_lambda", _vp), ("gate_logits", _vp),
+        ("lam_logits", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 # Every symbol include/gdla.h declares.
 EXPORTED = ("gdla_latent_expand", "gdla_prefill_workspace_size", "gdla_prefill", "gdla_prefill_host_workspace_size",
             "gdla_prefill_host", "gdla_attend", "gdla_decode_workspace_size", "gdla_decode", "gdla_decode_noalloc",
-            "gdla_status_string", "gdla_workspace_status", "gdla_build_info", "gdla_diag_wait_timeout")
+            "gdla_gates_workspace_size", "gdla_gates", "gdla_status_string", "gdla_workspace_status",
+            "gdla_build_info", "gdla_diag_wait_timeout")
 
 _lock = threading.Lock()
 _lib = None
@@ -94,6 +102,10 @@ def load(path: str = LIB_PATH):
         lib.gdla_decode.restype = ctypes.c_int
         lib.gdla_decode_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         lib.gdla_decode_noalloc.restype = ctypes.c_int
+        lib.gdla_gates_workspace_size.argtypes = [ctypes.POINTER(GatesArgs)]
+        lib.gdla_gates_workspace_size.restype = ctypes.c_size_t
+        lib.gdla_gates.argtypes = [ctypes.POINTER(GatesArgs), _vp]
+        lib.gdla_gates.restype = ctypes.c_int
         lib.gdla_status_string.argtypes = [ctypes.c_int]
         lib.gdla_status_string.restype = ctypes.c_char_p
         lib.gdla_workspace_status.argtypes = [_vp, _vp]

@@ -4,7 +4,9 @@
 //   * norm_rope_kernel: per-token RMSNorm of c_KV (fp32 statistics) and RoPE of
 //     the shared rotary key k_R, one warp per token;
 //   * gemm_simt_kernel: the expansion c_hat @ W_UKV with CUDA-core FMAs, used for
-//     fp32 tensors and for shapes the tensor-core GEMM does not take.
+//     fp32 tensors and for shapes the tensor-core GEMM does not take; also the
+//     lambda projection x @ W_lambda (fp32 output) and, for such shapes, the gate
+//     projection.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -52,14 +54,15 @@ cudaError_t launch_norm_rope(const NormRopeParams& p, gdla_dtype dt, cudaStream_
 
 // ---------------------------------------------------------------- SIMT GEMM
 // 128x128 output tile per block, 8x8 per thread, k-step 8, fp32 accumulation.
-template <typename T>
+// T is the input type; TO the output type (T, or fp32 for the lambda logits).
+template <typename T, typename TO>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
   constexpr int BM = 128, BN = 128, BK = 8;
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][BN + 4];
   const T* A = reinterpret_cast<const T*>(p.A);
   const T* Bm = reinterpret_cast<const T*>(p.Bm);
-  T* C = reinterpret_cast<T*>(p.C);
+  TO* C = reinterpret_cast<TO*>(p.C);
   const long m0 = (long)blockIdx.y * BM;
   const int n0 = blockIdx.x * BN;
   const int tid = threadIdx.x;
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int gn = n0 + tx * 8 + j;
-      if (gn < p.N) C[gm * p.N + gn] = from_f<T>(acc[i][j]);
+      if (gn < p.N) C[gm * p.N + gn] = from_f<TO>(acc[i][j]);
     }
   }
 }
@@ -113,9 +116,18 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
 cudaError_t launch_gemm_simt(const GemmParams& p, gdla_dtype dt, cudaStream_t s) {
   dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + 127) / 128));
   if (dt == GDLA_BF16)
-    gemm_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+    gemm_simt_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>(p);
   else
-    gemm_simt_kernel<float><<<grid, 256, 0, s>>>(p);
+    gemm_simt_kernel<float, float><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_simt_f32out(const GemmParams& p, gdla_dtype dt, cudaStream_t s) {
+  dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)((p.M + 127) / 128));
+  if (dt == GDLA_BF16)
+    gemm_simt_kernel<__nv_bfloat16, float><<<grid, 256, 0, s>>>(p);
+  else
+    gemm_simt_kernel<float, float><<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

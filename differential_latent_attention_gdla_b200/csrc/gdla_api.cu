@@ -534,6 +534,53 @@ gdla_status gdla_decode(const gdla_decode_args* a, void* stream) {
   return cuda_status(e);
 }
 
+size_t gdla_gates_workspace_size(const gdla_gates_args* a) {
+  if (!a || a->B < 1 || a->L < 1) return 0;
+  size_t n = kStatusBytes;
+  if (a->c_q && a->d_q > 0) n += align256((size_t)a->B * a->L * a->d_q * esize(a->dtype));
+  return n;
+}
+
+gdla_status gdla_gates(const gdla_gates_args* a, void* stream) {
+  if (!a || a->B < 1 || a->L < 1 || a->n_signal < 1) return GDLA_ERR_INVALID_ARG;
+  if (a->dtype != GDLA_BF16 && a->dtype != GDLA_FP32) return GDLA_ERR_INVALID_ARG;
+  if (!aligned16(a->workspace) || ((uintptr_t)a->workspace & 255) != 0) return GDLA_ERR_INVALID_ARG;
+  if (a->workspace_bytes < gdla_gates_workspace_size(a)) return GDLA_ERR_INVALID_ARG;
+  if (a->c_q) {
+    if (a->d_q < 1 || a->d_v < 1) return GDLA_ERR_INVALID_ARG;
+    const void* req[] = {a->c_q, a->gamma_q, a->w_g, a->gate_logits};
+    for (const void* p : req)
+      if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  }
+  if (a->x) {
+    if (a->d_x < 1) return GDLA_ERR_INVALID_ARG;
+    const void* req[] = {a->x, a->w_lambda, a->lam_logits};
+    for (const void* p : req)
+      if (!aligned16(p)) return GDLA_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  char* ws = (char*)a->workspace;
+  int* status = (int*)ws;
+  const long tokens = (long)a->B * a->L;
+  cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, s);
+  if (e == cudaSuccess && a->c_q) {
+    void* c_hat_q = ws + kStatusBytes;
+    // the latent RMSNorm kernel without a rotary part (d_rope = 0)
+    NormRopeParams np{tokens, a->L, a->d_q, 0, 0, a->rms_eps > 0.f ? a->rms_eps : 1e-6f, a->c_q, a->gamma_q,
+                      nullptr, nullptr, nullptr, c_hat_q, nullptr};
+    e = launch_norm_rope(np, a->dtype, s);
+    GemmParams gp{tokens, a->n_signal * a->d_v, a->d_q, c_hat_q, a->w_g, a->gate_logits};
+    if (e == cudaSuccess)
+      e = (a->dtype == GDLA_BF16 && gemm_tc_supported(gp)) ? launch_gemm_tc(gp, status, s)
+                                                           : launch_gemm_simt(gp, a->dtype, s);
+  }
+  if (e == cudaSuccess && a->x) {
+    GemmParams lp{tokens, a->n_signal, a->d_x, a->x, a->w_lambda, a->lam_logits};
+    e = launch_gemm_simt_f32out(lp, a->dtype, s);
+  }
+  return cuda_status(e);
+}
+
 gdla_status gdla_diag_wait_timeout(void* status_word, void* stream) {
   if (!status_word || ((uintptr_t)status_word & 255) != 0) return GDLA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;

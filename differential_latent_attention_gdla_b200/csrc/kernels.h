@@ -27,6 +27,8 @@ struct GemmParams {
   const void* A; const void* Bm; void* C;
 };
 cudaError_t launch_gemm_simt(const GemmParams& p, gdla_dtype dt, cudaStream_t s);
+// the same product with an fp32 C whatever the input type (lambda logits)
+cudaError_t launch_gemm_simt_f32out(const GemmParams& p, gdla_dtype dt, cudaStream_t s);
 // tcgen05/TMA version (bf16 only; M any, N % 256 == 0, K % 64 == 0).
 bool gemm_tc_supported(const GemmParams& p);
 cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s);

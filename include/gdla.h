@@ -274,6 +274,43 @@ gdla_status gdla_decode(const gdla_decode_args* args, void* stream);
 #define GDLA_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
 gdla_status gdla_decode_noalloc(const gdla_decode_args* args, void* stream);
 
+/* ---------------------------------------------------------------------- gates
+ * The per-token inputs of the differential epilogue, computed from the layer's
+ * activations ("Motif 3: Technical Report", section "Architecture": lambda_t =
+ * sigmoid(x_t W_lambda), and the output gate is computed from the normalised query
+ * latent). The sigmoids stay in the attention epilogue: this call produces the
+ * logits that gdla_prefill, gdla_prefill_host, gdla_attend and gdla_decode take.
+ *   c_hat_q[t]     = gamma_q (.) c_q[t] / sqrt(mean(c_q[t]^2) + rms_eps)
+ *   gate_logits[t] = c_hat_q[t] @ W_G       ([n_signal * d_v], in `dtype`)
+ *   lam_logits[t]  = x[t] @ W_lambda        ([n_signal], fp32)
+ * for the B*L tokens (a decode step: L = 1). Either half may be skipped:
+ *  - c_q == NULL skips the gate (gamma_q, w_g and gate_logits are then ignored);
+ *  - x == NULL skips lambda (w_lambda and lam_logits are then ignored).
+ * The normalisation is the latent RMSNorm of gdla_latent_expand with its own gain.
+ * The gate product runs on the tensor cores for bf16 with n_signal*d_v a multiple
+ * of 256 and d_q a multiple of 64 (the report's shapes: d_q = 1536, n_signal*d_v =
+ * 4096 or 6144), and on the CUDA cores otherwise; lambda always on the CUDA cores.
+ * The workspace (>= gdla_gates_workspace_size(args) bytes, 256-byte aligned) holds
+ * the status word and, when the gate is computed, c_hat_q [B*L, d_q]. */
+typedef struct {
+  int B, L;                  /* tokens = B * L */
+  int d_q, d_x, n_signal, d_v;
+  gdla_dtype dtype;          /* element type of c_q, gamma_q, w_g, x, w_lambda and gate_logits */
+  float rms_eps;             /* <= 0 selects 1e-6 */
+  const void* c_q;           /* [B, L, d_q] query latent before normalisation, or NULL */
+  const void* gamma_q;       /* [d_q] its RMSNorm gain */
+  const void* w_g;           /* [d_q, n_signal * d_v] */
+  const void* x;             /* [B, L, d_x] layer input, or NULL */
+  const void* w_lambda;      /* [d_x, n_signal] */
+  void* gate_logits;         /* [B, L, n_signal, d_v] (out) */
+  float* lam_logits;         /* [B, L, n_signal] fp32 (out) */
+  void* workspace;
+  size_t workspace_bytes;
+} gdla_gates_args;
+
+size_t gdla_gates_workspace_size(const gdla_gates_args* args);
+gdla_status gdla_gates(const gdla_gates_args* args, void* stream);
+
 /* ---------------------------------------------------------------- utilities */
 const char* gdla_status_string(gdla_status s);
 

@@ -59,7 +59,7 @@ def _c_layout(struct: str, fields):
 
 @pytest.mark.parametrize("cls,cname", [(_abi.ExpandArgs, "gdla_expand_args"), (_abi.PrefillArgs, "gdla_prefill_args"),
                                        (_abi.AttendArgs, "gdla_attend_args"),
-                                       (_abi.DecodeArgs, "gdla_decode_args")])
+                                       (_abi.DecodeArgs, "gdla_decode_args"), (_abi.GatesArgs, "gdla_gates_args")])
 def test_ctypes_mirror_matches_c_layout(cls, cname):
     fields = [f[0] for f in cls._fields_]
     got = [ctypes.sizeof(cls)] + [getattr(cls, f).offset for f in fields]
@@ -202,3 +202,44 @@ def test_prefill_host_workspace_size(lib):
     assert lib.gdla_prefill_host_workspace_size(ctypes.byref(a), 0) == s_full
     assert s_full > s64
     assert lib.gdla_prefill_host_workspace_size(None, 64) == 0
+
+
+def good_gates():
+    a = _abi.GatesArgs(2, 100, 1536, 2048, 48, 128, _abi.GDLA_BF16, 0.0)
+    base = 0x10000000
+    for i, f in enumerate(("c_q", "gamma_q", "w_g", "x", "w_lambda", "gate_logits", "lam_logits", "workspace")):
+        setattr(a, f, base + i * 0x1000000)
+    a.workspace_bytes = lib_gates_ws(a)
+    return a
+
+
+def lib_gates_ws(a):
+    return _abi.load().gdla_gates_workspace_size(ctypes.byref(a))
+
+
+def test_gates_workspace_size(lib):
+    a = good_gates()
+    assert lib.gdla_gates_workspace_size(ctypes.byref(a)) == 256 + 2 * 100 * 1536 * 2  # status + c_hat_q
+    a.c_q = None  # lambda only: the status word alone
+    assert lib.gdla_gates_workspace_size(ctypes.byref(a)) == 256
+    assert lib.gdla_gates_workspace_size(None) == 0
+
+
+def test_gates_validation_rejects_before_launch(lib):
+    E = _abi.GDLA_ERR_INVALID_ARG
+
+    def st(mut):
+        a = good_gates()
+        mut(a)
+        return lib.gdla_gates(ctypes.byref(a), None)
+
+    assert st(lambda a: setattr(a, "B", 0)) == E
+    assert st(lambda a: setattr(a, "n_signal", 0)) == E
+    assert st(lambda a: setattr(a, "dtype", 3)) == E
+    assert st(lambda a: setattr(a, "w_g", 0)) == E                     # gate requested without W_G
+    assert st(lambda a: setattr(a, "gate_logits", 0x10000004)) == E    # misaligned output
+    assert st(lambda a: setattr(a, "w_lambda", 0)) == E                # lambda requested without W_lambda
+    assert st(lambda a: setattr(a, "d_x", 0)) == E
+    assert st(lambda a: setattr(a, "workspace", a.workspace + 16)) == E
+    assert st(lambda a: setattr(a, "workspace_bytes", a.workspace_bytes - 1)) == E
+    assert lib.gdla_gates(None, None) == E
