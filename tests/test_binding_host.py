@@ -51,3 +51,13 @@ def test_unsupported_dtype_is_rejected():
     with pytest.raises(ValueError, match="dtype"):
         gdla.prefill(inp["c_kv"].half(), inp["gamma"], inp["k_rope"], inp["q"], inp["w_ukv"], cos, cos,
                      inp["lam_logits"], inp["gate_logits"], g=SHAPE.g)
+
+
+def test_gates_binding_checks():
+    # neither half requested, and CPU tensors where the library reads device memory
+    with pytest.raises(ValueError, match="c_q"):
+        gdla.gates(n_signal=4)
+    c_q = torch.zeros((2, 8, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA device tensors"):
+        gdla.gates(c_q, torch.ones(64, dtype=torch.bfloat16), torch.zeros((64, 128), dtype=torch.bfloat16),
+                   n_signal=4, d_v=32)
