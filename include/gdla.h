@@ -18,6 +18,10 @@
  *    row-major in the layout stated beside them, 16-byte aligned. The library
  *    allocates no memory and keeps no per-call state; scratch comes from the
  *    caller's workspace, sized by the matching *_workspace_size function.
+ *    Two entry points state their exceptions beside them: gdla_prefill_host
+ *    takes its activations as host pointers and creates (and releases) its own
+ *    copy and compute streams, and gdla_decode_noalloc uses a fixed scratch
+ *    array inside the library instead of a workspace.
  *  - `stream` is a cudaStream_t passed as void*. All work is enqueued on it and
  *    the call returns without synchronising.
  *  - Argument errors (NULL pointer, misalignment, unsupported size, a too
