@@ -9,16 +9,25 @@ in HBM:
   * decode of B=64 sequences over a 32768-token latent cache, g=2, through
     gdla_decode.
 `value` is the prefill's algorithmic TFLOP/s (expansion GEMM plus QK and PV
-over the visible pairs, all ranks' work over the slowest rank's time);
-`decode` carries the decode's algorithmic GB/s (the cache read once). Inputs are
-larger than L2 (q alone is 805 MB), so no flush is needed between steps.
-`e2e` is the same prefill through gdla_prefill_host: the activations start in
-page-locked host memory and Y ends there, and the call overlaps the chunked
-copies with the kernels.
+over the visible pairs, all ranks' work over the slowest rank's time). Inputs
+are larger than L2 (q alone is 805 MB, the decode cache 2.4 GB), so no flush is
+needed between steps.
+
+Beside the timed steps (measured after them, outside their timed region):
+  * `decode`: the decode call timed in its own loop after its own warm-up (the
+    `roofline` of the decode), and its time inside the steps (`in_step_ms`),
+    where it follows the power-capped prefill;
+  * `prefill_cfg2` (B=4 L=4096 g=2 causal), `prefill_cfg4` (B=2 L=65536 g=2,
+    4096-token window) and the report's own layout, g=4 (80 heads):
+    `prefill_g4_swa128` (128-token window) and `decode_g4`;
+  * `e2e`: the same prefill through gdla_prefill_host (activations start in
+    page-locked host memory, Y ends there; the chunked copies overlap the
+    kernels), and `e2e.decode`: q, lambda and gate copied in from page-locked
+    host memory, gdla_decode, Y copied back, every step.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 With --impl reference the fp64 CPU oracle is timed on a bounded sample of the
-same prefill workload, on this host's cores.
+same prefill workload (the sample of the `cpu_baseline` leg), on this host's cores.
 """
 from __future__ import annotations
 
@@ -75,6 +84,8 @@ def parse():
     ap.add_argument("--e2e-chunk", type=int, default=0, help="tokens per host-copy chunk (0: library default)")
     ap.add_argument("--prefill", default=PREFILL_NAME, help="prefill workload name (profiling uses smaller ones)")
     ap.add_argument("--decode", default=DECODE_NAME, help="decode workload name")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the other configurations (profiling runs of one workload)")
     return ap.parse_args()
 
 
@@ -99,11 +110,51 @@ def rank_seed(seed: int, rank: int, which: str) -> int:
     return seed + rank + (1000 if which == "decode" else 0)
 
 
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 (NVIDIA's figure without 2:4 sparsity)
+NOMINAL_HBM_GBS = 8000.0      # the "~8 TB/s" HBM3e figure
+
+
 def peaks():
     try:
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "fallback": True}
+
+
+def tensor_roofline(tflops: float, pk: dict) -> dict:
+    """A tensor-bound kernel timed alone (milliseconds, not a seconds-long loop):
+    the fraction of the measured burst bf16 peak; the sustained and nominal
+    fractions beside it."""
+    return {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tflops / pk["bf16_tflops"],
+            "peak_kind": "measured burst bf16" + (" (fallback)" if pk.get("fallback") else ""),
+            "frac_of_sustained": tflops / pk["bf16_tflops_sustained"],
+            "frac_of_nominal": tflops / NOMINAL_BF16_TFLOPS}
+
+
+def hbm_roofline(gbs: float, pk: dict) -> dict:
+    return {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+            "peak_kind": "measured copy" + (" (fallback)" if pk.get("fallback") else ""),
+            "frac_of_nominal": gbs / NOMINAL_HBM_GBS}
+
+
+# The cpu_baseline leg and the reference arm time the oracle on the same sample.
+ORACLE_ROWS = 24
+
+
+def oracle_kv_groups(shape):
+    return list(range(shape.n_kv))
+
+
+def bench_config(prefill_key: str, decode_key: str, world: int) -> dict:
+    """The workload description both arms print (workload keys of workloads.py)."""
+    from differential_latent_attention_gdla_b200 import workloads as wl
+
+    P, D = wl.PREFILL[prefill_key], wl.DECODE[decode_key]
+    return {"workload": f"prefill {P.name} (value, TFLOP/s) + decode {D.name} (decode.value, GB/s)",
+            "prefill": prefill_key, "decode": decode_key,
+            "l2": "inputs larger than L2 (q 805 MB, cache 2.4 GB); no flush",
+            "parallelism": f"{world} independent replicas (weak scaling)"}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -137,7 +188,8 @@ def oracle_sample(shape, inp_cpu, n_rows: int, kv_groups):
 
 
 def run_reference(a):
-    """The fp64 oracle on host cores, one bounded sample per step."""
+    """The fp64 oracle on host cores, one bounded sample per step: the sample of
+    the cpu_baseline leg (ORACLE_ROWS rows of every KV group)."""
     import torch
 
     from differential_latent_attention_gdla_b200 import workloads as wl
@@ -149,7 +201,7 @@ def run_reference(a):
     inp = wl.make_prefill_inputs(shape, seed=a.seed, device="cpu")
     times, flops, desc, thr = [], 0.0, "", 1
     for k in range(a.warmup + a.steps):
-        dt, fl, desc, thr = oracle_sample(shape, inp, n_rows=8, kv_groups=[(4 * k + u) % shape.n_kv for u in range(4)])
+        dt, fl, desc, thr = oracle_sample(shape, inp, n_rows=ORACLE_ROWS, kv_groups=oracle_kv_groups(shape))
         if k >= a.warmup:
             times.append(dt)
             flops = fl
@@ -157,8 +209,8 @@ def run_reference(a):
     value = flops / mean / 1e12
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"prefill {PREFILL_NAME}: bounded oracle sample per step", "sample": desc},
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) recipe)",
+            "config": bench_config(PREFILL_NAME, DECODE_NAME, 1),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     del torch
@@ -210,6 +262,23 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------- our path
+def time_loop(fn, steps: int, warmup: int, stream):
+    """Mean milliseconds of fn() over `steps` calls after `warmup` untimed ones
+    (CUDA events on `stream`, synchronised on both sides)."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def run_ours(a):
     import torch
     import torch.distributed as dist
@@ -233,31 +302,48 @@ def run_ours(a):
 
     P = wl.PREFILL[a.prefill]
     D = wl.DECODE[a.decode]
-    # every rank runs its own independent problem (weak scaling, no collective on the data path)
-    pin = wl.make_prefill_inputs(P, seed=rank_seed(a.seed, rank, "prefill"), device=dev)
-    din = wl.make_decode_inputs(D, seed=rank_seed(a.seed, rank, "decode"), device=dev)
-    cos, sin = gdla.rope_tables(max(P.L, D.T), P.d_R, device=dev)
-    kv = torch.empty((P.B, P.L, P.n_kv, P.d_n + P.d_v), dtype=torch.bfloat16, device=dev)
-    krot = torch.empty((P.B, P.L, P.d_R), dtype=torch.bfloat16, device=dev)
-    chat = torch.empty((P.B, P.L, P.d_c), dtype=torch.bfloat16, device=dev)
-    y = torch.empty((P.B, P.L, P.n_S, P.d_v), dtype=torch.bfloat16, device=dev)
-    status = torch.zeros(256, dtype=torch.uint8, device=dev)
-    yd = torch.empty((D.B, D.n_S, D.d_v), dtype=torch.bfloat16, device=dev)
-    dws = torch.empty(gdla.decode_workspace_size(B=D.B, T_max=D.T, d_c=D.d_c, d_rope=D.d_R, n_kv=D.n_kv,
-                                                 d_nope=D.d_n, d_v=D.d_v, g=D.g), dtype=torch.uint8, device=dev)
+    pk = peaks()
     stream = torch.cuda.current_stream()
 
-    def expand():
-        gdla.latent_expand(pin["c_kv"], pin["gamma"], pin["k_rope"], pin["w_ukv"], cos, sin, n_kv=P.n_kv,
-                           d_nope=P.d_n, d_v=P.d_v, kv_out=kv, k_rope_out=krot, c_hat_out=chat, stream=stream)
+    def prefill_case(shape, seed):
+        """Inputs and the two calls (expansion, attention) of one prefill workload."""
+        inp = wl.make_prefill_inputs(shape, seed=seed, device=dev)
+        cos, sin = gdla.rope_tables(shape.L, shape.d_R, device=dev)
+        kv = torch.empty((shape.B, shape.L, shape.n_kv, shape.d_n + shape.d_v), dtype=torch.bfloat16, device=dev)
+        krot = torch.empty((shape.B, shape.L, shape.d_R), dtype=torch.bfloat16, device=dev)
+        chat = torch.empty((shape.B, shape.L, shape.d_c), dtype=torch.bfloat16, device=dev)
+        y = torch.empty((shape.B, shape.L, shape.n_S, shape.d_v), dtype=torch.bfloat16, device=dev)
+        status = torch.zeros(256, dtype=torch.uint8, device=dev)
 
-    def attend():
-        gdla.attend(pin["q"], kv, krot, cos, sin, pin["lam_logits"], pin["gate_logits"], g=P.g, mask=P.mask,
-                    window=P.window, out=y, status=status, stream=stream)
+        def expand():
+            gdla.latent_expand(inp["c_kv"], inp["gamma"], inp["k_rope"], inp["w_ukv"], cos, sin, n_kv=shape.n_kv,
+                               d_nope=shape.d_n, d_v=shape.d_v, kv_out=kv, k_rope_out=krot, c_hat_out=chat,
+                               stream=stream)
 
-    def decode():
-        gdla.decode(din["c_cache"], din["kr_cache"], din["q"], din["w_ukv"], cos, sin, din["lam_logits"],
-                    din["gate_logits"], din["seqlens"], g=D.g, out=yd, workspace=dws, stream=stream)
+        def attend():
+            gdla.attend(inp["q"], kv, krot, cos, sin, inp["lam_logits"], inp["gate_logits"], g=shape.g,
+                        mask=shape.mask, window=shape.window, out=y, status=status, stream=stream)
+
+        return inp, (cos, sin), expand, attend, status
+
+    def decode_case(shape, seed):
+        din = wl.make_decode_inputs(shape, seed=seed, device=dev)
+        cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=dev)
+        yd = torch.empty((shape.B, shape.n_S, shape.d_v), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(gdla.decode_workspace_size(B=shape.B, T_max=shape.T, d_c=shape.d_c, d_rope=shape.d_R,
+                                                    n_kv=shape.n_kv, d_nope=shape.d_n, d_v=shape.d_v, g=shape.g),
+                         dtype=torch.uint8, device=dev)
+
+        def decode():
+            gdla.decode(din["c_cache"], din["kr_cache"], din["q"], din["w_ukv"], cos, sin, din["lam_logits"],
+                        din["gate_logits"], din["seqlens"], g=shape.g, mask=shape.mask, window=shape.window,
+                        out=yd, workspace=ws, stream=stream)
+
+        return din, (cos, sin), yd, ws, decode
+
+    # every rank runs its own independent problem (weak scaling, no collective on the data path)
+    pin, pcs, expand, attend, status = prefill_case(P, rank_seed(a.seed, rank, "prefill"))
+    din, dcs, yd, dws, decode = decode_case(D, rank_seed(a.seed, rank, "decode"))
 
     launches_per_step = 2 + 1 + 3  # norm+rope, expansion GEMM | attention | absorb, split-KV, combine
     for _ in range(a.warmup):
@@ -290,82 +376,140 @@ def run_ours(a):
     t_att = sum(e[1].elapsed_time(e[2]) for e in ev) / a.steps
     t_dec = sum(e[2].elapsed_time(e[3]) for e in ev) / a.steps
     t_step = ev[0][0].elapsed_time(ev[-1][3]) / a.steps
-    t_exp, t_att, t_dec, t_step = max_over_ranks([t_exp, t_att, t_dec, t_step], world, dev)
 
-    pf = P.algorithmic_flops()
-    f_exp = 2.0 * P.B * P.L * P.d_c * P.n_kv * (P.d_n + P.d_v)
-    f_att = pf - f_exp
-    db = D.algorithmic_bytes()
-    pk = peaks()
-    value = weak_scaling_value(pf, world, (t_exp + t_att) * 1e-3) / 1e12
-    att_tflops = f_att / (t_att * 1e-3) / 1e12
-    dec_gbs = weak_scaling_value(db, world, t_dec * 1e-3) / 1e9
+    # ---- measured after the timed steps, outside their region
+    # the decode call alone, in its own loop after its own warm-up
+    t_dec_alone = time_loop(decode, a.steps, a.warmup, stream)
+    if int(gdla.workspace_status(dws)) != 0:
+        raise RuntimeError("device status word reports a failed wait (decode)")
 
-    # end to end through the public host-buffer call (gdla_prefill_host): the activations
-    # start in page-locked host memory and Y ends there; every copy is inside the timed region
-    e2e = None
+    # end to end through host buffers: the prefill through gdla_prefill_host, and the
+    # decode with its per-token inputs copied in and Y copied back every step
+    e2e, t_e2e, t_e2e_dec, e2e_extra = None, 0.0, 0.0, {}
     if a.e2e_steps > 0:
         keys = ["c_kv", "k_rope", "q", "lam_logits", "gate_logits"]
         host = {k: pin[k].cpu().pin_memory() for k in keys}
-        yh = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        yh = torch.empty((P.B, P.L, P.n_S, P.d_v), dtype=torch.bfloat16, pin_memory=True)
         ws = torch.empty(gdla.prefill_host_workspace_size(B=P.B, L=P.L, d_c=P.d_c, d_rope=P.d_R, n_kv=P.n_kv,
                                                           d_nope=P.d_n, d_v=P.d_v, g=P.g,
                                                           chunk_tokens=a.e2e_chunk),
                          dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            gdla.prefill_host(host["c_kv"], pin["gamma"], host["k_rope"], host["q"], pin["w_ukv"], cos, sin,
+            gdla.prefill_host(host["c_kv"], pin["gamma"], host["k_rope"], host["q"], pin["w_ukv"], pcs[0], pcs[1],
                               host["lam_logits"], host["gate_logits"], g=P.g, mask=P.mask, window=P.window,
                               chunk_tokens=a.e2e_chunk, out=yh, workspace=ws, stream=stream)
 
-        e2e_step()
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(a.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        (t,) = max_over_ranks([e0.elapsed_time(e1) / a.e2e_steps], world, dev)
-        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
-        e2e = {"value": weak_scaling_value(pf, world, t * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": yh.numel() * yh.element_size(), "ms_per_step": t}
+        t_e2e = time_loop(e2e_step, a.e2e_steps, 1, stream)
         if int(gdla.workspace_status(ws)) != 0:
             raise RuntimeError("device status word reports a failed wait (host-buffer prefill)")
-        e2e["chunk_tokens"] = a.e2e_chunk if a.e2e_chunk > 0 else "library default"
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        e2e_extra["prefill"] = {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": yh.numel() * yh.element_size(),
+                                "chunk_tokens": a.e2e_chunk if a.e2e_chunk > 0 else "library default"}
         del ws, host
+
+        dkeys = ["q", "lam_logits", "gate_logits"]
+        dhost = {k: din[k].cpu().pin_memory() for k in dkeys}
+        ddev = {k: torch.empty_like(din[k]) for k in dkeys}
+        ydh = torch.empty(yd.shape, dtype=yd.dtype, pin_memory=True)
+
+        def e2e_decode():
+            for k in dkeys:
+                ddev[k].copy_(dhost[k], non_blocking=True)
+            gdla.decode(din["c_cache"], din["kr_cache"], ddev["q"], din["w_ukv"], dcs[0], dcs[1],
+                        ddev["lam_logits"], ddev["gate_logits"], din["seqlens"], g=D.g, out=yd, workspace=dws,
+                        stream=stream)
+            ydh.copy_(yd, non_blocking=True)
+
+        t_e2e_dec = time_loop(e2e_decode, a.steps, a.warmup, stream)
+        e2e_extra["decode"] = {"h2d_bytes_per_step": sum(dhost[k].numel() * dhost[k].element_size() for k in dkeys),
+                               "d2h_bytes_per_step": ydh.numel() * ydh.element_size()}
+
+    # the other prefill configurations and the report's own head layout (g = 4)
+    extra_ms = {}
+    if a.extras:
+        for key, name in (("prefill_cfg2", "b4_l4k_g2"), ("prefill_cfg4", "b2_l64k_swa4k"),
+                          ("prefill_g4_swa128", "b1_l32k_g4_swa128")):
+            S = wl.PREFILL[name]
+            _, _, ex, at, st = prefill_case(S, rank_seed(a.seed, rank, "prefill"))
+            t_e = time_loop(ex, 3, 2, stream)
+            t_a = time_loop(at, 3, 2, stream)
+            if int(gdla.workspace_status(st)) != 0:
+                raise RuntimeError(f"device status word reports a failed wait ({name})")
+            extra_ms[key] = (name, S, t_e, t_a)
+            torch.cuda.empty_cache()
+        S = wl.DECODE["b64_t32k_g4"]
+        _, _, _, ws4, dec4 = decode_case(S, rank_seed(a.seed, rank, "decode"))
+        t4 = time_loop(dec4, 10, 3, stream)
+        if int(gdla.workspace_status(ws4)) != 0:
+            raise RuntimeError("device status word reports a failed wait (decode g=4)")
+        extra_ms["decode_g4"] = ("b64_t32k_g4", S, t4, None)
+
+    vals = [t_exp, t_att, t_dec, t_step, t_dec_alone, t_e2e, t_e2e_dec]
+    for key in sorted(extra_ms):
+        vals += [extra_ms[key][2], extra_ms[key][3] or 0.0]
+    vals = max_over_ranks(vals, world, dev)
+    t_exp, t_att, t_dec, t_step, t_dec_alone, t_e2e, t_e2e_dec = vals[:7]
+
+    pf = P.algorithmic_flops()
+    f_exp = 2.0 * P.B * P.L * P.d_c * P.n_kv * (P.d_n + P.d_v)
+    f_att = pf - f_exp
+    db = D.algorithmic_bytes()
+    value = weak_scaling_value(pf, world, (t_exp + t_att) * 1e-3) / 1e12
+    att_tflops = f_att / (t_att * 1e-3) / 1e12
+    dec_gbs = weak_scaling_value(db, world, t_dec_alone * 1e-3) / 1e9
+
+    if a.e2e_steps > 0:
+        e2e = {"value": weak_scaling_value(pf, world, t_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               **e2e_extra["prefill"], "ms_per_step": t_e2e,
+               "decode": {"value": weak_scaling_value(db, world, t_e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
+                          "ms_per_step": t_e2e_dec, **e2e_extra["decode"]}}
+
+    extras = {}
+    i = 7
+    for key in sorted(extra_ms):
+        name, S, t_first, t_second = extra_ms[key]
+        te, ta = vals[i], vals[i + 1]
+        i += 2
+        if t_second is None:  # a decode workload
+            gbs = weak_scaling_value(S.algorithmic_bytes(), world, te * 1e-3) / 1e9
+            extras[key] = {"workload": S.name, "value": gbs, "unit": "GB/s", "ms": te,
+                           "roofline": hbm_roofline(gbs / world, pk)}
+        else:
+            fl = S.algorithmic_flops()
+            fe = 2.0 * S.B * S.L * S.d_c * S.n_kv * (S.d_n + S.d_v)
+            tf = weak_scaling_value(fl, world, (te + ta) * 1e-3) / 1e12
+            extras[key] = {"workload": S.name, "value": tf, "unit": "TFLOP/s", "ms": te + ta, "expand_ms": te,
+                           "attend_ms": ta, "algorithmic_tflop": fl / 1e12,
+                           "roofline": dict(tensor_roofline((fl - fe) / (ta * 1e-3) / 1e12, pk),
+                                            kernel="gdla_attend")}
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         inp_cpu = {k: v.cpu() for k, v in pin.items()}
-        dt, fl, desc, thr = oracle_sample(P, inp_cpu, n_rows=24, kv_groups=list(range(P.n_kv)))
+        dt, fl, desc, thr = oracle_sample(P, inp_cpu, n_rows=ORACLE_ROWS, kv_groups=oracle_kv_groups(P))
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": desc,
                "seconds": dt}
 
     if rank == 0:
+        roof = tensor_roofline(att_tflops, pk)
+        roof.update({"traffic": measured_traffic("attn_tc_kernel", a.prefill),
+                     "kernel": "gdla_attend (attention + differential epilogue)"})
+        droof = hbm_roofline(dec_gbs / world, pk)
+        droof.update({"kernel": "whole gdla_decode call (absorb, split-KV, combine)",
+                      "traffic": measured_traffic("decode_tc_kernel", a.decode),
+                      "traffic_kernel": "decode_tc_kernel (split-KV pass)"})
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": t_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) recipe)",
-            "config": {"workload": f"prefill {P.name} (value, TFLOP/s) + decode {D.name} "
-                                   f"(decode.value, GB/s)", "prefill": a.prefill, "decode": a.decode,
-                       "l2": "inputs larger than L2 (q 805 MB, cache 2.4 GB); no flush",
-                       "parallelism": f"{world} independent replicas (weak scaling)"},
+            "config": bench_config(a.prefill, a.decode, world),
             "prefill": {"ms": t_exp + t_att, "expand_ms": t_exp, "attend_ms": t_att,
                         "algorithmic_tflop": pf / 1e12},
-            "decode": {"value": dec_gbs, "unit": "GB/s", "ms": t_dec, "algorithmic_gb": db / 1e9,
-                       "roofline": {"bound": "hbm", "achieved": dec_gbs / world, "peak": pk["hbm_gbs"],
-                                    "unit": "GB/s", "frac": dec_gbs / world / pk["hbm_gbs"],
-                                    "peak_kind": "measured copy", "kernel": "whole gdla_decode call",
-                                    "traffic": measured_traffic("decode_tc_kernel", a.decode),
-                                    "traffic_kernel": "decode_tc_kernel (split-KV pass)"}},
-            "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": pk["bf16_tflops_sustained"],
-                         "unit": "TFLOP/s", "frac": att_tflops / pk["bf16_tflops_sustained"],
-                         "traffic": measured_traffic("attn_tc_kernel", a.prefill),
-                         "kernel": "gdla_attend (attention + differential epilogue)",
-                         "peak_kind": "measured sustained bf16 (burst %.1f: frac %.3f)" % (
-                             pk["bf16_tflops"], att_tflops / pk["bf16_tflops"])},
+            "decode": {"value": dec_gbs, "unit": "GB/s", "ms": t_dec_alone, "algorithmic_gb": db / 1e9,
+                       "timing": "own loop after its own warm-up", "in_step_ms": t_dec,
+                       "in_step_value": weak_scaling_value(db, world, t_dec * 1e-3) / 1e9, "roofline": droof},
+            "roofline": roof, **extras,
             "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches_per_step * a.steps, "clocks": clk,
             "wall_s": wall,
         }

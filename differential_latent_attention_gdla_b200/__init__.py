@@ -71,42 +71,41 @@ def _mask(mask: str) -> int:
     return GDLA_MASK_CAUSAL if mask == "causal" else GDLA_MASK_SLIDING
 
 
+def _tables(fill, max_pos: int, d_rope: int, device):
+    cos = torch.empty((max_pos, d_rope // 2), dtype=torch.float32)
+    sin = torch.empty_like(cos)
+    fp = ctypes.POINTER(ctypes.c_float)
+    _abi.check(fill(ctypes.cast(cos.data_ptr(), fp), ctypes.cast(sin.data_ptr(), fp)), "RoPE tables")
+    return cos.to(device), sin.to(device)
+
+
 def rope_tables(max_pos: int, d_rope: int, base: float = 10000.0, device="cuda"):
     """cos/sin tables [max_pos, d_rope/2] (fp32) of the rotate-half RoPE with
-    frequencies theta_k = base^(-2k/d_rope). Model set-up, computed once in
-    double precision like any other constant input (e.g. a YaRN variant only
-    changes these tables)."""
-    k = torch.arange(d_rope // 2, dtype=torch.float64)
-    theta = base ** (-2.0 * k / d_rope)
-    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * theta[None, :]
-    return ang.cos().float().to(device), ang.sin().float().to(device)
+    frequencies theta_k = base^(-2k/d_rope), built by the library
+    (gdla_rope_tables) on the host and moved to ``device``. Model set-up,
+    computed once like any other constant input (a YaRN variant only changes
+    these tables)."""
+    return _tables(lambda c, s: _lib().gdla_rope_tables(int(max_pos), int(d_rope), float(base), c, s), max_pos,
+                   d_rope, device)
 
 
 def yarn_rope_tables(max_pos: int, d_rope: int, factor: float, original_max_pos: int, base: float = 10000.0,
                      beta_fast: float = 32.0, beta_slow: float = 1.0, device="cuda"):
     """cos/sin tables [max_pos, d_rope/2] (fp32) of RoPE with YaRN frequency scaling
-    ("Context Extension via YaRN", page 1, section 2), for extending a model trained
-    on ``original_max_pos`` tokens by ``factor``: a frequency whose wavelength
-    2 pi / theta is below original_max_pos / beta_fast is kept, one above
-    original_max_pos / beta_slow is divided by ``factor``, and in between the
-    divisor moves linearly with the wavelength. Model set-up, like ``rope_tables``;
-    pair the tables with ``softmax_scale = yarn_mscale(factor)**2 / sqrt(d_qk)``."""
-    theta = base ** (-2.0 * torch.arange(d_rope // 2, dtype=torch.float64) / d_rope)
-    wavelength = 2.0 * math.pi / theta
-    short, long_ = original_max_pos / beta_fast, original_max_pos / beta_slow
-    if long_ > short:
-        ramp = ((wavelength - short) / (long_ - short)).clamp(0.0, 1.0)
-    else:
-        ramp = (wavelength > short).to(torch.float64)
-    theta = theta * ((1.0 - ramp) + ramp / factor)
-    ang = torch.arange(max_pos, dtype=torch.float64)[:, None] * theta[None, :]
-    return ang.cos().float().to(device), ang.sin().float().to(device)
+    ("Open-Source Frontier Models: Architecture and Benchmarks of Rnj-1 and
+    Motif-2", section 2, the Scale(i) equation), built by the library
+    (gdla_yarn_rope_tables). Pair them with
+    ``softmax_scale = yarn_mscale(factor)**2 / sqrt(d_qk)``."""
+    return _tables(lambda c, s: _lib().gdla_yarn_rope_tables(int(max_pos), int(d_rope), float(base), float(factor),
+                                                             int(original_max_pos), float(beta_fast),
+                                                             float(beta_slow), c, s), max_pos, d_rope, device)
 
 
 def yarn_mscale(factor: float) -> float:
-    """YaRN's attention temperature m = 1 + 0.1 ln(factor) (1 for factor <= 1); the
-    logits are multiplied by m^2, which the caller folds into softmax_scale."""
-    return 1.0 + 0.1 * math.log(factor) if factor > 1.0 else 1.0
+    """YaRN's attention temperature m = 1 + 0.1 ln(factor) (1 for factor <= 1),
+    from the library (gdla_yarn_mscale); the logits are multiplied by m^2, which
+    the caller folds into softmax_scale."""
+    return float(_lib().gdla_yarn_mscale(float(factor)))
 
 
 # ------------------------------------------------------------------- expansion

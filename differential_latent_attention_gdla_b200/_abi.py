@@ -67,7 +67,8 @@ class GatesArgs(ctypes.Structure):
 EXPORTED = ("gdla_latent_expand", "gdla_prefill_workspace_size", "gdla_prefill", "gdla_prefill_host_workspace_size",
             "gdla_prefill_host", "gdla_attend", "gdla_decode_workspace_size", "gdla_decode", "gdla_decode_noalloc",
             "gdla_gates_workspace_size", "gdla_gates", "gdla_status_string", "gdla_workspace_status",
-            "gdla_build_info", "gdla_diag_wait_timeout")
+            "gdla_build_info", "gdla_diag_wait_timeout", "gdla_rope_tables", "gdla_yarn_rope_tables",
+            "gdla_yarn_mscale")
 
 _lock = threading.Lock()
 _lib = None
@@ -114,6 +115,13 @@ def load(path: str = LIB_PATH):
         lib.gdla_workspace_status.restype = ctypes.c_int
         lib.gdla_build_info.argtypes = []
         lib.gdla_build_info.restype = ctypes.c_char_p
+        lib.gdla_rope_tables.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double, _fp, _fp]
+        lib.gdla_rope_tables.restype = ctypes.c_int
+        lib.gdla_yarn_rope_tables.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                              ctypes.c_int, ctypes.c_double, ctypes.c_double, _fp, _fp]
+        lib.gdla_yarn_rope_tables.restype = ctypes.c_int
+        lib.gdla_yarn_mscale.argtypes = [ctypes.c_double]
+        lib.gdla_yarn_mscale.restype = ctypes.c_double
         _lib = lib
         return lib
 

@@ -559,9 +559,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-bool attn_tc_supported(const AttnParams& p, gdla_dtype dt) {
-  return dt == GDLA_BF16 && p.d_nope == DN && p.d_rope == DR && p.d_v == DV && p.g >= 1 && p.g <= 8 &&
-         get_encode_tiled() != nullptr;
+bool attn_tc_shape(const AttnParams& p, gdla_dtype dt) {
+  return dt == GDLA_BF16 && p.d_nope == DN && p.d_rope == DR && p.d_v == DV && p.g >= 1 && p.g <= 8;
 }
 
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {

@@ -7,13 +7,16 @@
 //   q_nope . (c_hat W_UK) = (W_UK q_nope) . c_hat      (absorbed query)
 //   sum_j p_j (c_hat_j W_UV) = (sum_j p_j c_hat_j) W_UV (latent weighted sum)
 // Kernels: decode_absorb (q_abs = W_UK q_nope, RoPE of q_rope at position
-// seqlen-1), decode_split (split-KV online softmax over the cache, partial
-// results per split) and decode_combine (log-sum-exp merge of the splits, W_UV,
+// seqlen-1; for the tensor-core split kernel it writes the query operand in that
+// kernel's bf16 shared-memory image), decode_split (split-KV online softmax over
+// the cache, partial results per split; the tensor-core version is in
+// decode_tc.cu) and decode_combine (log-sum-exp merge of the partials, W_UV,
 // differential and gate epilogue).
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace gdla {
 
@@ -49,6 +52,9 @@ __host__ __device__ inline int combine_seqs(const DecodeParams& p) {
 // rows) x ABS_RPW (query rows) tile, so each shared load feeds several FMAs.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
+  // the split kernel may start its set-up and first cache loads; it reads the
+  // query images only after this grid has completed
+  sm100::grid_dep_launch();
   const int h = blockIdx.x, c0 = blockIdx.y * ABS_C;
   const int spb = absorb_seqs(p), b0 = blockIdx.z * spb;
   const int nb = min(spb, p.B - b0);
@@ -117,6 +123,8 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
       acc[i][3] = fmaf(wv.w, qv, acc[i][3]);
     }
   }
+  // tensor-core path: the query image is pre-scaled by tau*log2(e) and bf16
+  const float isc = p.scale * kLog2e;
   if (4 * lane < nrows) {
 #pragma unroll
     for (int i = 0; i < ABS_RPW; ++i) {
@@ -124,8 +132,17 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
       if (r >= R) break;
       const int bl = r / G1, u = r % G1;
       const int head = u < p.g ? h * p.g + u : n_S + h;
-      *reinterpret_cast<float4*>(p.q_abs + ((long)(b0 + bl) * H_q + head) * p.d_c + c0 + 4 * lane) =
-          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      const int b = b0 + bl, d = c0 + 4 * lane;
+      if (p.tc) {
+        const int hgi = head / p.hpc, lh = head - hgi * p.hpc;
+        uint8_t* img = p.qimg + ((long)b * p.n_hg + hgi) * kDtcImageBytes;
+        *reinterpret_cast<uint2*>(img + dtc_image_offset(lh, d)) =
+            make_uint2(sm100::pack_bf16x2(acc[i][0] * isc, acc[i][1] * isc),
+                       sm100::pack_bf16x2(acc[i][2] * isc, acc[i][3] * isc));
+      } else {
+        *reinterpret_cast<float4*>(p.q_abs + ((long)b * H_q + head) * p.d_c + d) =
+            make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      }
     }
   }
   // RoPE of the rotary query parts at position seqlen-1 (once per block row 0)
@@ -135,13 +152,36 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
     const int r = e / half, k = e % half, bl = r / G1, u = r % G1;
     const int b = b0 + bl;
     const int head = u < p.g ? h * p.g + u : n_S + h;
-    const int pos = p.seqlens[b] - 1;
+    // a sequence length outside [1, T_max] is clamped (the split kernel reports it)
+    const int pos = min(max(p.seqlens[b], 1), p.T_max) - 1;
     const T* qr = q + ((long)b * H_q + head) * dqk + p.d_nope;
     const float cs = p.cos_tab[(long)pos * half + k], sn = p.sin_tab[(long)pos * half + k];
     const float x1 = to_f(qr[k]), x2 = to_f(qr[k + half]);
-    float* o = p.q_rot + ((long)b * H_q + head) * p.d_rope;
-    o[k] = x1 * cs - x2 * sn;
-    o[k + half] = x2 * cs + x1 * sn;
+    const float y1 = x1 * cs - x2 * sn, y2 = x2 * cs + x1 * sn;
+    if (p.tc) {
+      const int hgi = head / p.hpc, lh = head - hgi * p.hpc;
+      uint8_t* img = p.qimg + ((long)b * p.n_hg + hgi) * kDtcImageBytes;
+      *reinterpret_cast<__nv_bfloat16*>(img + dtc_image_offset(lh, p.d_c + k)) = __float2bfloat16_rn(y1 * isc);
+      *reinterpret_cast<__nv_bfloat16*>(img + dtc_image_offset(lh, p.d_c + k + half)) =
+          __float2bfloat16_rn(y2 * isc);
+    } else {
+      float* o = p.q_rot + ((long)b * H_q + head) * p.d_rope;
+      o[k] = y1;
+      o[k + half] = y2;
+    }
+  }
+  // tensor-core path: image rows of padding heads (beyond each head group's heads) are zero
+  if (p.tc && h == 0) {
+    for (int bl = 0; bl < nb; ++bl)
+      for (int hgi = 0; hgi < p.n_hg; ++hgi) {
+        const int nh = min(p.hpc, H_q - hgi * p.hpc);
+        uint8_t* img = p.qimg + ((long)(b0 + bl) * p.n_hg + hgi) * kDtcImageBytes;
+        const int chunks = (kDtcHeads - nh) * 9 * 8;  // 16-byte chunks of the padding rows
+        for (int e = threadIdx.x; e < chunks; e += blockDim.x) {
+          const int lh = nh + e / 72, bx = (e % 72) / 8, c = e % 8;
+          *reinterpret_cast<uint4*>(img + bx * (kDtcHeads * 128) + lh * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
   }
 }
 
@@ -173,7 +213,9 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
     mrow[e] = -INFINITY;
     lrow[e] = 0.f;
   }
-  const int Tb = p.seqlens[b];
+  const int raw = p.seqlens[b];
+  if ((raw < 1 || raw > p.T_max) && s == 0 && tid == 0) atomicCAS(p.status, 0, (int)GDLA_ERR_INVALID_ARG);
+  const int Tb = min(max(raw, 1), p.T_max);  // out-of-range lengths are clamped (and reported)
   const int lo = p.sliding ? max(0, Tb - p.window) : 0;
   const int t0 = max(lo, s * p.split_len), t1 = min(Tb, (s + 1) * p.split_len);
 
@@ -240,7 +282,7 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
   }
   __syncthreads();
   // partial results of this split
-  const long base = ((long)b * p.n_splits + s) * H_q;
+  const long base = ((long)b * p.n_splits + s) * p.part_heads;
 #pragma unroll
   for (int a = 0; a < HPT; ++a) {
     const int hh = warp + 8 * a;
@@ -261,19 +303,24 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
 //   H = O_lat W_UV, D = H_S - sigmoid(lam) H_N, Y = sigmoid(G) D.
 // W_UV is staged CMB_KC latent rows at a time; every thread accumulates a 4 (query
 // rows) x 16-byte-vector (value columns) tile of H over one K-slice of each block.
+// `max_parts` bounds the partials of one sequence (the splits, or the ranges of one
+// head group on the tensor-core path).
 template <typename T>
-__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p, int max_parts) {
   const int spb = combine_seqs(p);
   const int h = blockIdx.x, b0 = blockIdx.y * spb;
   const int nb = min(spb, p.B - b0);
-  const int n_S = p.g * p.n_kv, H_q = n_S + p.n_kv, G1 = p.g + 1, R = nb * G1, NS = p.n_splits;
+  const int n_S = p.g * p.n_kv, G1 = p.g + 1, R = nb * G1, NP = max_parts;
   const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v);
   extern __shared__ float sm[];
   float* olat = sm;                              // [CMB_R][d_c]
   float* hsm = olat + CMB_R * d_c;               // [CMB_R][DV]
-  float* wgt = hsm + CMB_R * DV;                 // [CMB_R][NS] merge weights (scaled by 1 / denominator)
-  T* wch = reinterpret_cast<T*>(wgt + CMB_R * NS);  // 2 x [CMB_KC][DV] staged W_UV rows
+  float* wgt = hsm + CMB_R * DV;                 // [CMB_R][NP] merge weights (scaled by 1 / denominator)
+  T* wch = reinterpret_cast<T*>(wgt + CMB_R * NP);  // 2 x [CMB_KC][DV] staged W_UV rows
   float* red = reinterpret_cast<float*>(wch + 2 * CMB_KC * DV);  // [K-slices][CMB_R][DV] partial products
+  __shared__ long long rec0[CMB_R];              // first partial record of each row
+  __shared__ long long rec_step[CMB_R];          // record stride between consecutive partials of the row
+  __shared__ int n_parts[CMB_R];
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   const T* gate = reinterpret_cast<const T*>(p.gate);
   T* out = reinterpret_cast<T*>(p.out);
@@ -305,27 +352,48 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     }
   };
   load_w(0);
+  // the partials (and their index on the tensor-core path) come from the split kernel
+  sm100::grid_dep_wait();
 
+  // ---- where each row's partials are: record index of the first, stride, count
+  if (tid < R) {
+    const int r = tid, b = b0 + r / G1, head = head_of_row(r);
+    if (p.tc) {
+      const int hgi = head / p.hpc, lh = head - hgi * p.hpc;
+      // the first and last range covering sequence b (clamped, so that a call whose
+      // split kernel gave up early still reads inside the records)
+      const int2 info = p.seqinfo[b];
+      const int x = min(max(info.x, 0), p.n_ranges - 1), y = min(max(info.y, x), p.n_ranges - 1);
+      rec0[r] = ((long long)(x + b) * p.n_hg + hgi) * p.part_heads + lh;
+      rec_step[r] = (long long)p.n_hg * p.part_heads;
+      n_parts[r] = y - x + 1;
+    } else {
+      rec0[r] = (long long)b * p.n_splits * p.part_heads + head;
+      rec_step[r] = p.part_heads;
+      n_parts[r] = p.n_splits;
+    }
+  }
+  __syncthreads();
   // ---- merge weights: one warp per query row
   for (int r = warp; r < R; r += 8) {
-    const int b = b0 + r / G1, head = head_of_row(r);
-    const float* ml = p.part_ml + ((long)b * NS * H_q + head) * 2;
+    const int np = n_parts[r];
+    const long long r0 = rec0[r], rs = rec_step[r];
     float M = -INFINITY;
-    for (int sp = lane; sp < NS; sp += 32) M = fmaxf(M, ml[(long)sp * H_q * 2]);
+    for (int sp = lane; sp < np; sp += 32) M = fmaxf(M, p.part_ml[(r0 + sp * rs) * 2]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float den = 0.f;
-    for (int sp = lane; sp < NS; sp += 32) {
-      const float m = ml[(long)sp * H_q * 2], l = ml[(long)sp * H_q * 2 + 1];
+    for (int sp = lane; sp < np; sp += 32) {
+      const float m = p.part_ml[(r0 + sp * rs) * 2], l = p.part_ml[(r0 + sp * rs) * 2 + 1];
       const float wv = (m == -INFINITY) ? 0.f : exp2f(m - M);
-      wgt[r * NS + sp] = wv;
+      wgt[r * NP + sp] = wv;
       den += wv * l;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float inv = den > 0.f ? 1.f / den : 0.f;
     __syncwarp();
-    for (int sp = lane; sp < NS; sp += 32) wgt[r * NS + sp] *= inv;
+    for (int sp = lane; sp < np; sp += 32) wgt[r * NP + sp] *= inv;
   }
   __syncthreads();
   // ---- O_lat rows (float4 over the latent dimension); rows R .. CMB_R-1 are zero
@@ -334,20 +402,20 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     reinterpret_cast<float4*>(olat)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = tid; e < R * c4; e += blockDim.x) {
     const int r = e / c4, v = e % c4;
-    const int b = b0 + r / G1, head = head_of_row(r);
-    const float4* src = reinterpret_cast<const float4*>(p.part_o + ((long)b * NS * H_q + head) * d_c) + v;
-    const long stride4 = (long)H_q * d_c / 4;
-    const float* wr = wgt + r * NS;
+    const int np = n_parts[r];
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + rec0[r] * d_c) + v;
+    const long long stride4 = rec_step[r] * d_c / 4;
+    const float* wr = wgt + r * NP;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    // up to kMergeBatch splits' partials in flight at a time (the loads are independent)
-    for (int sp0 = 0; sp0 < NS; sp0 += kMergeBatch) {
+    // up to kMergeBatch partials in flight at a time (the loads are independent)
+    for (int sp0 = 0; sp0 < np; sp0 += kMergeBatch) {
       float4 x[kMergeBatch];
 #pragma unroll
       for (int q = 0; q < kMergeBatch; ++q)
-        x[q] = sp0 + q < NS ? src[(sp0 + q) * stride4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[q] = sp0 + q < np ? src[(sp0 + q) * stride4] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < kMergeBatch; ++q) {
-        const float wv = sp0 + q < NS ? wr[sp0 + q] : 0.f;
+        const float wv = sp0 + q < np ? wr[sp0 + q] : 0.f;
         acc.x = fmaf(wv, x[q].x, acc.x);
         acc.y = fmaf(wv, x[q].y, acc.y);
         acc.z = fmaf(wv, x[q].z, acc.z);
@@ -485,24 +553,34 @@ cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaS
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s) {
   const size_t esz = dt == GDLA_BF16 ? 2 : 4;
   const int spb = combine_seqs(p);
+  const int max_parts = p.tc ? p.n_ranges : p.n_splits;
   // O_lat, H, merge weights, two staged W_UV blocks, and the K-slices' partial products
   // (n_slices x CMB_R x d_v = 1024 x (16 / esz) floats)
-  const size_t smem = sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * p.d_v + (size_t)CMB_R * p.n_splits) +
+  const size_t smem = sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * p.d_v + (size_t)CMB_R * max_parts) +
                       esz * 2 * (size_t)CMB_KC * p.d_v + sizeof(float) * 1024 * (16 / esz);
-  dim3 grid((unsigned)p.n_kv, (unsigned)((p.B + spb - 1) / spb));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)p.n_kv, (unsigned)((p.B + spb - 1) / spb));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  // programmatic dependent launch: the blocks stage their first W_UV rows while the
+  // split kernel finishes, and wait for it before reading its partials
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e;
   if (dt == GDLA_BF16) {
     auto k = decode_combine_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 256, smem, s>>>(p);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k, p, max_parts);
   } else {
     auto k = decode_combine_kernel<float>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 256, smem, s>>>(p);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k, p, max_parts);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace gdla

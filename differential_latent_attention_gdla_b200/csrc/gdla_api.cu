@@ -5,6 +5,10 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
 #include "../../include/gdla.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -97,47 +101,143 @@ HostLayout host_layout(const gdla_prefill_args* a, int chunk_tokens) {
   return l;
 }
 
+// The side streams and events of one gdla_prefill_host call. Created on first use
+// and kept in a per-device pool: a call borrows a set and returns it when it has
+// enqueued its work (the next user's work is ordered after it on the same streams),
+// so repeated calls create nothing and concurrent calls get different sets.
+struct HostSide {
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_c[kComputeStreams] = {};
+  cudaEvent_t ev_start = nullptr, ev_kv = nullptr, ev_exp = nullptr, ev_end = nullptr;
+  cudaEvent_t ev_in[kHostSlots] = {}, ev_comp[kHostSlots] = {}, ev_out[kHostSlots] = {};
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_host_mu;
+std::vector<HostSide*> g_host_free[kMaxDevices];
+
+cudaError_t host_side_create(HostSide* h) {
+  cudaError_t e = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking);
+  for (int i = 0; i < kComputeStreams && e == cudaSuccess; ++i)
+    e = cudaStreamCreateWithFlags(&h->s_c[i], cudaStreamNonBlocking);
+  cudaEvent_t* single[] = {&h->ev_start, &h->ev_kv, &h->ev_exp, &h->ev_end};
+  for (cudaEvent_t* ev : single)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  for (int i = 0; i < kHostSlots && e == cudaSuccess; ++i) {
+    e = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_comp[i], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming);
+  }
+  return e;
+}
+
+void host_side_destroy(HostSide* h) {
+  for (int i = 0; i < kHostSlots; ++i) {
+    if (h->ev_in[i]) cudaEventDestroy(h->ev_in[i]);
+    if (h->ev_comp[i]) cudaEventDestroy(h->ev_comp[i]);
+    if (h->ev_out[i]) cudaEventDestroy(h->ev_out[i]);
+  }
+  for (cudaEvent_t ev : {h->ev_start, h->ev_kv, h->ev_exp, h->ev_end})
+    if (ev) cudaEventDestroy(ev);
+  if (h->s_in) cudaStreamDestroy(h->s_in);
+  if (h->s_out) cudaStreamDestroy(h->s_out);
+  for (int i = 0; i < kComputeStreams; ++i)
+    if (h->s_c[i]) cudaStreamDestroy(h->s_c[i]);
+  delete h;
+}
+
+// A set of side streams and events for the current device (nullptr if creation failed).
+HostSide* host_side_acquire(int* dev_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  *dev_out = dev;
+  {
+    std::lock_guard<std::mutex> lock(g_host_mu);
+    if (!g_host_free[dev].empty()) {
+      HostSide* h = g_host_free[dev].back();
+      g_host_free[dev].pop_back();
+      return h;
+    }
+  }
+  HostSide* h = new HostSide();
+  if (host_side_create(h) != cudaSuccess) {
+    host_side_destroy(h);
+    return nullptr;
+  }
+  return h;
+}
+
+void host_side_release(HostSide* h, int dev) {
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  g_host_free[dev].push_back(h);
+}
+
+// Whether the decode runs on the tensor-core split kernel (bf16 with the report's
+// latent and rotary widths) or on the CUDA-core one.
+bool decode_uses_tc(const gdla_decode_args* a) {
+  return a->dtype == GDLA_BF16 && a->d_c == 512 && a->d_rope == 64;
+}
+
 struct DecodeLayout {
-  size_t status, q_abs, q_rot, part_o, part_ml, total;
-  int n_splits, split_len;
+  size_t status, q_abs, q_rot, qimg, seqinfo, part_o, part_ml, total;
+  int tc, n_splits, split_len, n_ranges, n_hg, hpc, part_heads;
 };
 
 DecodeLayout decode_layout(const gdla_decode_args* a) {
-  DecodeLayout l;
+  DecodeLayout l{};
   const int H_q = a->n_kv * (a->g + 1);
-  // split the cache of every sequence into n chunks (multiples of 64 tokens):
-  // B*n blocks run in waves of one block per SM, and a block moves its cache
-  // tiles plus its partial result (written here, read back by the merge).
-  // Minimise waves(B*n) * (bytes one block moves).
-  const int tile = 64;
-  const int tiles = (a->T_max + tile - 1) / tile;
-  const double tile_bytes = (double)tile * (a->d_c + a->d_rope) * 2.0;
-  const double partial_bytes = 2.0 * H_q * (a->d_c + 2) * 4.0;
-  int best_n = 1;
-  double best = 1e300;
-  for (int n = 1; n <= tiles && n <= 256; ++n) {
-    const long waves = ((long)a->B * n + kNumSMs - 1) / kNumSMs;
-    const long per = (tiles + n - 1) / n;
-    const double cost = (double)waves * (per * tile_bytes + partial_bytes);
-    if (cost < best) {
-      best = cost;
-      best_n = n;
-    }
-  }
-  const int len = ((tiles + best_n - 1) / best_n) * tile;
-  l.split_len = len;
-  l.n_splits = (a->T_max + len - 1) / len;
+  l.tc = decode_uses_tc(a) ? 1 : 0;
   size_t off = 0;
   l.status = off;
   off += kStatusBytes;
-  l.q_abs = off;
-  off = align256(off + sizeof(float) * (size_t)a->B * H_q * a->d_c);
-  l.q_rot = off;
-  off = align256(off + sizeof(float) * (size_t)a->B * H_q * a->d_rope);
+  size_t records = 0;
+  if (l.tc) {
+    // head groups of at most kDtcHeads heads; per head group, ranges of equal shares
+    // of all cache tiles, one CTA each: all CTAs together fill the SMs once, and a
+    // share is at least two tiles
+    l.n_hg = (H_q + kDtcHeads - 1) / kDtcHeads;
+    l.hpc = (H_q + l.n_hg - 1) / l.n_hg;
+    l.part_heads = kDtcHeads;
+    const long tiles_max = (long)a->B * ((a->T_max + kDtcTile - 1) / kDtcTile);
+    l.n_ranges = (int)std::max(1L, std::min((long)std::max(1, kNumSMs / l.n_hg), tiles_max / 2));
+    records = ((size_t)l.n_ranges + a->B) * l.n_hg;  // record (r + b) of every head group
+    l.qimg = off;
+    off = align256(off + (size_t)a->B * l.n_hg * kDtcImageBytes);
+    l.seqinfo = off;
+    off = align256(off + sizeof(int2) * (size_t)a->B);
+  } else {
+    // split the cache of every sequence into n chunks (multiples of 64 tokens):
+    // B*n blocks run in waves of one block per SM, and a block moves its cache
+    // tiles plus its partial result (written here, read back by the merge).
+    // Minimise waves(B*n) * (bytes one block moves).
+    const int tile = 64;
+    const int tiles = (a->T_max + tile - 1) / tile;
+    const double tile_bytes = (double)tile * (a->d_c + a->d_rope) * esize(a->dtype);
+    const double partial_bytes = 2.0 * H_q * (a->d_c + 2) * 4.0;
+    int best_n = 1;
+    double best = 1e300;
+    for (int n = 1; n <= tiles && n <= 256; ++n) {
+      const long waves = ((long)a->B * n + kNumSMs - 1) / kNumSMs;
+      const long per = (tiles + n - 1) / n;
+      const double cost = (double)waves * (per * tile_bytes + partial_bytes);
+      if (cost < best) {
+        best = cost;
+        best_n = n;
+      }
+    }
+    const int len = ((tiles + best_n - 1) / best_n) * tile;
+    l.split_len = len;
+    l.n_splits = (a->T_max + len - 1) / len;
+    l.part_heads = H_q;
+    records = (size_t)a->B * l.n_splits;
+    l.q_abs = off;
+    off = align256(off + sizeof(float) * (size_t)a->B * H_q * a->d_c);
+    l.q_rot = off;
+    off = align256(off + sizeof(float) * (size_t)a->B * H_q * a->d_rope);
+  }
   l.part_o = off;
-  off = align256(off + sizeof(float) * (size_t)a->B * l.n_splits * H_q * a->d_c);
+  off = align256(off + sizeof(float) * records * l.part_heads * a->d_c);
   l.part_ml = off;
-  off = align256(off + sizeof(float) * (size_t)a->B * l.n_splits * H_q * 2);
+  off = align256(off + sizeof(float) * records * l.part_heads * 2);
   l.total = off;
   return l;
 }
@@ -171,7 +271,8 @@ gdla_status validate_decode(const gdla_decode_args* a) {
   gdla_status st = common_dims(a->B, a->T_max, a->d_c, a->d_rope, a->n_kv, a->d_nope, a->d_v, a->n_noise,
                                a->g, a->dtype);
   if (st != GDLA_OK) return st;
-  if ((long)a->n_kv * (a->g + 1) > 64) return GDLA_ERR_UNSUPPORTED;  // query heads of one decode block
+  // the CUDA-core split kernel holds every query head of a sequence in one block
+  if (!decode_uses_tc(a) && (long)a->n_kv * (a->g + 1) > 64) return GDLA_ERR_UNSUPPORTED;
   if (a->mask != GDLA_MASK_CAUSAL && a->mask != GDLA_MASK_SLIDING) return GDLA_ERR_INVALID_ARG;
   if (a->mask == GDLA_MASK_SLIDING && a->window < 1) return GDLA_ERR_INVALID_ARG;
   if (a->rope_max_pos < a->T_max) return GDLA_ERR_INVALID_ARG;
@@ -221,7 +322,8 @@ static cudaError_t expand_rows(const gdla_expand_args* a, long tokens, int L, in
   cudaError_t e = launch_norm_rope(np, a->dtype, s);
   if (e != cudaSuccess) return e;
   GemmParams gp{tokens, a->n_kv * (a->d_nope + a->d_v), a->d_c, a->c_hat_out, a->w_ukv, a->kv_out};
-  if (a->dtype == GDLA_BF16 && gemm_tc_supported(gp)) return launch_gemm_tc(gp, status, s);
+  if (a->dtype == GDLA_BF16 && gemm_tc_shape(gp))
+    return tensor_maps_available() ? launch_gemm_tc(gp, status, s) : cudaErrorNotSupported;
   return launch_gemm_simt(gp, a->dtype, s);
 }
 
@@ -254,8 +356,8 @@ static gdla_status attend_impl(const gdla_attend_args* a, cudaStream_t s, bool c
   cudaError_t e = cudaSuccess;
   if (clear_status) e = cudaMemsetAsync(a->workspace, 0, kStatusBytes, s);
   if (e != cudaSuccess) return cuda_status(e);
-  if (attn_tc_supported(ap, a->dtype))
-    e = launch_attn_tc(ap, s);
+  if (attn_tc_shape(ap, a->dtype))
+    e = tensor_maps_available() ? launch_attn_tc(ap, s) : cudaErrorNotSupported;
   else
     e = launch_attn_simt(ap, a->dtype, s);
   return cuda_status(e);
@@ -355,23 +457,20 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
 
   // two copy streams and the compute streams; events: start, latent inputs landed,
   // latent expanded, one per slot for inputs landed / compute done / output copied,
-  // and the end of each side stream
-  cudaStream_t s_in = nullptr, s_out = nullptr, s_c[kComputeStreams] = {};
-  cudaEvent_t ev_start = nullptr, ev_kv = nullptr, ev_exp = nullptr, ev_end = nullptr;
-  cudaEvent_t ev_in[kHostSlots] = {}, ev_comp[kHostSlots] = {}, ev_out[kHostSlots] = {};
-  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
-  for (int i = 0; i < kComputeStreams && e == cudaSuccess; ++i)
-    e = cudaStreamCreateWithFlags(&s_c[i], cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_kv, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_exp, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_end, cudaEventDisableTiming);
-  for (int i = 0; i < kHostSlots && e == cudaSuccess; ++i) {
-    e = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_comp[i], cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming);
+  // and the end of each side stream (borrowed from the device's pool)
+  int device = 0;
+  HostSide* hs = host_side_acquire(&device);
+  if (!hs) {
+    cudaGetLastError();
+    return GDLA_ERR_CUDA;
   }
+  cudaStream_t s_in = hs->s_in, s_out = hs->s_out, s_c[kComputeStreams];
+  for (int i = 0; i < kComputeStreams; ++i) s_c[i] = hs->s_c[i];
+  cudaEvent_t ev_start = hs->ev_start, ev_kv = hs->ev_kv, ev_exp = hs->ev_exp, ev_end = hs->ev_end;
+  cudaEvent_t* ev_in = hs->ev_in;
+  cudaEvent_t* ev_comp = hs->ev_comp;
+  cudaEvent_t* ev_out = hs->ev_out;
+  cudaError_t e = cudaSuccess;
   bool forked = false;
   if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, kStatusBytes, s);
   if (e == cudaSuccess) e = cudaEventRecord(ev_start, s);
@@ -487,20 +586,8 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
     }
     if (e == cudaSuccess) e = j;
   }
-  // released by the runtime once their pending work completes
-  for (int i = 0; i < kHostSlots; ++i) {
-    if (ev_in[i]) cudaEventDestroy(ev_in[i]);
-    if (ev_comp[i]) cudaEventDestroy(ev_comp[i]);
-    if (ev_out[i]) cudaEventDestroy(ev_out[i]);
-  }
-  if (ev_start) cudaEventDestroy(ev_start);
-  if (ev_kv) cudaEventDestroy(ev_kv);
-  if (ev_exp) cudaEventDestroy(ev_exp);
-  if (ev_end) cudaEventDestroy(ev_end);
-  if (s_in) cudaStreamDestroy(s_in);
-  if (s_out) cudaStreamDestroy(s_out);
-  for (int i = 0; i < kComputeStreams; ++i)
-    if (s_c[i]) cudaStreamDestroy(s_c[i]);
+  // the set goes back to the pool: work enqueued by its next user is ordered after ours
+  host_side_release(hs, device);
   return cuda_status(e);
 }
 
@@ -514,22 +601,32 @@ gdla_status gdla_decode(const gdla_decode_args* a, void* stream) {
   if (st != GDLA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const DecodeLayout lay = decode_layout(a);
+  // the tensor-core path needs the driver's tensor-map encoder: no silent CUDA-core substitute
+  if (lay.tc && !tensor_maps_available()) return GDLA_ERR_CUDA;
   char* ws = (char*)a->workspace;
   DecodeParams p{};
   p.B = a->B; p.T_max = a->T_max; p.d_c = a->d_c; p.d_rope = a->d_rope; p.n_kv = a->n_kv; p.g = a->g;
   p.d_nope = a->d_nope; p.d_v = a->d_v; p.sliding = a->mask == GDLA_MASK_SLIDING;
   p.window = p.sliding ? a->window : 0; p.rope_max_pos = a->rope_max_pos;
   p.scale = default_scale(a->softmax_scale, a->d_nope, a->d_rope);
-  p.n_splits = lay.n_splits; p.split_len = lay.split_len; p.seqlens = a->seqlens;
+  p.tc = lay.tc; p.n_splits = lay.n_splits; p.split_len = lay.split_len;
+  p.n_ranges = lay.n_ranges; p.n_hg = lay.n_hg; p.hpc = lay.hpc; p.part_heads = lay.part_heads;
+  p.seqlens = a->seqlens;
   p.c_cache = a->c_cache; p.kr_cache = a->kr_cache; p.q = a->q; p.w_ukv = a->w_ukv;
   p.cos_tab = a->rope_cos; p.sin_tab = a->rope_sin; p.lam = a->lam_logits; p.gate = a->gate_logits;
-  p.out = a->out; p.q_abs = (float*)(ws + lay.q_abs); p.q_rot = (float*)(ws + lay.q_rot);
+  p.out = a->out;
+  if (lay.tc) {
+    p.qimg = (uint8_t*)(ws + lay.qimg);
+    p.seqinfo = (int2*)(ws + lay.seqinfo);
+  } else {
+    p.q_abs = (float*)(ws + lay.q_abs);
+    p.q_rot = (float*)(ws + lay.q_rot);
+  }
   p.part_o = (float*)(ws + lay.part_o); p.part_ml = (float*)(ws + lay.part_ml);
   p.status = (int*)(ws + lay.status);
   cudaError_t e = cudaMemsetAsync(p.status, 0, kStatusBytes, s);
   if (e == cudaSuccess) e = launch_decode_absorb(p, a->dtype, s);
-  if (e == cudaSuccess)
-    e = decode_tc_supported(p, a->dtype) ? launch_decode_split_tc(p, s) : launch_decode_split_simt(p, a->dtype, s);
+  if (e == cudaSuccess) e = lay.tc ? launch_decode_split_tc(p, s) : launch_decode_split_simt(p, a->dtype, s);
   if (e == cudaSuccess) e = launch_decode_combine(p, a->dtype, s);
   return cuda_status(e);
 }
@@ -571,8 +668,9 @@ gdla_status gdla_gates(const gdla_gates_args* a, void* stream) {
     e = launch_norm_rope(np, a->dtype, s);
     GemmParams gp{tokens, a->n_signal * a->d_v, a->d_q, c_hat_q, a->w_g, a->gate_logits};
     if (e == cudaSuccess)
-      e = (a->dtype == GDLA_BF16 && gemm_tc_supported(gp)) ? launch_gemm_tc(gp, status, s)
-                                                           : launch_gemm_simt(gp, a->dtype, s);
+      e = (a->dtype == GDLA_BF16 && gemm_tc_shape(gp))
+              ? (tensor_maps_available() ? launch_gemm_tc(gp, status, s) : cudaErrorNotSupported)
+              : launch_gemm_simt(gp, a->dtype, s);
   }
   if (e == cudaSuccess && a->x) {
     GemmParams lp{tokens, a->n_signal, a->d_x, a->x, a->w_lambda, a->lam_logits};

@@ -112,9 +112,7 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
-bool gemm_tc_supported(const GemmParams& p) {
-  return p.N % GN == 0 && p.K % GK == 0 && p.K >= GK && p.M >= 1 && get_encode_tiled() != nullptr;
-}
+bool gemm_tc_shape(const GemmParams& p) { return p.N % GN == 0 && p.K % GK == 0 && p.K >= GK && p.M >= 1; }
 
 cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s) {
   CUtensorMap ta, tb;

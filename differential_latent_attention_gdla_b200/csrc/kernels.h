@@ -29,8 +29,9 @@ struct GemmParams {
 cudaError_t launch_gemm_simt(const GemmParams& p, gdla_dtype dt, cudaStream_t s);
 // the same product with an fp32 C whatever the input type (lambda logits)
 cudaError_t launch_gemm_simt_f32out(const GemmParams& p, gdla_dtype dt, cudaStream_t s);
-// tcgen05/TMA version (bf16 only; M any, N % 256 == 0, K % 64 == 0).
-bool gemm_tc_supported(const GemmParams& p);
+// tcgen05/TMA version (bf16 only; M any, N % 256 == 0, K % 64 == 0): the shapes it
+// takes, and its launch.
+bool gemm_tc_shape(const GemmParams& p);
 cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s);
 
 // ---- steps 3-8: attention of every head of a KV group + differential + gate.
@@ -52,31 +53,60 @@ struct AttnParams {
   int* status;
 };
 cudaError_t launch_attn_simt(const AttnParams& p, gdla_dtype dt, cudaStream_t s);
-bool attn_tc_supported(const AttnParams& p, gdla_dtype dt);
+// shapes the tcgen05/TMA attention takes (bf16, heads of 128 + 64 rotary, d_v = 128)
+bool attn_tc_shape(const AttnParams& p, gdla_dtype dt);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
 
 // ---- decode (steps 3-8 over the latent cache, absorbed form).
+// Two layouts of the split-KV work:
+//  * tensor-core path (bf16, d_c = 512, d_rope = 64): the query heads are cut into
+//    n_hg head groups of at most kDtcHeads; per head group, n_ranges CTAs each take
+//    an equal share of all sequences' cache tiles (kDtcTile tokens each). absorb
+//    writes one query image per (sequence, head group); the split CTA of range r
+//    writes the partial of sequence b to record (r + b) * n_hg + hg, and seqinfo[b]
+//    names the first and last range that cover sequence b;
+//  * CUDA-core path (other shapes and fp32): fixed splits of [0, T_max), the
+//    partial of (b, split s) in record b * n_splits + s; q_abs / q_rot in fp32.
+constexpr int kDtcHeads = 48;                     // query heads of one split CTA
+constexpr int kDtcTile = 64;                      // cache tokens per ring stage
+constexpr int kDtcImageBytes = kDtcHeads * 576 * 2;  // query image: 9 boxes of [48 heads x 128 B]
+// byte offset of dimension d (of the 576-wide [latent | rotary] query) of local head lh
+// in a query image: 64-column boxes, rows of 128 bytes, 16-byte chunks swizzled by row
+__host__ __device__ inline int dtc_image_offset(int lh, int d) {
+  return (d >> 6) * (kDtcHeads * 128) + lh * 128 + ((((d & 63) >> 3) ^ (lh & 7)) << 4) + (d & 7) * 2;
+}
+
 struct DecodeParams {
   int B, T_max, d_c, d_rope, n_kv, g, d_nope, d_v;
   int sliding, window, rope_max_pos;
   float scale;
-  int n_splits, split_len;  // split-KV partition of [0, T_max)
+  int tc;                   // 1: tensor-core layout, 0: CUDA-core layout (see above)
+  int n_splits, split_len;  // CUDA-core path
+  int n_ranges, n_hg, hpc;  // tensor-core path: ranges per head group, head groups, heads per group
+  int part_heads;           // heads per partial record
   const int* seqlens;
   const void* c_cache; const void* kr_cache; const void* q; const void* w_ukv;
   const float* cos_tab; const float* sin_tab;
   const float* lam; const void* gate; void* out;
-  float* q_abs;     // [B, H_q, d_c]   W_UK-absorbed content query
-  float* q_rot;     // [B, H_q, d_rope] rotated rotary query
-  float* part_o;    // [B, n_splits, H_q, d_c]
-  float* part_ml;   // [B, n_splits, H_q, 2]  (running max in log2 units, sum)
+  float* q_abs;     // CUDA-core path: [B, H_q, d_c] W_UK-absorbed content query
+  float* q_rot;     // CUDA-core path: [B, H_q, d_rope] rotated rotary query
+  uint8_t* qimg;    // tensor-core path: [B * n_hg][kDtcImageBytes]
+  int2* seqinfo;    // tensor-core path: [B]
+  float* part_o;    // [records, part_heads, d_c]
+  float* part_ml;   // [records, part_heads, 2]  (running max in log2 units, sum)
   int* status;
 };
 cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
 cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
-// tcgen05/TMA split-KV pass (bf16, d_c = 512, d_rope = 64, at most 48 query heads).
-bool decode_tc_supported(const DecodeParams& p, gdla_dtype dt);
+// tcgen05/TMA split-KV pass (bf16, d_c = 512, d_rope = 64, any head count), launched
+// after absorb, whose tail it overlaps through programmatic dependent launch
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
+
+// Whether the driver's tensor-map encoder could be resolved. Every tensor-core
+// kernel needs it; a call whose shape selects one fails (GDLA_ERR_CUDA) without it
+// instead of running a CUDA-core substitute.
+bool tensor_maps_available();
 
 // ---- diagnostic: a device wait that can never complete ends at its limit and
 // records GDLA_ERR_TIMEOUT in the status word.

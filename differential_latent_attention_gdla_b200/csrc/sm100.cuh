@@ -46,6 +46,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// A CTA that starts after another one recorded a failed wait (or a launch-level
+// error) does no work. A reported argument error (an out-of-range sequence length,
+// which the kernels clamp) does not stop the others.
+__device__ __forceinline__ bool earlier_failure(const int* status) {
+  if (!status) return false;
+  const int code = *reinterpret_cast<const volatile int*>(status);
+  return code != 0 && code != (int)GDLA_ERR_INVALID_ARG;
+}
+
 // Bounded wait: gives up after ~kWaitLimitNs of wall time, or as soon as the
 // CTA's abort flag or the workspace status word is set by another waiter;
 // records GDLA_ERR_TIMEOUT and the caller's tag in the status word (if any) and
@@ -59,7 +68,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, int* sta
     if (mbar_try_wait(bar, phase)) return true;
     if ((it & 255u) == 255u) {
       const bool gave_up = globaltimer_ns() - t0 > kWaitLimitNs;
-      const bool other = (abort && *abort) || (status && *reinterpret_cast<volatile int*>(status));
+      const bool other = (abort && *abort) || earlier_failure(status);
       if (gave_up || other) {
         if (status && gave_up) {
           atomicCAS(status, 0, (int)GDLA_ERR_TIMEOUT);
@@ -69,11 +78,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, int* sta
       }
     }
   }
-}
-
-// A CTA that starts after another one recorded a failure does no work.
-__device__ __forceinline__ bool earlier_failure(const int* status) {
-  return status && *reinterpret_cast<const volatile int*>(status) != 0;
 }
 
 // ---------------------------------------------------------------------- TMA
@@ -113,6 +117,24 @@ __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// untiled bulk copy global -> this CTA's shared memory (both addresses 16-byte
+// aligned, bytes a multiple of 16), completing on an mbarrier
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// untiled L2 prefetch of a contiguous range (16-byte aligned, a multiple of 16 bytes)
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
+// ------------------------------------------------ programmatic dependent launch
+// wait until the grids this one depends on have completed and their writes are visible
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// let the next kernel in the stream (launched with programmatic serialisation) start
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 // generic-proxy smem writes -> visible to the async proxy (tcgen05.mma operands)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -20,6 +20,8 @@ EncodeTiledFn get_encode_tiled() {
   return fn;
 }
 
+bool tensor_maps_available() { return get_encode_tiled() != nullptr; }
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
                     const uint32_t* box) {
   EncodeTiledFn enc = get_encode_tiled();

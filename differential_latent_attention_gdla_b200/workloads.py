@@ -131,11 +131,18 @@ PREFILL = {
     "b2_l8k_g3": PrefillShape("bf16 prefill, causal, B=2 L=8192 g=3", B=2, L=8192, g=3),
     "b2_l64k_swa4k": PrefillShape("bf16 prefill, sliding window W=4096, B=2 L=65536 g=2", B=2, L=65536, g=2,
                                   mask="sliding", window=4096),
+    # the report's own attention layout: 16 KV heads with g = 4 (80 query heads); its
+    # sliding layers use a 128-token window
+    "b1_l32k_g4_swa128": PrefillShape("bf16 prefill, sliding window W=128, B=1 L=32768 g=4 (80 heads)", B=1,
+                                      L=32768, g=4, mask="sliding", window=128),
+    "b1_l32k_g4": PrefillShape("bf16 prefill, causal, B=1 L=32768 g=4 (80 heads)", B=1, L=32768, g=4),
 }
 DECODE = {
     "b64_t32k": DecodeShape("bf16 decode, B=64, 32768-token latent cache, g=2", B=64, T=32768, g=2),
     # a quarter-size case for profiler captures (0.6 GB of cache, still far above L2)
     "b16_t32k": DecodeShape("bf16 decode, B=16, 32768-token latent cache, g=2", B=16, T=32768, g=2),
+    # the report's 80 query heads (g = 4) over the same cache
+    "b64_t32k_g4": DecodeShape("bf16 decode, B=64, 32768-token latent cache, g=4 (80 heads)", B=64, T=32768, g=4),
 }
 
 

@@ -236,8 +236,11 @@ typedef struct {
   int window;
   float softmax_scale;       /* <= 0 selects 1/sqrt(d_nope + d_rope) */
   gdla_dtype dtype;
-  int rope_max_pos;          /* > max(seqlens) - 1 */
-  const int* seqlens;        /* [B] int32, 1 <= seqlens[b] <= T_max (device) */
+  int rope_max_pos;          /* rows of the RoPE tables; must be >= T_max (the query position is at most T_max - 1) */
+  const int* seqlens;        /* [B] int32 on the device, 1 <= seqlens[b] <= T_max. The host cannot check
+                                them: a value outside the range is clamped into it by the kernels (every
+                                access stays inside the cache and the tables) and reported as
+                                GDLA_ERR_INVALID_ARG in the workspace status word (gdla_workspace_status) */
   const void* c_cache;       /* [B, T_max, d_c] normalised latent */
   const void* kr_cache;      /* [B, T_max, d_rope] rotated rotary key */
   const void* q;             /* [B, n_signal+n_noise, d_nope+d_rope], rotary part pre-RoPE */
@@ -314,6 +317,37 @@ typedef struct {
 
 size_t gdla_gates_workspace_size(const gdla_gates_args* args);
 gdla_status gdla_gates(const gdla_gates_args* args, void* stream);
+
+/* --------------------------------------------------------------- RoPE tables
+ * The cos/sin tables every entry point takes (rope_cos, rope_sin), built on the
+ * host in double precision and rounded to fp32: model set-up, like loading the
+ * weights (copy them to the device once). Both write [max_pos, d_rope/2] row-major
+ * into caller-owned HOST arrays; entry (m, k) is cos / sin of m * theta_k.
+ *
+ * gdla_rope_tables: plain RoPE ("Open-Source Frontier Models: Architecture and
+ * Benchmarks of Rnj-1 and Motif-2", section 2, the rotation-matrix equation),
+ * theta_k = base^(-2k/d_rope), the pair (k, k + d_rope/2) rotated together.
+ *
+ * gdla_yarn_rope_tables: YaRN context extension (same section, the three-regime
+ * Scale(i) equation) of a model trained on original_max_pos tokens by `factor`:
+ * with the wavelength lambda_k = 2 pi / theta_k, a frequency is kept below
+ * original_max_pos / beta_fast, divided by `factor` above original_max_pos /
+ * beta_slow, and multiplied by (1 - a) + a / factor in between, where a grows
+ * linearly with the wavelength from 0 to 1 across that band (the report's full
+ * layers use factor 64 from 4K). Pair the tables with
+ * softmax_scale = gdla_yarn_mscale(factor)^2 / sqrt(d_nope + d_rope).
+ *
+ * gdla_yarn_mscale: YaRN's temperature 1 + 0.1 ln(factor) (1 for factor <= 1),
+ * the factor by which that section's listing scales both rotated vectors, so the
+ * logits grow by its square.
+ *
+ * Errors: GDLA_ERR_INVALID_ARG for NULL arrays, max_pos < 1, d_rope odd, < 2 or
+ * above 1024, base <= 1, factor <= 0, original_max_pos < 1 or a beta <= 0;
+ * nothing is written then. */
+gdla_status gdla_rope_tables(int max_pos, int d_rope, double base, float* cos_tab, float* sin_tab);
+gdla_status gdla_yarn_rope_tables(int max_pos, int d_rope, double base, double factor, int original_max_pos,
+                                  double beta_fast, double beta_slow, float* cos_tab, float* sin_tab);
+double gdla_yarn_mscale(double factor);
 
 /* ---------------------------------------------------------------- utilities */
 const char* gdla_status_string(gdla_status s);

@@ -27,3 +27,21 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Achieved parity margins of every comparison run in this session."""
+    try:
+        from gdla_testutil import MARGINS
+    except Exception:  # pragma: no cover
+        return
+    if not MARGINS:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", f"parity margins ({len(MARGINS)} comparisons)")
+    tr.write_line("dtype  max|e|      rms(e)/rms  max(|e|-2^-6|ref|)/rms  bound  case")
+    for what, dt, err, rel_rms, rel_elem, bound in MARGINS:
+        if dt == "fp32":
+            tr.write_line(f"fp32   {err:.3e}   -           -                       {bound:.0e}  {what}")
+        else:
+            tr.write_line(f"bf16   {err:.3e}   {rel_rms:.3e}   {rel_elem:+.3e}              {bound:.3g}   {what}")

@@ -133,7 +133,9 @@ def test_decode_validation_rejects_before_launch(lib):
     for mut, want in ((lambda a: setattr(a, "B", 0), E), (lambda a: setattr(a, "c_cache", 0), E),
                       (lambda a: setattr(a, "workspace_bytes", 1024), E), (lambda a: setattr(a, "rope_max_pos", 10), E),
                       (lambda a: setattr(a, "n_noise", 4), U), (lambda a: setattr(a, "d_rope", 48), U),
-                      (lambda a: setattr(a, "g", 4), U),  # 16 x 5 = 80 query heads: prefill only
+                      # 16 x 5 = 80 query heads: the tensor-core (bf16) decode takes them in two head
+                      # groups; the CUDA-core (fp32) decode holds at most 64 heads per block
+                      (lambda a: (setattr(a, "g", 4), setattr(a, "dtype", _abi.GDLA_FP32)), U),
                       (lambda a: (setattr(a, "mask", 1), setattr(a, "window", -3)), E)):
         a = good()
         mut(a)
@@ -243,3 +245,21 @@ def test_gates_validation_rejects_before_launch(lib):
     assert st(lambda a: setattr(a, "workspace", a.workspace + 16)) == E
     assert st(lambda a: setattr(a, "workspace_bytes", a.workspace_bytes - 1)) == E
     assert lib.gdla_gates(None, None) == E
+
+
+def test_rope_table_builders_reject_bad_arguments_and_write_nothing(lib):
+    fp = ctypes.POINTER(ctypes.c_float)
+    buf = (ctypes.c_float * 64)(*([7.0] * 64))
+    p = ctypes.cast(buf, fp)
+    E = _abi.GDLA_ERR_INVALID_ARG
+    assert lib.gdla_rope_tables(0, 8, 10000.0, p, p) == E
+    assert lib.gdla_rope_tables(4, 7, 10000.0, p, p) == E
+    assert lib.gdla_rope_tables(4, 8, 1.0, p, p) == E
+    assert lib.gdla_rope_tables(4, 8, 10000.0, None, p) == E
+    assert lib.gdla_yarn_rope_tables(4, 8, 10000.0, 0.0, 64, 32.0, 1.0, p, p) == E
+    assert lib.gdla_yarn_rope_tables(4, 8, 10000.0, 4.0, 0, 32.0, 1.0, p, p) == E
+    assert lib.gdla_yarn_rope_tables(4, 8, 10000.0, 4.0, 64, 0.0, 1.0, p, p) == E
+    assert list(buf) == [7.0] * 64
+    assert lib.gdla_rope_tables(4, 8, 10000.0, p, ctypes.cast(ctypes.byref(buf, 64), fp)) == _abi.GDLA_OK
+    assert buf[0] == 1.0 and buf[16] == 0.0  # position 0: cos 1, sin 0
+    assert lib.gdla_yarn_mscale(1.0) == 1.0 and lib.gdla_yarn_mscale(0.5) == 1.0

@@ -14,9 +14,11 @@ import torch
 
 import differential_latent_attention_gdla_b200 as gdla
 from differential_latent_attention_gdla_b200 import workloads as wl
-from gdla_testutil import assert_parity, f64, oracle_decode, oracle_prefill_rows
+from gdla_testutil import (assert_parity, f64, max_decode_logit, oracle_decode, oracle_prefill_rows,
+                           peaked_elem_bound)
 
 import oracle
+from differential_latent_attention_gdla_b200 import _abi
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -85,7 +87,7 @@ def test_prefill_full_size_sampled_rows(name):
     inp = wl.make_prefill_inputs(shape, seed=0, device=DEV)
     y = run_prefill(shape, inp)
     torch.cuda.synchronize()
-    rows = wl.sample_rows(shape, n_random=8 if shape.mask == "sliding" else 12)
+    rows = wl.sample_rows(shape, n_random=32)
     ref = oracle_prefill_rows(inp, rows, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=shape.mask,
                               window=shape.window)
     rb = torch.tensor([r[0] for r in rows], device=DEV)
@@ -160,7 +162,10 @@ def test_decode_small_every_element(case, act):
     assert_parity(f64(y), ref, wl.torch_dtype(shape.dtype), shape.name)
 
 
-def test_decode_full_size_sampled():
+def test_decode_full_size_every_sequence():
+    """The bench decode workload (64 sequences x 32768 cached tokens) in the bench's
+    launch configuration: every sequence is checked, each on one KV group (its g
+    signal heads and the noise head), the group rotating so all 16 are covered."""
     shape = wl.DECODE["b64_t32k"]
     inp = wl.make_decode_inputs(shape, seed=0, device=DEV)
     cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
@@ -168,9 +173,72 @@ def test_decode_full_size_sampled():
                     inp["gate_logits"], inp["seqlens"], g=shape.g)
     torch.cuda.synchronize()
     assert torch.isfinite(y).all()
-    seqs = [0, 37, 63]
-    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, seqs=seqs, kv_sel=[0, 9, 15])
-    assert_parity(f64(y[seqs]), ref, torch.bfloat16, "decode b64_t32k")
+    got, ref = [], []
+    for b in range(shape.B):
+        h = b % shape.n_kv
+        r = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, seqs=[b], kv_sel=[h])[0]
+        got.append(f64(y[b, h * shape.g:(h + 1) * shape.g]))
+        ref.append(r[h * shape.g:(h + 1) * shape.g])
+    assert_parity(np.stack(got), np.stack(ref), torch.bfloat16, "decode b64_t32k, all sequences")
+
+
+def test_decode_80_heads_g4():
+    """The report's head layout in decode: 16 KV heads with g = 4 (64 signal + 16
+    noise = 80 query heads), split over two head groups of the split kernel."""
+    for mask, window in (("causal", 0), ("sliding", 128)):
+        shape = wl.DecodeShape("decode 80 heads", B=5, T=700, n_kv=16, g=4)
+        inp = wl.make_decode_inputs(shape, seed=51, device=DEV, act="unit", seqlens=[700, 513, 129, 48, 1])
+        cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+        y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                        inp["gate_logits"], inp["seqlens"], g=shape.g, mask=mask, window=window)
+        torch.cuda.synchronize()
+        ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=mask, window=window)
+        assert_parity(f64(y), ref, torch.bfloat16, f"decode 80 heads g=4 {mask}")
+
+
+def test_decode_many_sequences_per_split_block():
+    """Many short sequences: one split block covers several whole sequences and the
+    parts of two more, so it changes sequence (query operand, running maxima and
+    value accumulator) between tiles."""
+    shape = wl.DecodeShape("decode many short", B=300, T=200, n_kv=2, g=2)
+    gen = torch.Generator().manual_seed(5)
+    seqlens = torch.randint(1, shape.T + 1, (shape.B,), generator=gen).tolist()
+    seqlens[:4] = [1, 1, 48, 49]
+    inp = wl.make_decode_inputs(shape, seed=52, device=DEV, act="unit", seqlens=seqlens)
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g)
+    torch.cuda.synchronize()
+    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
+    assert_parity(f64(y), ref, torch.bfloat16, "decode 300 short sequences")
+
+
+def test_decode_out_of_range_seqlens_are_clamped_and_reported():
+    """A sequence length outside [1, T_max] (which the host cannot see: seqlens live
+    on the device) is clamped into the cache by every decode kernel and reported as
+    GDLA_ERR_INVALID_ARG in the workspace status word; the other sequences are
+    still computed correctly."""
+    for dtype in ("bf16", "fp32"):
+        shape = wl.DecodeShape(f"decode bad seqlens {dtype}", B=4, T=160, n_kv=2, g=2, dtype=dtype)
+        inp = wl.make_decode_inputs(shape, seed=53, device=DEV, act="unit", seqlens=[160, 0, 77, 100000])
+        cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+        ws = torch.empty(gdla.decode_workspace_size(B=shape.B, T_max=shape.T, d_c=shape.d_c, d_rope=shape.d_R,
+                                                    n_kv=shape.n_kv, d_nope=shape.d_n, d_v=shape.d_v, g=shape.g,
+                                                    dtype=wl.torch_dtype(dtype)), dtype=torch.uint8, device=DEV)
+        y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                        inp["gate_logits"], inp["seqlens"], g=shape.g, workspace=ws)
+        torch.cuda.synchronize()
+        assert gdla.workspace_status(ws) == _abi.GDLA_ERR_INVALID_ARG
+        ok = [0, 2]
+        ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, seqs=ok)
+        assert_parity(f64(y[ok]), ref, wl.torch_dtype(dtype), f"decode with bad seqlens, good rows ({dtype})")
+        # the clamped ones equal the decode of their clamped lengths
+        inp2 = dict(inp, seqlens=torch.tensor([160, 1, 77, 160], dtype=torch.int32, device=DEV))
+        y2 = gdla.decode(inp2["c_cache"], inp2["kr_cache"], inp2["q"], inp2["w_ukv"], cos, sin, inp2["lam_logits"],
+                         inp2["gate_logits"], inp2["seqlens"], g=shape.g, workspace=ws)
+        torch.cuda.synchronize()
+        assert gdla.workspace_status(ws) == 0
+        assert torch.equal(y, y2)
 
 
 def test_binding_raises_on_invalid_arguments():
@@ -193,9 +261,11 @@ def test_decode_peaked_softmax_rescale_path(scale):
     torch.cuda.synchronize()
     ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
     # logits reach |s| ~ 50-150 here: the bf16 absorbed query moves single
-    # exponents by ~|s| 2^-9, so only the RMS bar applies (a wrong rescale
-    # would be an O(1) error)
-    assert_parity(f64(y), ref, torch.bfloat16, f"decode peaked x{scale}", elementwise=False)
+    # exponents by ~|s| 2^-9, so the element bound grows with the largest logit
+    # (a wrong rescale would be an O(1) error in the RMS bar as well)
+    smax = max_decode_logit(inp, g=shape.g, d_nope=shape.d_n, scale=gdla.default_scale(shape.d_n, shape.d_R))
+    assert_parity(f64(y), ref, torch.bfloat16, f"decode peaked x{scale} (max logit {smax:.0f})",
+                  elem_bound=peaked_elem_bound(smax))
 
 
 @pytest.mark.parametrize("g", [1, 5, 8])
@@ -225,7 +295,9 @@ def test_decode_peaked_multi_tile_splits():
                     inp["gate_logits"], inp["seqlens"], g=shape.g)
     torch.cuda.synchronize()
     ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
-    assert_parity(f64(y), ref, torch.bfloat16, "decode peaked multi-tile", elementwise=False)
+    smax = max_decode_logit(inp, g=shape.g, d_nope=shape.d_n, scale=gdla.default_scale(shape.d_n, shape.d_R))
+    assert_parity(f64(y), ref, torch.bfloat16, f"decode peaked multi-tile (max logit {smax:.0f})",
+                  elem_bound=peaked_elem_bound(smax))
 
 
 # ------------------------------------------------------------------ YaRN context extension
