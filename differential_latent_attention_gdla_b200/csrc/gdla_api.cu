@@ -674,7 +674,9 @@ gdla_status gdla_gates(const gdla_gates_args* a, void* stream) {
   }
   if (e == cudaSuccess && a->x) {
     GemmParams lp{tokens, a->n_signal, a->d_x, a->x, a->w_lambda, a->lam_logits};
-    e = launch_gemm_simt_f32out(lp, a->dtype, s);
+    e = (a->dtype == GDLA_BF16 && gemm_tc_shape(lp))
+            ? (tensor_maps_available() ? launch_gemm_tc_f32out(lp, status, s) : cudaErrorNotSupported)
+            : launch_gemm_simt_f32out(lp, a->dtype, s);
   }
   return cuda_status(e);
 }

@@ -1,132 +1,272 @@
-// gemm_tc.cu -- the single W_UKV up-projection of the normalised latent on the
-// 5th-generation tensor cores ("Motif 3: Technical Report", Architecture: the
-// KV latent is expanded through a single projection into the shared key/value
-// heads): KV[M, N] = c_hat[M, K] @ W_UKV[K, N], bf16 in, fp32 accumulate in
-// TMEM, bf16 out.
+// gemm_tc.cu -- C[M, N] = A[M, K] @ B[K, N] (row-major, bf16 in, fp32 accumulation
+// in TMEM) on the 5th-generation tensor cores. It serves the single W_UKV
+// up-projection of the normalised latent ("Motif 3: Technical Report",
+// Architecture: the KV latent is expanded through a single projection into the
+// shared key/value heads), the gate projection of the normalised query latent
+// (bf16 out) and the lambda projection x W_lambda (fp32 out, N = n_signal).
 //
-// One CTA per 128 x 256 output tile. Warp 0 (one lane) streams K-blocks of 64
-// through a 4-stage TMA ring (A: K-major 128x64 tile; B: four MN-major 64x64
-// tiles of W), warp 1 (one lane) issues tcgen05.mma 128x256x16 into a 256-column
-// TMEM accumulator, and all four warps drain TMEM (one row per thread) into
-// bf16 rows of KV.
+// Persistent: one CTA per SM walks the 128 x BN output tiles in row-major tile
+// order (CTA i takes tiles i, i + grid, ...), so the CTAs running at one time
+// share their A rows in L2. Warp roles (256 threads):
+//   warp 0      TMA producer (one lane): K-blocks of 64 through a STAGES-deep ring
+//               (A: a K-major 128 x 64 box; B: BN/64 MN-major 64 x 64 boxes of W);
+//   warp 1      MMA issuer (one lane): tcgen05.mma 128 x BN x 16 into one of two
+//               TMEM accumulators (BN columns each), alternating per tile;
+//   warps 4-7   epilogue: warp w drains TMEM lanes 32(w-4) .. +31 (one output row
+//               per thread) of the finished accumulator and stores the row, while
+//               the MMAs of the next tile fill the other accumulator.
+// Tails: rows of A beyond M and columns of B beyond N are zero-filled by TMA and
+// not stored; a K that is not a multiple of 64 is zero-filled the same way.
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace gdla {
-namespace {
-constexpr int GM = 128, GN = 256, GK = 64, GSTAGES = 4;
-constexpr int A_BYTES = GM * GK * 2;  // 16 KB
-constexpr int B_BYTES = GK * GN * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GEMM_SMEM = GSTAGES * STAGE_BYTES + 1024;
-}  // namespace
+namespace gtc {
 
-__global__ void __launch_bounds__(128, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   __nv_bfloat16* __restrict__ C, long M, int N, int K, int* status) {
+constexpr int GM = 128, GK = 64;
+constexpr int GTHREADS = 256;
+constexpr int kNumSMs = 148;
+
+template <int BN, int STAGES>
+struct Cfg {
+  static constexpr int A_BYTES = GM * GK * 2;  // 16 KB
+  static constexpr int B_BYTES = GK * BN * 2;  // BN/64 boxes of 8 KB
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int OFF_BARS = STAGES * STAGE;
+  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+  static_assert(BN % 64 == 0 && BN <= 256, "B is loaded in 64-column boxes; one MMA covers N <= 256");
+  static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation: a power of two <= 512");
+};
+
+template <int STAGES>
+struct Bars {
+  uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], mma_done;
+  uint32_t tmem_slot;
+  int abort_flag;
+};
+
+template <typename OutT>
+__device__ __forceinline__ void store_chunk(OutT* dst, const uint32_t (&r)[32], int ncols);
+
+// 32 accumulator columns of one row: bf16 (four 16-byte stores) ...
+template <>
+__device__ __forceinline__ void store_chunk<__nv_bfloat16>(__nv_bfloat16* dst, const uint32_t (&r)[32], int ncols) {
   using namespace sm100;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full[GSTAGES], empty[GSTAGES], acc_full;
-  __shared__ uint32_t tmem_slot;
+  uint32_t p[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) p[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  // a column tail stores whole 16-byte pieces (N is a multiple of 8)
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (8 * i < ncols) d[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+}
+// ... or fp32 (eight 16-byte stores)
+template <>
+__device__ __forceinline__ void store_chunk<float>(float* dst, const uint32_t (&r)[32], int ncols) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (4 * i < ncols) d[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+}
+
+}  // namespace gtc
+
+struct GemmTcArgs {
+  long M;
+  int N, K;
+  int n_tm, n_tn;  // output tiles along M and N
+  void* C;
+  int* status;
+};
+
+template <int BN, int STAGES, typename OutT>
+__global__ void __launch_bounds__(gtc::GTHREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmTcArgs a) {
+  using namespace sm100;
+  using namespace gtc;
+  using C_ = Cfg<BN, STAGES>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  Bars<STAGES>& bars = *reinterpret_cast<Bars<STAGES>*>(smem + C_::OFF_BARS);
+  volatile int& abort_flag = bars.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * GN;
-  const long m0 = (long)blockIdx.y * GM;
-  const int KT = K / GK;
+  if (smem_u32(smem) & 1023u) {
+    // the swizzled operand tiles need 1024-byte alignment: report instead of computing garbage
+    if (threadIdx.x == 0 && a.status) {
+      atomicCAS(a.status, 0, (int)GDLA_ERR_CUDA);
+      atomicCAS(a.status + 1, 0, 199);
+    }
+    return;
+  }
+  if (earlier_failure(a.status)) return;
+  const long n_tiles = (long)a.n_tm * a.n_tn;
+  const int KT = (a.K + GK - 1) / GK;
+  // tiles of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int my_tiles = (int)((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < GSTAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&bars.full[s]), 1);
+      mbar_init(smem_u32(&bars.empty[s]), 1);
     }
-    mbar_init(smem_u32(&acc_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars.acc_full[i]), 1);
+      mbar_init(smem_u32(&bars.acc_empty[i]), 128);
+    }
+    mbar_init(smem_u32(&bars.mma_done), 1);
     fence_mbar_init();
+    abort_flag = 0;
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&tmem_slot), 256);
+    tmem_alloc(smem_u32(&bars.tmem_slot), C_::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_slot;
+  const uint32_t tmem = bars.tmem_slot;
 
-  if (warp == 0 && lane == 0) {
-    // TMA producer
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % GSTAGES;
-      if (kt >= GSTAGES && !mbar_wait(smem_u32(&empty[s]), ((kt / GSTAGES) & 1) ^ 1, status, 101)) break;
-      const uint32_t a_dst = smem_u32(smem + s * STAGE_BYTES), b_dst = a_dst + A_BYTES;
-      const uint32_t bar = smem_u32(&full[s]);
-      mbar_expect_tx(bar, STAGE_BYTES);
-      tma_load_2d(a_dst, &tmA, bar, kt * GK, (int)m0);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      long kc = 0;  // K-blocks issued over all tiles (ring position and phase)
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const long t = blockIdx.x + (long)i * gridDim.x;
+        const long m0 = (t / a.n_tn) * GM;
+        const int n0 = (int)(t % a.n_tn) * BN;
+        for (int kb = 0; kb < KT; ++kb, ++kc) {
+          const int s = (int)(kc % STAGES);
+          if (kc >= STAGES &&
+              !mbar_wait(smem_u32(&bars.empty[s]), (int)((kc / STAGES) & 1) ^ 1, a.status, 101, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = smem_u32(smem + s * C_::STAGE), b_dst = a_dst + C_::A_BYTES;
+          const uint32_t bar = smem_u32(&bars.full[s]);
+          mbar_expect_tx(bar, C_::STAGE);
+          tma_load_2d(a_dst, &tmA, bar, kb * GK, (int)m0);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * (GK * 64 * 2), &tmB, bar, n0 + 64 * j, kt * GK);
+          for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * (GK * 128), &tmB, bar, n0 + 64 * j, kb * GK);
+        }
+      }
+      if (!ok) {
+        abort_flag = 1;
+        // wait (bounded) for the copies in flight before the CTA may exit
+        for (long c = (kc > STAGES ? kc - STAGES : 0); c < kc; ++c)
+          mbar_wait(smem_u32(&bars.full[c % STAGES]), (int)((c / STAGES) & 1), nullptr, 0);
+      }
     }
-  } else if (warp == 1 && lane == 0) {
-    // MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(GM, GN, false, true);
-    bool ok = true;
-    for (int kt = 0; kt < KT && ok; ++kt) {
-      const int s = kt % GSTAGES;
-      ok = mbar_wait(smem_u32(&full[s]), (kt / GSTAGES) & 1, status, 102);
-      if (!ok) break;
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(GM, BN, false, true);
+      long kc = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int buf = i & 1;
+        // the epilogue has drained this accumulator (tile i - 2)
+        if (i >= 2)
+          ok = mbar_wait(smem_u32(&bars.acc_empty[buf]), ((i >> 1) & 1) ^ 1, a.status, 104, &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < KT; ++kb, ++kc) {
+          const int s = (int)(kc % STAGES);
+          ok = mbar_wait(smem_u32(&bars.full[s]), (int)((kc / STAGES) & 1), a.status, 102, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t as = smem_u32(smem + s * C_::STAGE), bs = as + C_::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < GK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(as + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(bs + kk * 2048, GK * 128, 1024);
+            mma_ss(acc, ad, bd, idesc, (kb | kk) != 0);
+          }
+          mma_commit(smem_u32(&bars.empty[s]));
+        }
+        if (ok) mma_commit(smem_u32(&bars.acc_full[buf]));
+      }
+      if (!ok) abort_flag = 1;
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(smem_u32(&bars.mma_done));
+      mbar_wait(smem_u32(&bars.mma_done), 0, nullptr, 105);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp - 4;
+    OutT* C = reinterpret_cast<OutT*>(a.C);
+    for (int i = 0; i < my_tiles; ++i) {
+      const int buf = i & 1;
+      bool ok = mbar_wait(smem_u32(&bars.acc_full[buf]), (i >> 1) & 1, a.status, 103, &abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        abort_flag = 1;
+        break;
+      }
       tc_fence_after();
-      const uint32_t a = smem_u32(smem + s * STAGE_BYTES), b = a + A_BYTES;
-#pragma unroll
-      for (int kk = 0; kk < GK / 16; ++kk) {
-        const uint64_t ad = sdesc_sw128(a + kk * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(b + kk * 2048, GK * 64 * 2, 1024);
-        mma_ss(tmem, ad, bd, idesc, (kt | kk) != 0);
-      }
-      mma_commit(smem_u32(&empty[s]));
-    }
-    mma_commit(smem_u32(&acc_full));
-  }
-  __syncwarp();
-  // epilogue: warp w drains TMEM lanes 32w..32w+31 (= tile rows)
-  const bool ok = mbar_wait(smem_u32(&acc_full), 0, status, 103);
-  tc_fence_after();
-  if (ok) {
-    const long row = m0 + warp * 32 + lane;
+      const long t = blockIdx.x + (long)i * gridDim.x;
+      const long row = (t / a.n_tn) * GM + q4 * 32 + lane;
+      const int n0 = (int)(t % a.n_tn) * BN;
 #pragma unroll 1
-    for (int ch = 0; ch < GN / 32; ++ch) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + ch * 32, r);
-      tmem_wait_ld();
-      if (row < M) {
-        uint32_t p[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) p[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-        uint4* dst = reinterpret_cast<uint4*>(C + row * N + n0 + ch * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN + ch * 32), r);
+        tmem_wait_ld();
+        const int c0 = n0 + ch * 32;
+        if (row < a.M && c0 < a.N) store_chunk<OutT>(C + row * a.N + c0, r, a.N - c0);
       }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars.acc_empty[buf]));
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 256);
+  if (warp == 0) tmem_dealloc(tmem, C_::TMEM_COLS);
 }
 
-bool gemm_tc_shape(const GemmParams& p) { return p.N % GN == 0 && p.K % GK == 0 && p.K >= GK && p.M >= 1; }
+bool gemm_tc_shape(const GemmParams& p) {
+  // TMA needs 16-byte row strides: K and N multiples of 8
+  return p.M >= 1 && p.K >= 8 && p.K % 8 == 0 && p.N >= 8 && p.N % 8 == 0;
+}
 
-cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s) {
+template <int BN, int STAGES, typename OutT>
+static cudaError_t launch_cfg(const GemmParams& p, int* status, cudaStream_t s) {
+  using C_ = gtc::Cfg<BN, STAGES>;
+  constexpr int SMEM = C_::OFF_BARS + (int)sizeof(gtc::Bars<STAGES>);
+  static_assert(SMEM <= 232448, "shared memory budget of one CTA");
   CUtensorMap ta, tb;
   const uint64_t adims[2] = {(uint64_t)p.K, (uint64_t)p.M}, astr[1] = {(uint64_t)p.K * 2};
-  const uint32_t abox[2] = {64, GM};
+  const uint32_t abox[2] = {64, gtc::GM};
   const uint64_t bdims[2] = {(uint64_t)p.N, (uint64_t)p.K}, bstr[1] = {(uint64_t)p.N * 2};
-  const uint32_t bbox[2] = {64, GK};
+  const uint32_t bbox[2] = {64, gtc::GK};
   if (!make_tmap_bf16(&ta, p.A, 2, adims, astr, abox) || !make_tmap_bf16(&tb, p.Bm, 2, bdims, bstr, bbox))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM);
+  GemmTcArgs a{};
+  a.M = p.M; a.N = p.N; a.K = p.K;
+  a.n_tm = (int)((p.M + gtc::GM - 1) / gtc::GM);
+  a.n_tn = (p.N + BN - 1) / BN;
+  a.C = p.C; a.status = status;
+  auto kern = gemm_tc_kernel<BN, STAGES, OutT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(p.N / GN), (unsigned)((p.M + GM - 1) / GM));
-  gemm_tc_kernel<<<grid, 128, GEMM_SMEM, s>>>(ta, tb, reinterpret_cast<__nv_bfloat16*>(p.C), p.M, p.N, p.K, status);
+  const long tiles = (long)a.n_tm * a.n_tn;
+  const int grid = (int)(tiles < gtc::kNumSMs ? tiles : gtc::kNumSMs);
+  kern<<<grid, gtc::GTHREADS, SMEM, s>>>(ta, tb, a);
   return cudaGetLastError();
+}
+
+// bf16 output: 128 x 256 tiles (the expansion, the gate projection), 128 x 64 when N is narrow
+cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s) {
+  return p.N > 64 ? launch_cfg<256, 4, __nv_bfloat16>(p, status, s) : launch_cfg<64, 8, __nv_bfloat16>(p, status, s);
+}
+
+// fp32 output (the lambda logits, N = n_signal): 128 x 64 tiles, 128 x 256 when N is wider
+cudaError_t launch_gemm_tc_f32out(const GemmParams& p, int* status, cudaStream_t s) {
+  return p.N > 64 ? launch_cfg<256, 4, float>(p, status, s) : launch_cfg<64, 8, float>(p, status, s);
 }
 
 }  // namespace gdla

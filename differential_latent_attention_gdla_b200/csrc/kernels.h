@@ -29,10 +29,11 @@ struct GemmParams {
 cudaError_t launch_gemm_simt(const GemmParams& p, gdla_dtype dt, cudaStream_t s);
 // the same product with an fp32 C whatever the input type (lambda logits)
 cudaError_t launch_gemm_simt_f32out(const GemmParams& p, gdla_dtype dt, cudaStream_t s);
-// tcgen05/TMA version (bf16 only; M any, N % 256 == 0, K % 64 == 0): the shapes it
-// takes, and its launch.
+// tcgen05/TMA version (bf16 inputs; any M, N and K multiples of 8): the shapes it
+// takes, and its launches with a bf16 or an fp32 C.
 bool gemm_tc_shape(const GemmParams& p);
 cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s);
+cudaError_t launch_gemm_tc_f32out(const GemmParams& p, int* status, cudaStream_t s);
 
 // ---- steps 3-8: attention of every head of a KV group + differential + gate.
 // The query side covers the block of positions q_start .. q_start+q_len-1 of every
@@ -56,6 +57,8 @@ cudaError_t launch_attn_simt(const AttnParams& p, gdla_dtype dt, cudaStream_t s)
 // shapes the tcgen05/TMA attention takes (bf16, heads of 128 + 64 rotary, d_v = 128)
 bool attn_tc_shape(const AttnParams& p, gdla_dtype dt);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+// the same attention with two head pairs in flight per CTA (attn_pp.cu)
+cudaError_t launch_attn_pp(const AttnParams& p, cudaStream_t s);
 
 // ---- decode (steps 3-8 over the latent cache, absorbed form).
 // Two layouts of the split-KV work:

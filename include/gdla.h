@@ -18,10 +18,10 @@
  *    row-major in the layout stated beside them, 16-byte aligned. The library
  *    allocates no memory and keeps no per-call state; scratch comes from the
  *    caller's workspace, sized by the matching *_workspace_size function.
- *    Two entry points state their exceptions beside them: gdla_prefill_host
- *    takes its activations as host pointers and creates (and releases) its own
- *    copy and compute streams, and gdla_decode_noalloc uses a fixed scratch
- *    array inside the library instead of a workspace.
+ *    Three entry points state their exceptions beside them: gdla_prefill_host
+ *    takes its activations as host pointers and keeps its own copy and compute
+ *    streams, gdla_decode_noalloc uses a fixed scratch array inside the library
+ *    instead of a workspace, and the RoPE table builders write host arrays.
  *  - `stream` is a cudaStream_t passed as void*. All work is enqueued on it and
  *    the call returns without synchronising.
  *  - Argument errors (NULL pointer, misalignment, unsupported size, a too
@@ -65,11 +65,14 @@ typedef enum { GDLA_BF16 = 0, GDLA_FP32 = 1 } gdla_dtype;
  * floor(i/g) and subtracts noise head floor(i/g) (Repeat_g as
  * repeat-interleave). Supported head shapes (d_nope, d_rope, d_v):
  * (128, 64, 128), (64, 32, 64), (32, 16, 32); d_c in {64, 128, 256, 512};
- * 1 <= g <= 8; decode additionally n_kv * (g + 1) <= 64 query heads (prefill
- * takes any head count, e.g. the report's 16 KV heads with g = 4, 80 heads).
- * Other sizes return GDLA_ERR_UNSUPPORTED. The tensor-core kernels serve bf16: prefill with
- * (128, 64, 128) heads, decode with d_c = 512, d_rope = 64 and at most 48
- * query heads; every other supported shape runs on the CUDA-core kernels. */
+ * 1 <= g <= 8. Other sizes return GDLA_ERR_UNSUPPORTED. The tensor-core kernels
+ * serve bf16: prefill with (128, 64, 128) heads and any head count (e.g. the
+ * report's 16 KV heads with g = 4, 80 query heads), decode with d_c = 512 and
+ * d_rope = 64 and any head count (in groups of at most 48 query heads); every
+ * other supported shape runs on the CUDA-core kernels, where decode holds at most
+ * 64 query heads. A call whose shape selects a tensor-core kernel fails with
+ * GDLA_ERR_CUDA if the driver's tensor-map encoder cannot be resolved; there is
+ * no CUDA-core substitute for those shapes. */
 
 /* ------------------------------------------------------------------ expansion
  * Steps 1-3 of the layer for a whole batch: latent RMSNorm, the single W_UKV
@@ -209,9 +212,10 @@ gdla_status gdla_attend(const gdla_attend_args* args, void* stream);
  * copies of c_kv and k_rope, and eight chunk-sized staging slots per query-side
  * tensor (q, lambda, gate, Y) that the chunks take in turn.
  *
- * Per call, the library creates two non-blocking copy streams, two compute
- * streams and a few events.
- * They are released once their work completes. All work is ordered after
+ * The call uses two non-blocking copy streams, two compute streams and a few
+ * events of its own. They are created by the first call on a device and kept by
+ * the library for later calls (a call that overlaps another one on the host gets
+ * a set of its own); nothing is created per call after that. All work is ordered after
  * earlier work on `stream`, and later work on `stream` waits for all of it.
  * Like every entry point, the call returns without synchronising, so `out` is
  * valid only after `stream` has been synchronised, and the host inputs must
@@ -294,9 +298,10 @@ gdla_status gdla_decode_noalloc(const gdla_decode_args* args, void* stream);
  *  - c_q == NULL skips the gate (gamma_q, w_g and gate_logits are then ignored);
  *  - x == NULL skips lambda (w_lambda and lam_logits are then ignored).
  * The normalisation is the latent RMSNorm of gdla_latent_expand with its own gain.
- * The gate product runs on the tensor cores for bf16 with n_signal*d_v a multiple
- * of 256 and d_q a multiple of 64 (the report's shapes: d_q = 1536, n_signal*d_v =
- * 4096 or 6144), and on the CUDA cores otherwise; lambda always on the CUDA cores.
+ * Both products run on the tensor cores for bf16 when their widths (d_q, d_x,
+ * n_signal*d_v, n_signal) are multiples of 8 (the report's shapes: d_q = 1536,
+ * n_signal*d_v = 4096 or 6144, n_signal = 32 or 48), lambda with fp32 output, and
+ * on the CUDA cores otherwise.
  * The workspace (>= gdla_gates_workspace_size(args) bytes, 256-byte aligned) holds
  * the status word and, when the gate is computed, c_hat_q [B*L, d_q]. */
 typedef struct {

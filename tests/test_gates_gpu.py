@@ -1,8 +1,9 @@
 """GPU parity of gdla_gates, the gate and lambda logits computed from the layer's
 activations ("Motif 3: Technical Report", section "Architecture": lambda_t =
 sigmoid(x_t W_lambda); the output gate comes from the normalised query latent),
-against the fp64 oracle on the same seeded inputs. The report's shapes take the
-tensor-core product; odd widths and fp32 take the CUDA cores."""
+against the fp64 oracle on the same seeded inputs. bf16 products whose widths are
+multiples of 8 run on the tensor cores (the gate with bf16 output, lambda with fp32
+output); other widths and fp32 take the CUDA cores."""
 import math
 
 import numpy as np
@@ -51,10 +52,27 @@ def test_gates_report_shapes_tensor_cores(n_S):
     check(inp, n_S, 128, torch.bfloat16, f"bf16 n_S={n_S}")
 
 
-def test_gates_odd_widths_cuda_cores():
-    # n_S * d_v = 384 is not a multiple of 256 and d_q = 200 not one of 64
+def test_gates_odd_widths():
+    # gate: n_S * d_v = 384 is not a multiple of the 256-column tile and d_q = 200 not one of
+    # the 64-deep K block (tensor cores, zero-filled tails); lambda: n_S = 6 (CUDA cores)
     inp = make(3, 77, 200, 96, 6, 64, torch.bfloat16, seed=5)
     check(inp, 6, 64, torch.bfloat16, "bf16 odd widths")
+
+
+def test_gates_many_tiles_per_block():
+    # 1024 tokens x 6144 gate columns = 192 output tiles of 128 x 256 on 148 blocks, and
+    # 40000 tokens of lambda = 313 tiles of 128 x 64 (fp32): both walk several tiles per
+    # block through the double-buffered accumulator, with a ragged last row tile
+    inp = make(1, 1024, 1536, 2048, 48, 128, torch.bfloat16, seed=11)
+    check(inp, 48, 128, torch.bfloat16, "bf16 1024 tokens, 48 signal heads")
+    g = torch.Generator(device="cpu").manual_seed(12)
+    x = torch.randn(40000, 2048, generator=g).to(torch.bfloat16).to(DEV)
+    w = (torch.randn(2048, 40, generator=g) / math.sqrt(2048)).to(torch.bfloat16).to(DEV)
+    _, lam = gdla.gates(x=x, w_lambda=w, n_signal=40)
+    torch.cuda.synchronize()
+    ref = oracle.lambda_logits(f64(x), f64(w))
+    err = np.abs(f64(lam) - ref)
+    assert err.max() <= 1e-4 * max(1.0, float(np.abs(ref).max())), err.max()
 
 
 def test_gates_fp32_tiny_config():
