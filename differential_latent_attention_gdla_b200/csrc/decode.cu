@@ -24,12 +24,13 @@ namespace gdla {
 constexpr int ABS_C = 128;   // latent rows per block: 32 threads x 4
 constexpr int ABS_R = 48;    // query rows per block at most: 8 warps x ABS_RPW
 constexpr int ABS_RPW = ABS_R / 8;
-// Combine blocks: KV group x (up to 16 query rows). The W_UV product gives each thread
-// 4 query rows x one 16-byte vector of value columns over one K-slice of every staged
-// block of latent rows; the slices' partial sums are added in a fixed order.
-constexpr int CMB_R = 16;   // query rows per block at most
-constexpr int CMB_KC = 64;   // latent rows of W_UV staged per step
+// Combine blocks: KV group x (up to CMB_R query rows = sequences x heads of the group).
+// A block stages its group's W_UV rows (all of them when they fit) before it waits for
+// the split kernel, and every thread accumulates 8 value columns of up to two query
+// rows over the whole latent dimension.
+constexpr int CMB_R = 32;   // query rows per block at most
 constexpr int kMergeBatch = 12;  // split partials loaded together by one thread
+constexpr size_t kCmbWBudget = 128 << 10;  // shared memory for staged W_UV rows
 
 constexpr int kMinBlocks = 128;  // about one block per SM
 // Sequences per absorb / combine block: as many as the row tile holds (they share the
@@ -40,9 +41,16 @@ __host__ __device__ inline int absorb_seqs(const DecodeParams& p) {
   const int fill = max(1, p.B * p.n_kv * ((p.d_c + ABS_C - 1) / ABS_C) / kMinBlocks);
   return min(max(1, ABS_R / (p.g + 1)), fill);
 }
+// Combine: as many sequences as the row tile holds, but few enough that about
+// kMinBlocks blocks run (one wave of one block per SM).
 __host__ __device__ inline int combine_seqs(const DecodeParams& p) {
-  const int fill = max(1, p.B * p.n_kv / kMinBlocks);
+  const int fill = max(1, (p.B * p.n_kv + kMinBlocks - 1) / kMinBlocks);
   return min(max(1, CMB_R / (p.g + 1)), fill);
+}
+// latent rows of W_UV staged at a time (all d_c rows when they fit the budget)
+__host__ __device__ inline int combine_kc(const DecodeParams& p, size_t esz) {
+  const int rows = (int)(kCmbWBudget / ((size_t)p.d_v * esz));
+  return rows >= p.d_c ? p.d_c : rows;
 }
 
 // q_abs[b, head, c] = sum_n W_UKV[c, h*(d_nope+d_v) + n] * q_nope[b, head, n] for the
@@ -70,37 +78,47 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int VEC = 16 / (int)sizeof(T);
   const int vrow = DN / VEC;
-  for (int e = tid; e < ABS_C * vrow; e += blockDim.x) {
-    const int cr = e % ABS_C, v = e / ABS_C;  // consecutive threads: consecutive latent rows (conflict-free stores)
-    float f[VEC];
-    if (cr < nrows) {
-      const uint4 x = *reinterpret_cast<const uint4*>(w + (long)(c0 + cr) * ncol + (long)h * (p.d_nope + p.d_v) + v * VEC);
-      const T* xe = reinterpret_cast<const T*>(&x);
+  // Staging: every thread issues all of its 16-byte loads (W_UK tile, then the query
+  // rows) before it converts and stores any, so the block waits for one round trip
+  // of global loads instead of one per piece. Consecutive threads take consecutive
+  // latent rows of W_UK (conflict-free transposed stores).
+  // pieces per thread for the widest head (d_nope = 128): W 128 rows, q 48 rows
+  constexpr int kWL = ABS_C * (128 / VEC) / 256, kQL = (ABS_R * (128 / VEC) + 255) / 256;
+  uint4 wl[kWL], ql[kQL];
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) f[i] = to_f(xe[i]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) f[i] = 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) wt[(v * VEC + i) * WT + cr] = f[i];
+  for (int u = 0; u < kWL; ++u) {
+    const int e = tid + u * 256, cr = e % ABS_C, v = e / ABS_C;
+    wl[u] = make_uint4(0, 0, 0, 0);
+    if (v < vrow && cr < nrows)
+      wl[u] = *reinterpret_cast<const uint4*>(w + (long)(c0 + cr) * ncol + (long)h * (p.d_nope + p.d_v) + v * VEC);
   }
-  for (int e = tid; e < ABS_R * vrow; e += blockDim.x) {
-    const int r = e / vrow, v = e % vrow;
-    float f[VEC];
+#pragma unroll
+  for (int u = 0; u < kQL; ++u) {
+    const int e = tid + u * 256, r = e / vrow, v = e % vrow;
+    ql[u] = make_uint4(0, 0, 0, 0);
     if (r < R) {
-      const int bl = r / G1, u = r % G1;
-      const int head = u < p.g ? h * p.g + u : n_S + h;
-      const uint4 x = *reinterpret_cast<const uint4*>(q + ((long)(b0 + bl) * H_q + head) * dqk + v * VEC);
-      const T* xe = reinterpret_cast<const T*>(&x);
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) f[i] = to_f(xe[i]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) f[i] = 0.f;
+      const int bl = r / G1, uu = r % G1;
+      const int head = uu < p.g ? h * p.g + uu : n_S + h;
+      ql[u] = *reinterpret_cast<const uint4*>(q + ((long)(b0 + bl) * H_q + head) * dqk + v * VEC);
     }
+  }
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) qs[r * DN + v * VEC + i] = f[i];
+  for (int u = 0; u < kWL; ++u) {
+    const int e = tid + u * 256, cr = e % ABS_C, v = e / ABS_C;
+    if (v < vrow) {
+      const T* xe = reinterpret_cast<const T*>(&wl[u]);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) wt[(v * VEC + i) * WT + cr] = to_f(xe[i]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kQL; ++u) {
+    const int e = tid + u * 256, r = e / vrow, v = e % vrow;
+    if (r < ABS_R) {
+      const T* xe = reinterpret_cast<const T*>(&ql[u]);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) qs[r * DN + v * VEC + i] = to_f(xe[i]);
+    }
   }
   __syncthreads();
   // thread: latent rows 4*lane .. +3, query rows 6*warp .. +5
@@ -301,57 +319,64 @@ __global__ void __launch_bounds__(256) decode_split_simt_kernel(DecodeParams p) 
 //   O_lat = sum_s w_s O_s with w_s = exp2(m_s - M) / sum_s' exp2(m_s' - M) l_s'
 //   (log-sum-exp merge of the split-KV partials),
 //   H = O_lat W_UV, D = H_S - sigmoid(lam) H_N, Y = sigmoid(G) D.
-// W_UV is staged CMB_KC latent rows at a time; every thread accumulates a 4 (query
-// rows) x 16-byte-vector (value columns) tile of H over one K-slice of each block.
+// Everything that does not depend on the split kernel (the first W_UV rows, lambda
+// and the gate logits of the block's rows) is loaded before the block waits for it;
+// after the wait come one round trip for the merge weights and one for the partials.
 // `max_parts` bounds the partials of one sequence (the splits, or the ranges of one
-// head group on the tensor-core path).
+// head group on the tensor-core path); `kc` is the W_UV rows staged at a time.
 template <typename T>
-__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p, int max_parts) {
+__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p, int max_parts, int kc) {
   const int spb = combine_seqs(p);
   const int h = blockIdx.x, b0 = blockIdx.y * spb;
   const int nb = min(spb, p.B - b0);
   const int n_S = p.g * p.n_kv, G1 = p.g + 1, R = nb * G1, NP = max_parts;
   const int d_c = p.d_c, DV = p.d_v, ncol = p.n_kv * (p.d_nope + p.d_v);
-  extern __shared__ float sm[];
-  float* olat = sm;                              // [CMB_R][d_c]
-  float* hsm = olat + CMB_R * d_c;               // [CMB_R][DV]
-  float* wgt = hsm + CMB_R * DV;                 // [CMB_R][NP] merge weights (scaled by 1 / denominator)
-  T* wch = reinterpret_cast<T*>(wgt + CMB_R * NP);  // 2 x [CMB_KC][DV] staged W_UV rows
-  float* red = reinterpret_cast<float*>(wch + 2 * CMB_KC * DV);  // [K-slices][CMB_R][DV] partial products
-  __shared__ long long rec0[CMB_R];              // first partial record of each row
-  __shared__ long long rec_step[CMB_R];          // record stride between consecutive partials of the row
+  extern __shared__ __align__(16) float sm[];
+  T* wsm = reinterpret_cast<T*>(sm);                              // [kc][DV] staged W_UV rows
+  float* hsm = sm;                                                // [CMB_R][DV] H (reuses wsm after the product)
+  float* olat = reinterpret_cast<float*>(wsm + (size_t)kc * DV);  // [CMB_R][d_c]
+  float* wgt = olat + CMB_R * d_c;                                // [CMB_R][NP] merge weights
+  T* gsm = reinterpret_cast<T*>(wgt + CMB_R * NP);                // [CMB_R][DV] gate logits (signal rows)
+  __shared__ float lsm[CMB_R];                                    // sigmoid(lambda) (signal rows)
+  __shared__ long long rec0[CMB_R];                               // first partial record of each row
+  __shared__ long long rec_step[CMB_R];                           // record stride between a row's partials
   __shared__ int n_parts[CMB_R];
   const T* w = reinterpret_cast<const T*>(p.w_ukv);
   const T* gate = reinterpret_cast<const T*>(p.gate);
   T* out = reinterpret_cast<T*>(p.out);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   auto head_of_row = [&](int r) { const int u = r % G1; return u < p.g ? h * p.g + u : n_S + h; };
-  // W_UV rows [k0, k0 + CMB_KC) of this KV group: register-staged, so that the loads of
-  // the next rows overlap the products on the current ones
   constexpr int VEC = 16 / (int)sizeof(T);
-  const int per_row = DV / VEC;
-  const int n_w = CMB_KC * per_row;  // 16-byte pieces per staged block
-  constexpr int kWPT = 8;            // pieces per thread (n_w <= 256 * kWPT for every supported width)
-  uint4 wreg[kWPT];
-  auto load_w = [&](int k0) {
+  const int per_row = DV / VEC;  // 16-byte pieces of one W_UV row
+  // W_UV rows [k0, k0 + kc) of this KV group into wsm: all loads issued, then stored
+  auto stage_w = [&](int k0) {
+    const int n = min(kc, d_c - k0) * per_row;
+    for (int e0 = 0; e0 < n; e0 += 256 * 8) {
+      uint4 v[8];
 #pragma unroll
-    for (int q = 0; q < kWPT; ++q) {
-      const int e = tid + q * 256;
-      if (e < n_w) {
-        const int c = e / per_row, v = e % per_row;
-        wreg[q] = *reinterpret_cast<const uint4*>(w + (long)(k0 + c) * ncol + (long)h * (p.d_nope + DV) + p.d_nope +
-                                                  v * VEC);
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + tid + 256 * u;
+        if (e < n)
+          v[u] = *reinterpret_cast<const uint4*>(w + (long)(k0 + e / per_row) * ncol + (long)h * (p.d_nope + DV) +
+                                                 p.d_nope + (e % per_row) * VEC);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + tid + 256 * u;
+        if (e < n) reinterpret_cast<uint4*>(wsm)[e] = v[u];
       }
     }
   };
-  auto store_w = [&](T* dst) {
-#pragma unroll
-    for (int q = 0; q < kWPT; ++q) {
-      const int e = tid + q * 256;
-      if (e < n_w) *reinterpret_cast<uint4*>(dst + (e / per_row) * DV + (e % per_row) * VEC) = wreg[q];
+  stage_w(0);
+  // lambda and the gate logits of the block's signal rows (inputs of the caller)
+  for (int e = tid; e < R * DV / VEC; e += 256) {
+    const int r = e / (DV / VEC), v = e % (DV / VEC), u = r % G1;
+    if (u < p.g) {
+      const int b = b0 + r / G1, sh = h * p.g + u;
+      reinterpret_cast<uint4*>(gsm)[e] = *reinterpret_cast<const uint4*>(gate + ((long)b * n_S + sh) * DV + v * VEC);
     }
-  };
-  load_w(0);
+  }
+  if (tid < R && tid % G1 < p.g) lsm[tid] = sigmoidf_(p.lam[(long)(b0 + tid / G1) * n_S + h * p.g + tid % G1]);
   // the partials (and their index on the tensor-core path) come from the split kernel
   sm100::grid_dep_wait();
 
@@ -396,10 +421,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p, int
     for (int sp = lane; sp < np; sp += 32) wgt[r * NP + sp] *= inv;
   }
   __syncthreads();
-  // ---- O_lat rows (float4 over the latent dimension); rows R .. CMB_R-1 are zero
+  // ---- O_lat rows (float4 over the latent dimension)
   const int c4 = d_c / 4;
-  for (int e = R * c4 + tid; e < CMB_R * c4; e += blockDim.x)
-    reinterpret_cast<float4*>(olat)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = tid; e < R * c4; e += blockDim.x) {
     const int r = e / c4, v = e % c4;
     const int np = n_parts[r];
@@ -424,73 +447,64 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p, int
     }
     reinterpret_cast<float4*>(olat + r * d_c)[v] = acc;
   }
-  // ---- H = O_lat W_UV. Thread (K-slice sl, rows 4 rg .. 4 rg + 3, columns VEC cg ..):
-  // per step it reads four W_UV rows as 16-byte vectors and O_lat as float4 along the
-  // latent dimension, so each shared load feeds 4 x VEC (or 4 x 4) FMAs
-  const int groups = DV / VEC;              // 16-byte column vectors per W_UV row
-  const int rgc = R <= 4 ? 1 : (R <= 8 ? 2 : 4);  // groups of 4 rows covering the R query rows
-  const int RT = 4 * rgc;                   // rows of the tile (R rounded up)
-  const int tps = groups * rgc;             // threads per K-slice
-  const int n_sl = min(256 / tps, CMB_KC / 4);  // K-slices (each at least 4 latent rows per block)
-  const int ks = CMB_KC / n_sl;             // latent rows per slice and staged block (multiple of 4)
-  const bool active = tid < n_sl * tps;
-  const int sl = tid / tps, rg = (tid % tps) / groups, cg = tid % groups;
-  float acc[4][VEC];
+  __syncthreads();
+  // ---- H = O_lat W_UV: thread (column group cg of 8 value columns, row slot rs) keeps
+  // rows rs and rs + n_rs over the whole latent dimension
+  const int ncg = DV / 8, n_rs = 256 / ncg;
+  const int cg = tid % ncg, rs = tid / ncg;
+  const int r0 = rs, r1 = rs + n_rs;
+  float acc0[8], acc1[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int c = 0; c < 8; ++c) acc0[c] = acc1[c] = 0.f;
+  for (int k0 = 0; k0 < d_c; k0 += kc) {
+    if (k0 > 0) {
+      __syncthreads();  // the previous rows are consumed
+      stage_w(k0);
+    }
+    __syncthreads();
+    const int nk = min(kc, d_c - k0);
+    if (r0 < R) {
+      const float* o0 = olat + r0 * d_c + k0;
+      const float* o1 = olat + (r1 < R ? r1 : r0) * d_c + k0;
+#pragma unroll 4
+      for (int k = 0; k < nk; ++k) {
+        float wv[8];
+        const T* wr = wsm + (size_t)k * DV + cg * 8;
+        if constexpr (sizeof(T) == 2) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(wr);
+          const T* xe = reinterpret_cast<const T*>(&raw);
 #pragma unroll
-    for (int j = 0; j < VEC; ++j) acc[i][j] = 0.f;
-  store_w(wch);
-  __syncthreads();  // O_lat and the first W_UV rows are in shared memory
-  for (int k0 = 0, it = 0; k0 < d_c; k0 += CMB_KC, ++it) {
-    const T* wcur = wch + (it & 1) * (CMB_KC * DV);
-    if (k0 + CMB_KC < d_c) load_w(k0 + CMB_KC);
-    for (int kk = 0; active && kk < ks; kk += 4) {
-      const int kr = sl * ks + kk;  // row of the staged block
-      float wv[4][VEC];
+          for (int c = 0; c < 8; ++c) wv[c] = to_f(xe[c]);
+        } else {
+          const float4 a0 = reinterpret_cast<const float4*>(wr)[0], a1 = reinterpret_cast<const float4*>(wr)[1];
+          wv[0] = a0.x; wv[1] = a0.y; wv[2] = a0.z; wv[3] = a0.w;
+          wv[4] = a1.x; wv[5] = a1.y; wv[6] = a1.z; wv[7] = a1.w;
+        }
+        const float x0 = o0[k], x1 = o1[k];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(wcur + (kr + q) * DV + cg * VEC);
-        const T* xe = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) wv[q][j] = to_f(xe[j]);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 ov = *reinterpret_cast<const float4*>(olat + (4 * rg + i) * d_c + k0 + kr);
-#pragma unroll
-        for (int j = 0; j < VEC; ++j)
-          acc[i][j] = fmaf(ov.w, wv[3][j], fmaf(ov.z, wv[2][j], fmaf(ov.y, wv[1][j], fmaf(ov.x, wv[0][j], acc[i][j]))));
+        for (int c = 0; c < 8; ++c) {
+          acc0[c] = fmaf(x0, wv[c], acc0[c]);
+          acc1[c] = fmaf(x1, wv[c], acc1[c]);
+        }
       }
     }
-    if (k0 + CMB_KC < d_c) store_w(wch + ((it + 1) & 1) * (CMB_KC * DV));
-    __syncthreads();  // next rows staged; the buffer just read may be refilled
   }
-  if (active) {
+  __syncthreads();  // W_UV is consumed: its space takes H
+  if (r0 < R) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < VEC; j += 4)
-        *reinterpret_cast<float4*>(red + (sl * RT + 4 * rg + i) * DV + cg * VEC + j) =
-            make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
+    for (int c = 0; c < 8; ++c) hsm[r0 * DV + cg * 8 + c] = acc0[c];
   }
-  __syncthreads();
-  // the slices' partial products, added in slice order (deterministic)
-  for (int e = tid; e < R * DV; e += blockDim.x) {
-    const int r = e / DV, c = e % DV;
-    float v = 0.f;
-    for (int q = 0; q < n_sl; ++q) v += red[(q * RT + r) * DV + c];
-    hsm[r * DV + c] = v;
+  if (r1 < R) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) hsm[r1 * DV + cg * 8 + c] = acc1[c];
   }
   __syncthreads();
   // ---- differential and gate
   for (int e = tid; e < nb * p.g * DV; e += blockDim.x) {
     const int bl = e / (p.g * DV), u = (e / DV) % p.g, nn = e % DV;
-    const int b = b0 + bl, sh = h * p.g + u;
-    const float lam = sigmoidf_(p.lam[(long)b * n_S + sh]);
-    const long idx = ((long)b * n_S + sh) * DV + nn;
-    const float d = hsm[(bl * G1 + u) * DV + nn] - lam * hsm[(bl * G1 + p.g) * DV + nn];
-    out[idx] = from_f<T>(sigmoidf_(to_f(gate[idx])) * d);
+    const int b = b0 + bl, sh = h * p.g + u, r = bl * G1 + u;
+    const float d = hsm[r * DV + nn] - lsm[r] * hsm[(bl * G1 + p.g) * DV + nn];
+    out[((long)b * n_S + sh) * DV + nn] = from_f<T>(sigmoidf_(to_f(gsm[r * DV + nn])) * d);
   }
 }
 
@@ -554,17 +568,20 @@ cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStre
   const size_t esz = dt == GDLA_BF16 ? 2 : 4;
   const int spb = combine_seqs(p);
   const int max_parts = p.tc ? p.n_ranges : p.n_splits;
-  // O_lat, H, merge weights, two staged W_UV blocks, and the K-slices' partial products
-  // (n_slices x CMB_R x d_v = 1024 x (16 / esz) floats)
-  const size_t smem = sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * p.d_v + (size_t)CMB_R * max_parts) +
-                      esz * 2 * (size_t)CMB_KC * p.d_v + sizeof(float) * 1024 * (16 / esz);
+  const int kc = combine_kc(p, esz);
+  // staged W_UV rows (at least the DV x CMB_R floats of H, which reuse them), O_lat,
+  // merge weights, gate logits
+  const size_t w_bytes = (size_t)kc * p.d_v * esz > (size_t)CMB_R * p.d_v * 4 ? (size_t)kc * p.d_v * esz
+                                                                               : (size_t)CMB_R * p.d_v * 4;
+  const size_t smem = w_bytes + sizeof(float) * ((size_t)CMB_R * p.d_c + (size_t)CMB_R * max_parts) +
+                      esz * (size_t)CMB_R * p.d_v;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((unsigned)p.n_kv, (unsigned)((p.B + spb - 1) / spb));
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  // programmatic dependent launch: the blocks stage their first W_UV rows while the
-  // split kernel finishes, and wait for it before reading its partials
+  // programmatic dependent launch: the blocks stage W_UV and their gate logits while
+  // the split kernel finishes, and wait for it before reading its partials
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -574,11 +591,11 @@ cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStre
   if (dt == GDLA_BF16) {
     auto k = decode_combine_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k, p, max_parts);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k, p, max_parts, kc);
   } else {
     auto k = decode_combine_kernel<float>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k, p, max_parts);
+    if (e == cudaSuccess) e = cudaLaunchKernelEx(&cfg, k, p, max_parts, kc);
   }
   return e;
 }

@@ -166,8 +166,8 @@ def rope_freqs(d_R: int, base: float = DEFAULT_ROPE_BASE) -> np.ndarray:
 
 def yarn_inv_freq(d_R: int, factor: float, original_max_pos: float, base: float = DEFAULT_ROPE_BASE,
                   beta_fast: float = 32.0, beta_slow: float = 1.0) -> np.ndarray:
-    """RoPE frequencies rescaled by YaRN ("Context Extension via YaRN", page 1,
-    section 2): kept where the wavelength is below original_max_pos/beta_fast,
+    """RoPE frequencies rescaled by YaRN ("Open-Source Frontier Models: Architecture and Benchmarks of Rnj-1 and Motif-2",
+    section 2, the Scale(i) equation): kept where the wavelength is below original_max_pos/beta_fast,
     divided by ``factor`` above original_max_pos/beta_slow, blended linearly in the
     wavelength in between (computed by the C oracle)."""
     out = np.empty(d_R // 2)

@@ -143,7 +143,7 @@ void gdla_oracle_rope(const double* x, long pos, int d_R, double base, double* y
   rope_apply(x, pos, d_R, base, 0, y);
 }
 
-/* ---- YaRN frequency scaling ("Context Extension via YaRN", page 1, section 2) ----
+/* ---- YaRN frequency scaling ("Open-Source Frontier Models: Architecture and Benchmarks of Rnj-1 and Motif-2", section 2) ----
  * Extending the context by a factor s = L_new / L_native: with the wavelength of
  * frequency k, lambda_k = 2 pi / theta_k, frequencies whose wavelength is below
  * orig/beta_fast are kept (scale 1), those above orig/beta_slow are interpolated
