@@ -26,8 +26,11 @@
 //   warp 0      TMA producer: TT-token cache tiles (9 boxes: 8 latent + 1 rotary)
 //               in a STAGES-deep ring, each tile also prefetched into L2 PF
 //               tiles ahead of its ring load;
-//   warp 1      issues the score MMAs (one lane); warp 2 the value MMAs;
-//   warp 3      loads the query operand of each sequence (one bulk copy);
+//   warps 1, 3  issue the score MMAs (one lane each), each over one half of K into
+//               its own accumulator (the softmax adds the two): the issue time of an
+//               MMA instruction, not the tensor pipe, bounds one issuing thread;
+//               warp 3 also loads the query operand of each sequence (one bulk copy);
+//   warp 2      issues the value MMAs;
 //   warps 4-7   softmax over S^T: each warp's lanes 0-15 own 16 tokens (the M = 64
 //               accumulator layout) and lanes 16-31 take the upper 24 heads of
 //               the same tokens; P^T is written token-major (16-byte stores).
@@ -53,8 +56,11 @@ constexpr int NPV = 64;                            // N of the value MMA: heads 
 constexpr int QT_BYTES = kDtcImageBytes;           // 54 KB
 constexpr int DTHREADS = 256;
 constexpr float kThr = 8.0f;
-constexpr uint32_t COL_ST = 0;    // S^T buffers at [0, 48) and [64, 112)
-constexpr uint32_t COL_OT = 128;  // O^T M-tile mt at 128 + 64 mt
+// S^T of tile k: two partial sums over the two halves of K (issued by two warps), in
+// buffer k & 1: half hk at COL_ST + 64 (2 (k & 1) + hk), 48 columns each
+constexpr uint32_t COL_ST = 0;
+constexpr uint32_t COL_OT = 256;  // O^T M-tile mt at 256 + 64 mt
+constexpr int KSPLIT = NBOX * 2;  // K-steps (of 16) of the first score warp; the second takes the rest
 static_assert(NQ == 48, "the softmax lane split assumes 48 heads (3 x 16-byte P^T chunks per lane half)");
 
 template <int TT, int STAGES, int PST>
@@ -261,14 +267,14 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
       mbar_init(smem_u32(&sh.empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sh.s_full[i]), 1);
+      mbar_init(smem_u32(&sh.s_full[i]), 2);  // one commit per score warp
       mbar_init(smem_u32(&sh.p_full[i]), 128);
     }
     for (int i = 0; i < PST; ++i) mbar_init(smem_u32(&sh.p_free[i]), 1);
     mbar_init(smem_u32(&sh.q_full), 1);
-    mbar_init(smem_u32(&sh.q_free), 1);
+    mbar_init(smem_u32(&sh.q_free), 2);
     mbar_init(smem_u32(&sh.seg_done), 1);
-    mbar_init(smem_u32(&sh.mma_done), 2);  // one commit per MMA-issuing warp
+    mbar_init(smem_u32(&sh.mma_done), 3);  // one commit per MMA-issuing warp
     fence_mbar_init();
     abort_flag = 0;
     prefetch_tmap(&tmC);
@@ -326,34 +332,10 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
         for (int q = (k > STAGES ? k - STAGES : 0); q < k; ++q)
           mbar_wait(smem_u32(&sh.full[q % STAGES]), (q / STAGES) & 1, nullptr, 0);
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------- query operand loader
-    if (lane == 0) {
-      Walker<TT> w;
-      w.init(a, b0, p0);
-      int seg = 0;
-      bool ok = true;
-      for (long long t = start; t < end && ok && !abort_flag; t = w.pb + w.st.n, ++seg) {
-        w.seek(t);
-        if (seg == 0)
-          grid_dep_wait();  // the absorb kernel has written the query images
-        else
-          ok = mbar_wait(smem_u32(&sh.q_free), (seg - 1) & 1, a.status, 331, &abort_flag);
-        if (!ok) break;
-        const uint32_t bar = smem_u32(&sh.q_full);
-        mbar_expect_tx(bar, QT_BYTES);
-        bulk_load(smem_u32(qt), a.qimg + ((long long)w.b * a.n_hg + hg) * QT_BYTES, QT_BYTES, bar);
-        // the copy must land before the next segment may overwrite it (and before exit)
-        if (!mbar_wait(bar, seg & 1, a.status, 332, &abort_flag)) {
-          mbar_wait(bar, seg & 1, nullptr, 0);
-          ok = false;
-        }
-      }
-      if (!ok) abort_flag = 1;
-    }
-  } else if (warp == 1 || warp == 2) {
-    // warp 1 issues the score MMAs, warp 2 the value MMAs: neither waits behind
-    // the other's instructions
+  } else if (warp >= 1 && warp <= 3) {
+    // warps 1 and 3 issue the score MMAs (K-steps [0, KSPLIT) and [KSPLIT, 36)), warp 2
+    // the value MMAs: none waits behind another's instructions. Warp 3 also loads each
+    // sequence's query operand, once the previous one's score MMAs are done.
     if (lane == 0) {
       constexpr uint32_t id1 = idesc_bf16_f32(64, NQ, false, false);
       constexpr uint32_t id2 = idesc_bf16_f32(128, NPV, true, true);
@@ -362,14 +344,29 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
       w.init(a, b0, p0);
       int seg = -1;
       bool ok = true;
-      if (warp == 1) {
+      if (warp != 2) {
+        const int hk = warp == 1 ? 0 : 1;
+        const int kk0 = hk ? KSPLIT : 0, kk1 = hk ? NBOX * 4 : KSPLIT;
         for (int k = 0; k < n_tiles && ok; ++k) {
           const long long t = start + k;
           w.seek(t);
           const bool first = (k == 0) || t == w.pb, last = (k == n_tiles - 1) || t == w.pb + w.st.n - 1;
           if (first) {
             ++seg;
-            ok = mbar_wait(smem_u32(&sh.q_full), seg & 1, a.status, 310, &abort_flag);
+            if (hk) {
+              // the query operand of this sequence: after the absorb kernel (first), or
+              // once both score warps are done with the previous sequence's
+              if (seg == 0)
+                grid_dep_wait();
+              else
+                ok = mbar_wait(smem_u32(&sh.q_free), (seg - 1) & 1, a.status, 331, &abort_flag);
+              if (ok) {
+                const uint32_t bar = smem_u32(&sh.q_full);
+                mbar_expect_tx(bar, QT_BYTES);
+                bulk_load(smem_u32(qt), a.qimg + ((long long)w.b * a.n_hg + hg) * QT_BYTES, QT_BYTES, bar);
+              }
+            }
+            if (ok) ok = mbar_wait(smem_u32(&sh.q_full), seg & 1, a.status, 310, &abort_flag);
           }
           if (ok) ok = mbar_wait(smem_u32(&sh.full[k % STAGES]), (k / STAGES) & 1, a.status, 311, &abort_flag);
           // S^T buffer k & 1 was last read by the softmax of tile k-2
@@ -378,14 +375,19 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
           if (!ok) break;
           tc_fence_after();
           const uint64_t c0 = sdesc_sw128(smem_u32(tiles + (k % STAGES) * Lay::TILE), 16, 1024);
-#pragma unroll
-          for (int kk = 0; kk < NBOX * 4; ++kk) {
+          const uint32_t dcol = tmem + COL_ST + 64 * (2 * (k & 1) + hk);
+#pragma unroll 6
+          for (int kk = kk0; kk < kk1; ++kk) {
             const uint32_t off = (kk & 3) * 32;
-            mma_ss(tmem + COL_ST + 64 * (k & 1), c0 + (((kk >> 2) * Lay::BOX + off) >> 4),
-                   qd0 + (((kk >> 2) * (NQ * 128) + off) >> 4), id1, kk > 0);
+            mma_ss(dcol, c0 + (((kk >> 2) * Lay::BOX + off) >> 4), qd0 + (((kk >> 2) * (NQ * 128) + off) >> 4), id1,
+                   kk > kk0);
           }
           mma_commit(smem_u32(&sh.s_full[k & 1]));
           if (last) mma_commit(smem_u32(&sh.q_free));  // the query operand may be replaced
+        }
+        if (!ok && hk) {
+          // a query copy in flight lands before the CTA may exit
+          if (seg >= 0) mbar_wait(smem_u32(&sh.q_full), seg & 1, nullptr, 0);
         }
       } else {
         for (int k = 0; k < n_tiles && ok; ++k) {
@@ -452,11 +454,16 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
       bool exceed = false;
       if (w_ok) {
         tc_fence_after();
-        uint32_t xr[NQ];
-        const uint32_t tS = tmem + lane_base + COL_ST + 64 * (k & 1);
+        uint32_t xr[NQ], xr2[NQ];
+        const uint32_t tS = tmem + lane_base + COL_ST + 64 * (2 * (k & 1));
         tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&xr[0]));
         tmem_ld16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&xr[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&xr2[0]));
+        tmem_ld16(tS + 96, *reinterpret_cast<uint32_t(*)[16]>(&xr2[32]));
         tmem_wait_ld();
+        // the two K halves of the scores
+#pragma unroll
+        for (int h = 0; h < NQ; ++h) xr[h] = __float_as_uint(__uint_as_float(xr[h]) + __uint_as_float(xr2[h]));
         const int j = (w.st.jt0 + (int)(t - w.pb)) * TT + tok_local;
         const bool valid = tok_real && j >= w.st.lo && j < w.st.Tb;
 #pragma unroll
@@ -608,6 +615,472 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- absorb
+// The absorbed query of the tensor-core path, on the tensor cores: for KV group h
+// and a tile of 128 query rows (row = (sequence b, head u of the group)),
+//   Qabs[rows x 256 latent dims] = Q_nope[rows x 128] . W_UK,h^T[128 x 256]
+// (half nh of the 512 latent dims per block), scaled by tau*log2(e) and written as
+// bf16 straight into the split kernel's query images; the nh = 0 blocks also rotate
+// the rotary query parts (RoPE at position seqlen-1) into the images, and the
+// blocks of KV group 0 zero the image rows of padding heads.
+struct AbsorbTcArgs {
+  int B, T_max, n_kv, g, H_q, n_hg, hpc, rope_max_pos;
+  float isc;
+  const __nv_bfloat16* q;  // [B, H_q, 192]
+  const int* seqlens;
+  const float* cos_tab;
+  const float* sin_tab;
+  uint8_t* qimg;
+  int* status;
+};
+
+namespace dtc {
+constexpr int AB_M = 128, AB_N = 256, AB_K = 128;
+constexpr int AB_A = AB_M * AB_K * 2;   // 32 KB: two 64-dim chunks of [128 rows x 128 B]
+constexpr int AB_B = AB_N * AB_K * 2;   // 64 KB: two 64-dim chunks of [256 latent rows x 128 B]
+constexpr int AB_SMEM = AB_A + AB_B + 64;
+}  // namespace dtc
+
+__global__ void __launch_bounds__(256, 1)
+    decode_absorb_tc_kernel(const __grid_constant__ CUtensorMap tmW, const AbsorbTcArgs a) {
+  using namespace sm100;
+  using namespace dtc;
+  // the split kernel may start its set-up and first cache loads; it reads the
+  // query images only after this grid has completed
+  grid_dep_launch();
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* as = smem;
+  uint8_t* bs = smem + AB_A;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + AB_A + AB_B);  // [0] W landed, [1] MMAs done
+  __shared__ uint32_t tmem_slot;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) {
+      atomicCAS(a.status, 0, (int)GDLA_ERR_CUDA);
+      atomicCAS(a.status + 1, 0, 398);
+    }
+    return;
+  }
+  const int h = blockIdx.x, nh = blockIdx.z;
+  const int G1 = a.g + 1, n_S = a.g * a.n_kv;
+  const int rows = a.B * G1;
+  const int r0 = blockIdx.y * AB_M;
+  if (tid == 0) {
+    mbar_init(smem_u32(&bar[0]), 1);
+    mbar_init(smem_u32(&bar[1]), 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmW);
+    mbar_expect_tx(smem_u32(&bar[0]), AB_B);
+    for (int kc = 0; kc < 2; ++kc) tma_load_2d(smem_u32(bs + kc * (AB_B / 2)), &tmW, smem_u32(&bar[0]),
+                                               h * 256 + kc * 64, nh * AB_N);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), AB_N);
+    tmem_relinquish();
+  }
+  auto head_of = [&](int u) { return u < a.g ? h * a.g + u : n_S + h; };
+  // Q_nope of the tile's rows, K-major with the 128-byte swizzle: each thread issues all
+  // of its 16-byte loads (pieces of a row on consecutive threads) before it stores any
+  constexpr int kPieces = AB_M * 16 / 256;
+  uint4 qv[kPieces];
+#pragma unroll
+  for (int u = 0; u < kPieces; ++u) {
+    const int e = tid + 256 * u, r = e >> 4, pc = e & 15, R = r0 + r;
+    qv[u] = make_uint4(0, 0, 0, 0);
+    if (R < rows) {
+      const int b = R / G1, head = head_of(R % G1);
+      qv[u] = *reinterpret_cast<const uint4*>(a.q + ((long)b * a.H_q + head) * 192 + pc * 8);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kPieces; ++u) {
+    const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+    const int kc = pc >> 3, c = pc & 7;
+    *reinterpret_cast<uint4*>(as + kc * (AB_A / 2) + r * 128 + ((c ^ (r & 7)) << 4)) = qv[u];
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 32) {
+    const bool ok = mbar_wait(smem_u32(&bar[0]), 0, a.status, 341);
+    if (ok) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16_f32(AB_M, AB_N, false, false);
+#pragma unroll
+      for (int kk = 0; kk < AB_K / 16; ++kk) {
+        const uint32_t off = (uint32_t)((kk & 3) * 32);
+        mma_ss(tmem, sdesc_sw128(smem_u32(as + (kk >> 2) * (AB_A / 2)) + off, 16, 1024),
+               sdesc_sw128(smem_u32(bs + (kk >> 2) * (AB_B / 2)) + off, 16, 1024), idesc, kk > 0);
+      }
+    }
+    mma_commit(smem_u32(&bar[1]));  // (also when the W load failed: the epilogue then ends)
+  }
+  __syncwarp();
+  const bool done = mbar_wait(smem_u32(&bar[1]), 0, a.status, 342);
+  tc_fence_after();
+  const int q4 = warp & 3;              // TMEM lane quadrant; warps q4 and q4 + 4 split the columns
+  const int R = r0 + q4 * 32 + lane;    // this thread's row (TMEM lane)
+  const bool real = done && R < rows && !earlier_failure(a.status);
+  int b = 0, head = 0, hgi = 0, lh = 0;
+  uint8_t* img = nullptr;
+  if (R < rows) {
+    b = R / G1;
+    head = head_of(R % G1);
+    hgi = head / a.hpc;
+    lh = head - hgi * a.hpc;
+    img = a.qimg + ((long)b * a.n_hg + hgi) * kDtcImageBytes;
+  }
+#pragma unroll 1
+  for (int ch = (warp >> 2) * (AB_N / 64); ch < ((warp >> 2) + 1) * (AB_N / 64); ++ch) {
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + ch * 32, v);
+    tmem_wait_ld();
+    if (real) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 o;
+        o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * a.isc, __uint_as_float(v[8 * q + 1]) * a.isc);
+        o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * a.isc, __uint_as_float(v[8 * q + 3]) * a.isc);
+        o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * a.isc, __uint_as_float(v[8 * q + 5]) * a.isc);
+        o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * a.isc, __uint_as_float(v[8 * q + 7]) * a.isc);
+        *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, nh * AB_N + ch * 32 + q * 8)) = o;
+      }
+    }
+  }
+  if (real && nh == 0 && warp < 4) {
+    // RoPE of the rotary query part at position seqlen-1 (a length outside [1, T_max]
+    // is clamped; the split kernel reports it)
+    const int pos = min(max(__ldg(a.seqlens + b), 1), a.T_max) - 1;
+    const __nv_bfloat16* qr = a.q + ((long)b * a.H_q + head) * 192 + 128;
+    const float* cs = a.cos_tab + (long)pos * 32;
+    const float* sn = a.sin_tab + (long)pos * 32;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {  // pairs (k, k + 32) for k = 8c .. 8c + 7
+      const uint4 xl = *reinterpret_cast<const uint4*>(qr + 8 * c);
+      const uint4 xh = *reinterpret_cast<const uint4*>(qr + 32 + 8 * c);
+      const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&xl);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&xh);
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x1 = __bfloat1622float2(l2[e]), x2 = __bfloat1622float2(h2[e]);
+        const int k = 8 * c + 2 * e;
+        const float c0 = cs[k], s0 = sn[k], c1 = cs[k + 1], s1 = sn[k + 1];
+        lo[e] = pack_bf16x2((x1.x * c0 - x2.x * s0) * a.isc, (x1.y * c1 - x2.y * s1) * a.isc);
+        hi[e] = pack_bf16x2((x2.x * c0 + x1.x * s0) * a.isc, (x2.y * c1 + x1.y * s1) * a.isc);
+      }
+      *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, 512 + 8 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, 512 + 32 + 8 * c)) =
+          make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+  }
+  // image rows of padding heads (beyond each head group's heads) are zero: the blocks of
+  // KV group 0 clear them for the sequences whose first row falls in their tile
+  if (h == 0 && nh == 0) {
+    const int b_lo = (r0 + G1 - 1) / G1, b_hi = min(a.B, (r0 + AB_M + G1 - 1) / G1);
+    for (int bb = b_lo; bb < b_hi; ++bb)
+      for (int hg2 = 0; hg2 < a.n_hg; ++hg2) {
+        const int nhd = min(a.hpc, a.H_q - hg2 * a.hpc);
+        uint8_t* im = a.qimg + ((long)bb * a.n_hg + hg2) * kDtcImageBytes;
+        for (int e = tid; e < (kDtcHeads - nhd) * 72; e += 256) {
+          const int l2 = nhd + e / 72, bx = (e % 72) / 8, c = e % 8;
+          *reinterpret_cast<uint4*>(im + bx * (kDtcHeads * 128) + l2 * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, AB_N);
+}
+
+cudaError_t launch_decode_absorb_tc(const DecodeParams& p, cudaStream_t s) {
+  CUtensorMap tw;
+  const int ncol = p.n_kv * (p.d_nope + p.d_v);
+  const uint64_t dims[2] = {(uint64_t)ncol, (uint64_t)p.d_c}, str[1] = {(uint64_t)ncol * 2};
+  const uint32_t box[2] = {64, (uint32_t)dtc::AB_N};
+  if (!make_tmap_bf16(&tw, p.w_ukv, 2, dims, str, box)) return cudaErrorInvalidValue;
+  AbsorbTcArgs a{};
+  a.B = p.B; a.T_max = p.T_max; a.n_kv = p.n_kv; a.g = p.g; a.H_q = p.n_kv * (p.g + 1);
+  a.n_hg = p.n_hg; a.hpc = p.hpc; a.rope_max_pos = p.rope_max_pos; a.isc = p.scale * kLog2e;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(p.q); a.seqlens = p.seqlens;
+  a.cos_tab = p.cos_tab; a.sin_tab = p.sin_tab; a.qimg = p.qimg; a.status = p.status;
+  cudaError_t e = cudaFuncSetAttribute(decode_absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dtc::AB_SMEM);
+  if (e != cudaSuccess) return e;
+  const int rows = p.B * (p.g + 1);
+  dim3 grid((unsigned)p.n_kv, (unsigned)((rows + dtc::AB_M - 1) / dtc::AB_M), 2);
+  decode_absorb_tc_kernel<<<grid, 256, dtc::AB_SMEM, s>>>(tw, a);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- combine
+// The merge and output epilogue of the tensor-core path, with the W_UV product on
+// the tensor cores. Block = (KV group h, whole sequences: up to 64 query rows, row =
+// (sequence b, head u of the group)):
+//   O_lat = log-sum-exp merge of the partials of the ranges covering sequence b,
+//           written as the bf16 A operand (K-major, 512 latent dims);
+//   H[rows x 128] = O_lat[rows x 512] . W_UV,h[512 x 128]   (M = 64, N = 128, K = 512)
+//   D = H_S - sigmoid(lambda) H_N, Y = sigmoid(G) D.
+// W_UV,h (128 KB, MN-major) is loaded by TMA before the block waits for the split
+// kernel (programmatic dependent launch), so only the merge, 32 MMAs and the
+// epilogue follow the split kernel's end.
+struct CombineTcArgs {
+  int B, n_kv, g, H_q, n_hg, hpc, n_ranges, part_heads, spb;
+  const int2* seqinfo;
+  const float* part_o;
+  const float* part_ml;
+  const float* lam;
+  const __nv_bfloat16* gate;
+  __nv_bfloat16* out;
+  int* status;
+};
+
+namespace dtc {
+constexpr int CB_M = 64, CB_N = 128, CB_K = 512;
+constexpr int CB_A = CB_M * CB_K * 2;   // 64 KB: 8 chunks of [64 rows x 128 B]
+constexpr int CB_B = CB_K * CB_N * 2;   // 128 KB: 2 MN blocks of [512 K rows x 128 B]
+constexpr int CB_SMEM = CB_A + CB_B + 64;
+}  // namespace dtc
+
+__global__ void __launch_bounds__(512, 1)
+    decode_combine_tc_kernel(const __grid_constant__ CUtensorMap tmW, const CombineTcArgs a) {
+  using namespace sm100;
+  using namespace dtc;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* as = smem;                                   // O_lat (bf16); later H (fp32 [64 x 128])
+  uint8_t* bs = smem + CB_A;                            // W_UV,h
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + CB_A + CB_B);
+  __shared__ long long rec0[CB_M];
+  __shared__ int rec_step[CB_M], n_parts[CB_M];
+  __shared__ float row_max[CB_M], row_inv[CB_M];  // log-sum-exp merge: maximum, 1 / denominator
+  __shared__ uint32_t tmem_slot;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) {
+      atomicCAS(a.status, 0, (int)GDLA_ERR_CUDA);
+      atomicCAS(a.status + 1, 0, 397);
+    }
+    return;
+  }
+  const int h = blockIdx.x, G1 = a.g + 1, n_S = a.g * a.n_kv;
+  const int b0 = blockIdx.y * a.spb, nb = min(a.spb, a.B - b0), R = nb * G1;
+  if (tid == 0) {
+    mbar_init(smem_u32(&bar[0]), 1);
+    mbar_init(smem_u32(&bar[1]), 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmW);
+    // W_UV,h: MN block j (value dims 64j .. 64j+63) x K half kh (latent rows 256kh ..)
+    mbar_expect_tx(smem_u32(&bar[0]), CB_B);
+    for (int j = 0; j < 2; ++j)
+      for (int kh = 0; kh < 2; ++kh)
+        tma_load_2d(smem_u32(bs + j * (CB_B / 2) + kh * (CB_B / 4)), &tmW, smem_u32(&bar[0]),
+                    h * 256 + 128 + 64 * j, 256 * kh);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), CB_N);
+    tmem_relinquish();
+  }
+  auto head_of = [&](int u) { return u < a.g ? h * a.g + u : n_S + h; };
+  // the partials and their index come from the split kernel
+  grid_dep_wait();
+  if (tid < CB_M) {
+    const int r = tid;
+    if (r < R) {
+      const int b = b0 + r / G1, head = head_of(r % G1);
+      const int hgi = head / a.hpc, lh = head - hgi * a.hpc;
+      // the first and last range covering sequence b (clamped: a call whose split kernel
+      // gave up early still reads inside the records)
+      const int2 info = a.seqinfo[b];
+      const int x = min(max(info.x, 0), a.n_ranges - 1), y = min(max(info.y, x), a.n_ranges - 1);
+      rec0[r] = ((long long)(x + b) * a.n_hg + hgi) * a.part_heads + lh;
+      rec_step[r] = a.n_hg * a.part_heads;
+      n_parts[r] = y - x + 1;
+    } else {
+      n_parts[r] = 0;
+    }
+  }
+  __syncthreads();
+  // merge weights w_s = exp2(m_s - M) / sum_s' exp2(m_s' - M) l_s': one warp per row
+  // finds M and the denominator; the weights are recomputed where they are used
+  for (int r = warp; r < R; r += 16) {
+    const int np = n_parts[r];
+    const long long r0 = rec0[r], rs = rec_step[r];
+    float M = -INFINITY;
+    for (int sp = lane; sp < np; sp += 32) M = fmaxf(M, a.part_ml[(r0 + sp * rs) * 2]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+    for (int sp = lane; sp < np; sp += 32) {
+      const float m = a.part_ml[(r0 + sp * rs) * 2], l = a.part_ml[(r0 + sp * rs) * 2 + 1];
+      den += (m == -INFINITY) ? 0.f : exp2f(m - M) * l;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane == 0) {
+      row_max[r] = M;
+      row_inv[r] = den > 0.f ? 1.f / den : 0.f;
+    }
+  }
+  __syncthreads();
+  // O_lat rows into the A operand: 8 latent dims (one 16-byte chunk) per item; a thread
+  // loads two items' partials (up to kMB each) together, so that many loads are in flight
+  constexpr int kMB = 4;
+  for (int e0 = tid; e0 < CB_M * (CB_K / 8); e0 += 2 * 512) {
+    float acc[2][8];
+    int rr[2], cc8[2];
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int e = e0 + 512 * it;
+      rr[it] = e / (CB_K / 8);
+      cc8[it] = e % (CB_K / 8);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[it][q] = 0.f;
+    }
+    int np[2];
+#pragma unroll
+    for (int it = 0; it < 2; ++it) np[it] = rr[it] < R ? n_parts[rr[it]] : 0;
+    for (int sp0 = 0; sp0 < max(np[0], np[1]); sp0 += kMB) {
+      float4 x[2][kMB][2];
+      float mq[2][kMB];
+#pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        const int r = rr[it];
+        const float* src = a.part_o + (r < R ? rec0[r] : 0) * CB_K + cc8[it] * 8;
+        const float* mls = a.part_ml + (r < R ? rec0[r] : 0) * 2;
+        const long long st = r < R ? rec_step[r] : 0;
+#pragma unroll
+        for (int q = 0; q < kMB; ++q) {
+          if (sp0 + q < np[it]) {
+            x[it][q][0] = reinterpret_cast<const float4*>(src + (sp0 + q) * st * CB_K)[0];
+            x[it][q][1] = reinterpret_cast<const float4*>(src + (sp0 + q) * st * CB_K)[1];
+            mq[it][q] = mls[(sp0 + q) * st * 2];
+          } else {
+            x[it][q][0] = x[it][q][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            mq[it][q] = -INFINITY;
+          }
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        if (rr[it] >= R) continue;
+        const float M = row_max[rr[it]], inv = row_inv[rr[it]];
+#pragma unroll
+        for (int q = 0; q < kMB; ++q) {
+          const float wv = mq[it][q] == -INFINITY ? 0.f : exp2f(mq[it][q] - M) * inv;
+          acc[it][0] = fmaf(wv, x[it][q][0].x, acc[it][0]); acc[it][1] = fmaf(wv, x[it][q][0].y, acc[it][1]);
+          acc[it][2] = fmaf(wv, x[it][q][0].z, acc[it][2]); acc[it][3] = fmaf(wv, x[it][q][0].w, acc[it][3]);
+          acc[it][4] = fmaf(wv, x[it][q][1].x, acc[it][4]); acc[it][5] = fmaf(wv, x[it][q][1].y, acc[it][5]);
+          acc[it][6] = fmaf(wv, x[it][q][1].z, acc[it][6]); acc[it][7] = fmaf(wv, x[it][q][1].w, acc[it][7]);
+        }
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int r = rr[it], kc = cc8[it] >> 3, c = cc8[it] & 7;
+      *reinterpret_cast<uint4*>(as + kc * (CB_M * 128) + r * 128 + ((c ^ (r & 7)) << 4)) =
+          make_uint4(pack_bf16x2(acc[it][0], acc[it][1]), pack_bf16x2(acc[it][2], acc[it][3]),
+                     pack_bf16x2(acc[it][4], acc[it][5]), pack_bf16x2(acc[it][6], acc[it][7]));
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 32) {
+    const bool ok = mbar_wait(smem_u32(&bar[0]), 0, a.status, 351);
+    if (ok) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16_f32(CB_M, CB_N, false, true);
+#pragma unroll
+      for (int kk = 0; kk < CB_K / 16; ++kk) {
+        const uint64_t ad = sdesc_sw128(smem_u32(as + (kk >> 2) * (CB_M * 128)) + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(smem_u32(bs) + kk * 2048, CB_B / 2, 1024);
+        mma_ss(tmem, ad, bd, idesc, kk > 0);
+      }
+    }
+    mma_commit(smem_u32(&bar[1]));
+  }
+  __syncwarp();
+  const bool done = mbar_wait(smem_u32(&bar[1]), 0, a.status, 352);
+  tc_fence_after();
+  // H rows from TMEM (the M = 64 layout: row 16 q + l in lane l < 16 of quadrant q) into
+  // shared memory, where the signal rows find their noise row; warp w reads quadrant
+  // w % 4, columns 32 (w / 4) .. +31
+  float* hs = reinterpret_cast<float*>(as);  // [64][128]; the A operand is consumed
+  {
+    const int q4 = warp & 3, c = warp >> 2;
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + c * 32, v);
+    tmem_wait_ld();
+    if (lane < 16) {
+      float* dst = hs + (q4 * 16 + lane) * CB_N + c * 32;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(dst)[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+    }
+  }
+  __syncthreads();
+  // differential and gate: 8 value dims of one signal row per item
+  if (done && !earlier_failure(a.status)) {
+    for (int e = tid; e < nb * a.g * (CB_N / 8); e += 512) {
+      const int bl = e / (a.g * (CB_N / 8)), u = (e / (CB_N / 8)) % a.g, c8 = e % (CB_N / 8);
+      const int b = b0 + bl, sh = h * a.g + u;
+      const float lamv = 1.f / (1.f + __expf(-a.lam[(long)b * n_S + sh]));
+      const long idx = ((long)b * n_S + sh) * CB_N + c8 * 8;
+      const uint4 gv = *reinterpret_cast<const uint4*>(a.gate + idx);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+      const float* hsr = hs + (bl * G1 + u) * CB_N + c8 * 8;
+      const float* hnr = hs + (bl * G1 + a.g) * CB_N + c8 * 8;
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 gf = __bfloat1622float2(g2[q]);
+        const float d0 = hsr[2 * q] - lamv * hnr[2 * q], d1 = hsr[2 * q + 1] - lamv * hnr[2 * q + 1];
+        o[q] = pack_bf16x2(d0 / (1.f + __expf(-gf.x)), d1 / (1.f + __expf(-gf.y)));
+      }
+      *reinterpret_cast<uint4*>(a.out + idx) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, CB_N);
+}
+
+cudaError_t launch_decode_combine_tc(const DecodeParams& p, cudaStream_t s) {
+  CUtensorMap tw;
+  const int ncol = p.n_kv * (p.d_nope + p.d_v);
+  const uint64_t dims[2] = {(uint64_t)ncol, (uint64_t)p.d_c}, str[1] = {(uint64_t)ncol * 2};
+  const uint32_t box[2] = {64, 256};
+  if (!make_tmap_bf16(&tw, p.w_ukv, 2, dims, str, box)) return cudaErrorInvalidValue;
+  CombineTcArgs a{};
+  a.B = p.B; a.n_kv = p.n_kv; a.g = p.g; a.H_q = p.n_kv * (p.g + 1); a.n_hg = p.n_hg; a.hpc = p.hpc;
+  a.n_ranges = p.n_ranges; a.part_heads = p.part_heads; a.spb = dtc::CB_M / (p.g + 1);
+  a.seqinfo = p.seqinfo; a.part_o = p.part_o; a.part_ml = p.part_ml; a.lam = p.lam;
+  a.gate = reinterpret_cast<const __nv_bfloat16*>(p.gate);
+  a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+  a.status = p.status;
+  cudaError_t e = cudaFuncSetAttribute(decode_combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dtc::CB_SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)p.n_kv, (unsigned)((p.B + a.spb - 1) / a.spb));
+  cfg.blockDim = dim3(512);
+  cfg.dynamicSmemBytes = dtc::CB_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_combine_tc_kernel, tw, a);
 }
 
 template <int TT, int STAGES, int PST, int PF>

@@ -625,9 +625,9 @@ gdla_status gdla_decode(const gdla_decode_args* a, void* stream) {
   p.part_o = (float*)(ws + lay.part_o); p.part_ml = (float*)(ws + lay.part_ml);
   p.status = (int*)(ws + lay.status);
   cudaError_t e = cudaMemsetAsync(p.status, 0, kStatusBytes, s);
-  if (e == cudaSuccess) e = launch_decode_absorb(p, a->dtype, s);
+  if (e == cudaSuccess) e = lay.tc ? launch_decode_absorb_tc(p, s) : launch_decode_absorb(p, a->dtype, s);
   if (e == cudaSuccess) e = lay.tc ? launch_decode_split_tc(p, s) : launch_decode_split_simt(p, a->dtype, s);
-  if (e == cudaSuccess) e = launch_decode_combine(p, a->dtype, s);
+  if (e == cudaSuccess) e = lay.tc ? launch_decode_combine_tc(p, s) : launch_decode_combine(p, a->dtype, s);
   return cuda_status(e);
 }
 

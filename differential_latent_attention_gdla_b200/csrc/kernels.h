@@ -102,6 +102,10 @@ struct DecodeParams {
 cudaError_t launch_decode_absorb(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
 cudaError_t launch_decode_split_simt(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
 cudaError_t launch_decode_combine(const DecodeParams& p, gdla_dtype dt, cudaStream_t s);
+// the absorbed query of the tensor-core path on the tensor cores (writes the query images),
+// and its merge + W_UV product + epilogue (after the split kernel)
+cudaError_t launch_decode_absorb_tc(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_decode_combine_tc(const DecodeParams& p, cudaStream_t s);
 // tcgen05/TMA split-KV pass (bf16, d_c = 512, d_rope = 64, any head count), launched
 // after absorb, whose tail it overlaps through programmatic dependent launch
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s);
