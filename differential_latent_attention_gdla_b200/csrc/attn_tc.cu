@@ -16,17 +16,20 @@
 //   warp 0      TMA producer: the pair's Q in three 64-dim chunks through a
 //               2-deep staging ring; K tiles (128 keys x 192) and V tiles
 //               (128 keys x 128), each in a 2-deep ring;
-//   warp 1      MMA issuer (one lane): S(j) into S buffer j % 2, then
-//               O += P(j) V(j), then S(j+2);
+//   warp 1      S issuer (one lane): S(j) into S buffer j % 2, once PV(j-2)
+//               has consumed the P that shares that buffer;
+//   warp 2      PV issuer (one lane): O += P(j) V(j). Two issuing threads: one
+//               thread issues an M = 128 x N = 128 MMA only every ~130 clocks,
+//               about 0.7 of the tensor pipe's rate; two together keep it busy;
 //   warps 4-19  four warpgroups; warpgroup c owns key columns 32c .. 32c+31 of
 //               every tile and value columns 32c .. 32c+31 of O. A thread takes
 //               one stacked row; the four threads of a row agree on the row
 //               maximum and sum through shared memory.
 // TMEM (512 columns): S buffers at 0 and 128 (P overwrites the first 64 columns
 // of its S buffer as bf16), O at 256, Q at 384 (96 columns of bf16 pairs). While
-// the softmax of tile j runs, the tensor core computes PV(j-1) and S(j+1). The
-// tensor core runs the MMAs of one thread in issue order, so S(j+2) (issued after
-// PV(j)) never overwrites P(j) too early.
+// the softmax of tile j runs, the tensor core computes PV(j-1) and S(j+1). The S
+// issuer waits for PV(j) to complete (barrier pv_free) before S(j+2) overwrites
+// P(j).
 // The noise head's normalised output H_N is parked in shared memory (bf16) for
 // the epilogues of all g signal heads, so neither H_S nor H_N goes to global
 // memory. O is rescaled only when a row's running maximum grows by more than
@@ -68,7 +71,7 @@ constexpr uint32_t kColO = 256u, kColQ = 384u;
 
 struct Bars {
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2], q_full[2], q_free[2];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full[2], p_full[2], pv_free[2];
   uint64_t pv_done, q_ready, o_full, mx_ready, ml_ready, hn_ready, mma_done;
   uint32_t tmem_slot;
   int abort_flag;
@@ -145,17 +148,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(smem_u32(&bars.v_full[i]), 1);
       mbar_init(smem_u32(&bars.v_empty[i]), 1);
       mbar_init(smem_u32(&bars.q_full[i]), 1);
-      mbar_init(smem_u32(&bars.q_free[i]), 128 * NWG);
+      mbar_init(smem_u32(&bars.q_free[i]), 4 * NWG);
       mbar_init(smem_u32(&bars.s_full[i]), 1);
-      mbar_init(smem_u32(&bars.p_full[i]), 128 * NWG);
+      mbar_init(smem_u32(&bars.p_full[i]), 4 * NWG);
+      mbar_init(smem_u32(&bars.pv_free[i]), 1);
     }
     mbar_init(smem_u32(&bars.pv_done), 1);
-    mbar_init(smem_u32(&bars.q_ready), 128 * NWG);
+    mbar_init(smem_u32(&bars.q_ready), 4 * NWG);
     mbar_init(smem_u32(&bars.o_full), 1);
-    mbar_init(smem_u32(&bars.mx_ready), 128 * NWG);
-    mbar_init(smem_u32(&bars.ml_ready), 128 * NWG);
-    mbar_init(smem_u32(&bars.hn_ready), 64 * NWG);
-    mbar_init(smem_u32(&bars.mma_done), 1);
+    mbar_init(smem_u32(&bars.mx_ready), 4 * NWG);
+    mbar_init(smem_u32(&bars.ml_ready), 4 * NWG);
+    mbar_init(smem_u32(&bars.hn_ready), 2 * NWG);
+    mbar_init(smem_u32(&bars.mma_done), 2);  // one commit from each issuer
+    // the softmax warps arrive once per warp (q_free .. hn_ready)
     fence_mbar_init();
     abort_flag = 0;
     // an earlier CTA of this call timed out: this one does no work (decided once for the CTA)
@@ -251,61 +256,72 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_wait(smem_u32(&bars.q_full[c & 1]), (c >> 1) & 1, nullptr, 0);
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // --------------------------------------------------------- MMA issuers
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(ROWS, BN, false, false);
-      constexpr uint32_t idO = idesc_bf16_f32(ROWS, DV, false, true);
-      int kc = 0, vc = 0;
-      int sg = 0, pg = 0;  // S / PV tiles issued over the whole CTA (S buffer index and phases)
       bool ok = true;
-      // S(jj) = Q K(jj)^T into S buffer sg % 2 (Q from TMEM); releases the K buffer when done
-      auto issue_s = [&]() -> bool {
-        const int u = sg & 1, sl = kc & 1;
-        if (!mbar_wait(smem_u32(&bars.k_full[sl]), (kc >> 1) & 1, a.status, 212, &abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kb = smem_u32(k_sm + sl * K_BYTES);
+      if (warp == 1) {
+        // S(jj) = Q K(jj)^T into S buffer sg % 2 (Q from TMEM); releases the K buffer when done
+        constexpr uint32_t idS = idesc_bf16_f32(ROWS, BN, false, false);
+        int kc = 0, sg = 0;  // K tiles / S tiles issued over the whole CTA (ring and buffer phases)
+        for (int p = 0; p < n_pairs && ok; ++p) {
+          // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
+          ok = mbar_wait(smem_u32(&bars.q_ready), p & 1, a.status, 211, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          for (int jj = 0; jj < n_tiles && ok; ++jj) {
+            const int u = sg & 1, sl = kc & 1;
+            // P(sg - 2), which PV(sg - 2) reads, lives in the columns S(sg) overwrites
+            if (sg >= 2 && !mbar_wait(smem_u32(&bars.pv_free[u]), ((sg >> 1) - 1) & 1, a.status, 215, &abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait(smem_u32(&bars.k_full[sl]), (kc >> 1) & 1, a.status, 212, &abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kb = smem_u32(k_sm + sl * K_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < (DN + DR) / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(kb + (kk >> 2) * K_CHUNK + (kk & 3) * 32, 16, 1024);
-          mma_ts(tmem + col_s(u), tmem + kColQ + kk * 8, bd, idS, kk > 0);
+            for (int kk = 0; kk < (DN + DR) / 16; ++kk) {
+              const uint64_t bd = sdesc_sw128(kb + (kk >> 2) * K_CHUNK + (kk & 3) * 32, 16, 1024);
+              mma_ts(tmem + col_s(u), tmem + kColQ + kk * 8, bd, idS, kk > 0);
+            }
+            mma_commit(smem_u32(&bars.s_full[u]));
+            mma_commit(smem_u32(&bars.k_empty[sl]));
+            ++kc;
+            ++sg;
+          }
         }
-        mma_commit(smem_u32(&bars.s_full[u]));
-        mma_commit(smem_u32(&bars.k_empty[sl]));
-        ++kc;
-        ++sg;
-        return true;
-      };
-      // O += P(jj) V(jj); releases the V buffer when done
-      auto issue_pv = [&](int jj) -> bool {
-        const int u = pg & 1, sl = vc & 1;
-        if (!mbar_wait(smem_u32(&bars.p_full[u]), (pg >> 1) & 1, a.status, 214, &abort_flag)) return false;
-        if (!mbar_wait(smem_u32(&bars.v_full[sl]), (vc >> 1) & 1, a.status, 213, &abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vb = smem_u32(v_sm + sl * V_BYTES);
+      } else {
+        // O += P(jj) V(jj); releases the V buffer and the S/P buffer when done
+        constexpr uint32_t idO = idesc_bf16_f32(ROWS, DV, false, true);
+        int vc = 0, pg = 0;  // V tiles / PV tiles issued over the whole CTA
+        for (int p = 0; p < n_pairs && ok; ++p) {
+          for (int jj = 0; jj < n_tiles && ok; ++jj) {
+            const int u = pg & 1, sl = vc & 1;
+            if (!mbar_wait(smem_u32(&bars.p_full[u]), (pg >> 1) & 1, a.status, 214, &abort_flag) ||
+                !mbar_wait(smem_u32(&bars.v_full[sl]), (vc >> 1) & 1, a.status, 213, &abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t vb = smem_u32(v_sm + sl * V_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(vb + kk * 2048, V_BLOCK, 1024);
-          mma_ts(tmem + kColO, tmem + col_s(u) + kk * 8, bd, idO, (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              const uint64_t bd = sdesc_sw128(vb + kk * 2048, V_BLOCK, 1024);
+              mma_ts(tmem + kColO, tmem + col_s(u) + kk * 8, bd, idO, (jj > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(smem_u32(&bars.pv_done));
+            mma_commit(smem_u32(&bars.pv_free[u]));
+            mma_commit(smem_u32(&bars.v_empty[sl]));
+            ++pg;
+            ++vc;
+          }
+          // every S MMA of the pair completed before its last P was written, so this
+          // commit covers all tensor-core work on the pair
+          if (ok) mma_commit(smem_u32(&bars.o_full));
         }
-        mma_commit(smem_u32(&bars.pv_done));
-        mma_commit(smem_u32(&bars.v_empty[sl]));
-        ++pg;
-        ++vc;
-        return true;
-      };
-      for (int p = 0; p < n_pairs && ok; ++p) {
-        // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
-        ok = mbar_wait(smem_u32(&bars.q_ready), p & 1, a.status, 211, &abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        ok = issue_s() && (n_tiles < 2 || issue_s());
-        for (int jj = 0; jj < n_tiles && ok; ++jj) {
-          ok = issue_pv(jj);
-          if (ok && jj + 2 < n_tiles) ok = issue_s();
-        }
-        if (!ok) break;
-        mma_commit(smem_u32(&bars.o_full));
       }
       if (!ok) abort_flag = 1;
       // every MMA this thread issued has completed before TMEM is released
@@ -366,12 +382,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_st4(tQ + 64 + 4 * c, lo);
           tmem_st4(tQ + 64 + 16 + 4 * c, hi);
         }
-        mbar_arrive(smem_u32(&bars.q_free[sl]));
+        mbar_arrive_warp(smem_u32(&bars.q_free[sl]));
       }
       if (failed) break;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars.q_ready));
+      mbar_arrive_warp(smem_u32(&bars.q_ready));
 
       // ---- online softmax over all key tiles, CW key columns per thread
       float m_ref = -INFINITY, l_part = 0.f;
@@ -408,7 +424,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float* xs = xm + (tc & 1) * (NWG * ROWS);
         xs[c * ROWS + r] = pm;
         tc_fence_before();  // this thread's S loads are done before another quarter overwrites them with P
-        mbar_arrive(smem_u32(&bars.mx_ready));
+        mbar_arrive_warp(smem_u32(&bars.mx_ready));
         ok = mbar_wait(smem_u32(&bars.mx_ready), tc & 1, a.status, 227, &abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           failed = true;
@@ -446,8 +462,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_st16(tS + (CW / 2) * c, pk);
         if (!first && __any_sync(0xffffffffu, need)) {
           // this quarter of O must hold every earlier tile before it is rescaled and PV(jj)
-          // adds to it: PV(jj-1) is the CTA's PV number tc - 1; PV(jj-2) preceded S(jj) in
-          // issue order, so the wait is within one phase
+          // adds to it: PV(jj-1) is the CTA's PV number tc - 1; PV(jj-2) completed before
+          // S(jj) was issued, so the wait is within one phase
           ok = mbar_wait(smem_u32(&bars.pv_done), (tc - 1) & 1, a.status, 226, &abort_flag);
           if (!__all_sync(0xffffffffu, ok)) {
             failed = true;
@@ -463,7 +479,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars.p_full[u]));
+        mbar_arrive_warp(smem_u32(&bars.p_full[u]));
       }
       if (failed) break;
 
@@ -479,7 +495,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       {
         float* xs = xm + (tc & 1) * (NWG * ROWS);
         xs[c * ROWS + r] = l_part;
-        mbar_arrive(smem_u32(&bars.ml_ready));
+        mbar_arrive_warp(smem_u32(&bars.ml_ready));
         ok = mbar_wait(smem_u32(&bars.ml_ready), p & 1, a.status, 225, &abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           failed = true;
@@ -508,7 +524,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             *reinterpret_cast<uint4*>(hn_sm + hn_off(r & (BM - 1), (cbase + 16 * ch) / 8 + q)) = pv;
           }
         }
-        mbar_arrive(smem_u32(&bars.hn_ready));
+        mbar_arrive_warp(smem_u32(&bars.hn_ready));
       } else if (real) {
         // signal head: D = H_S - lambda H_N, Y = sigmoid(G) D
         ok = mbar_wait(smem_u32(&bars.hn_ready), 0, a.status, 224, &abort_flag);

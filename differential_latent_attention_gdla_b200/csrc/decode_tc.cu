@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sh.s_full[i]), 2);  // one commit per score warp
-      mbar_init(smem_u32(&sh.p_full[i]), 128);
+      mbar_init(smem_u32(&sh.p_full[i]), 4);  // one arrival per softmax warp
     }
     for (int i = 0; i < PST; ++i) mbar_init(smem_u32(&sh.p_free[i]), 1);
     mbar_init(smem_u32(&sh.q_full), 1);
@@ -560,7 +560,7 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sh.p_full[k & 1]));
+      mbar_arrive_warp(smem_u32(&sh.p_full[k & 1]));
 
       if (last) {
         // ---- partial result of this sequence share: (m, l) per head and O^T

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(gtc::GTHREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars.acc_full[i]), 1);
-      mbar_init(smem_u32(&bars.acc_empty[i]), 128);
+      mbar_init(smem_u32(&bars.acc_empty[i]), 4);  // one arrival per epilogue warp
     }
     mbar_init(smem_u32(&bars.mma_done), 1);
     fence_mbar_init();
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(gtc::GTHREADS, 1)
         if (row < a.M && c0 < a.N) store_chunk<OutT>(C + row * a.N + c0, r, a.N - c0);
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars.acc_empty[buf]));
+      mbar_arrive_warp(smem_u32(&bars.acc_empty[buf]));
     }
   }
   tc_fence_before();
