@@ -281,12 +281,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t kb = smem_u32(k_sm + sl * K_BYTES);
+            // one base descriptor plus compile-time offsets: a few instructions per MMA
+            const uint64_t kd = sdesc_sw128(smem_u32(k_sm + sl * K_BYTES), 16, 1024);
+            const uint32_t dS = tmem + col_s(u), aQ = tmem + kColQ;
 #pragma unroll
-            for (int kk = 0; kk < (DN + DR) / 16; ++kk) {
-              const uint64_t bd = sdesc_sw128(kb + (kk >> 2) * K_CHUNK + (kk & 3) * 32, 16, 1024);
-              mma_ts(tmem + col_s(u), tmem + kColQ + kk * 8, bd, idS, kk > 0);
-            }
+            for (int kk = 0; kk < (DN + DR) / 16; ++kk)
+              mma_ts(dS, aQ + kk * 8, kd + (uint64_t)(((kk >> 2) * K_CHUNK + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
             mma_commit(smem_u32(&bars.s_full[u]));
             mma_commit(smem_u32(&bars.k_empty[sl]));
             ++kc;
@@ -306,12 +306,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t vb = smem_u32(v_sm + sl * V_BYTES);
+            const uint64_t vd = sdesc_sw128(smem_u32(v_sm + sl * V_BYTES), V_BLOCK, 1024);
+            const uint32_t dO = tmem + kColO, aP = tmem + col_s(u);
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              const uint64_t bd = sdesc_sw128(vb + kk * 2048, V_BLOCK, 1024);
-              mma_ts(tmem + kColO, tmem + col_s(u) + kk * 8, bd, idO, (jj > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ts(dO, aP + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idO, (jj > 0 || kk > 0) ? 1u : 0u);
             mma_commit(smem_u32(&bars.pv_done));
             mma_commit(smem_u32(&bars.pv_free[u]));
             mma_commit(smem_u32(&bars.v_empty[sl]));

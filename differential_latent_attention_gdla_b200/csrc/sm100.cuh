@@ -303,6 +303,8 @@ __device__ __forceinline__ float ex2_approx(float x) {
 //     -> sbo = 1024, lbo unused (16); advance K by 16 elements = +32 B.
 //   MN-major operand tile: 64-element MN blocks of [K rows x 128 B]
 //     -> lbo = bytes between MN blocks, sbo = 1024 (8 K rows); K by 16 = +2048 B.
+// The start address is held as addr / 16 in the low 14 bits, so for 16-byte-aligned
+// shared addresses (all below 256 KB) desc(addr + off) = desc(addr) + off / 16.
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
