@@ -57,8 +57,6 @@ cudaError_t launch_attn_simt(const AttnParams& p, gdla_dtype dt, cudaStream_t s)
 // shapes the tcgen05/TMA attention takes (bf16, heads of 128 + 64 rotary, d_v = 128)
 bool attn_tc_shape(const AttnParams& p, gdla_dtype dt);
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
-// the same attention with two head pairs in flight per CTA (attn_pp.cu)
-cudaError_t launch_attn_pp(const AttnParams& p, cudaStream_t s);
 
 // ---- decode (steps 3-8 over the latent cache, absorbed form).
 // Two layouts of the split-KV work:
