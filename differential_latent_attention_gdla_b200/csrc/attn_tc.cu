@@ -16,20 +16,18 @@
 //   warp 0      TMA producer: the pair's Q in three 64-dim chunks through a
 //               2-deep staging ring; K tiles (128 keys x 192) and V tiles
 //               (128 keys x 128), each in a 2-deep ring;
-//   warp 1      S issuer (one lane): S(j) into S buffer j % 2, once PV(j-2)
-//               has consumed the P that shares that buffer;
-//   warp 2      PV issuer (one lane): O += P(j) V(j). Two issuing threads: one
-//               thread issues an M = 128 x N = 128 MMA only every ~130 clocks,
-//               about 0.7 of the tensor pipe's rate; two together keep it busy;
+//   warp 1      MMA issuer (one lane): S(j) into S buffer j % 2, then
+//               O += P(j) V(j), then S(j+2). With its operand descriptors
+//               precomputed it issues at the tensor pipe's own rate;
 //   warps 4-19  four warpgroups; warpgroup c owns key columns 32c .. 32c+31 of
 //               every tile and value columns 32c .. 32c+31 of O. A thread takes
 //               one stacked row; the four threads of a row agree on the row
 //               maximum and sum through shared memory.
 // TMEM (512 columns): S buffers at 0 and 128 (P overwrites the first 64 columns
 // of its S buffer as bf16), O at 256, Q at 384 (96 columns of bf16 pairs). While
-// the softmax of tile j runs, the tensor core computes PV(j-1) and S(j+1). The S
-// issuer waits for PV(j) to complete (barrier pv_free) before S(j+2) overwrites
-// P(j).
+// the softmax of tile j runs, the tensor core computes PV(j-1) and S(j+1). The
+// tensor core runs the MMAs of one thread in issue order, so S(j+2) (issued after
+// PV(j)) never overwrites P(j) too early.
 // The noise head's normalised output H_N is parked in shared memory (bf16) for
 // the epilogues of all g signal heads, so neither H_S nor H_N goes to global
 // memory. O is rescaled only when a row's running maximum grows by more than
@@ -71,14 +69,18 @@ constexpr uint32_t kColO = 256u, kColQ = 384u;
 
 struct Bars {
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2], q_full[2], q_free[2];
-  uint64_t s_full[2], p_full[2], pv_free[2];
-  uint64_t pv_done, q_ready, o_full, mx_ready, ml_ready, hn_ready, mma_done;
+  uint64_t s_full[2], p_full[2];
+  uint64_t pv_done, q_ready, o_full, mma_done;
   uint32_t tmem_slot;
   int abort_flag;
   int skip_cta;
 };
 constexpr int SMEM_BYTES = OFF_BARS + (int)sizeof(Bars);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
+
+// named barrier 1: the 512 softmax threads (warps 4-19)
+__device__ __forceinline__ bool bar_or512(bool pred) { return sm100::named_bar_or(1, 128 * NWG, pred); }
+__device__ __forceinline__ void bar_sync512() { sm100::named_bar_sync(1, 128 * NWG); }
 
 // parked H_N: row r (of 64), 16-byte chunk c (of 16) stored at chunk c ^ (r & 15)
 __device__ __forceinline__ uint32_t hn_off(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 15)) << 4)); }
@@ -151,16 +153,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(smem_u32(&bars.q_free[i]), 4 * NWG);
       mbar_init(smem_u32(&bars.s_full[i]), 1);
       mbar_init(smem_u32(&bars.p_full[i]), 4 * NWG);
-      mbar_init(smem_u32(&bars.pv_free[i]), 1);
     }
     mbar_init(smem_u32(&bars.pv_done), 1);
     mbar_init(smem_u32(&bars.q_ready), 4 * NWG);
     mbar_init(smem_u32(&bars.o_full), 1);
-    mbar_init(smem_u32(&bars.mx_ready), 4 * NWG);
-    mbar_init(smem_u32(&bars.ml_ready), 4 * NWG);
-    mbar_init(smem_u32(&bars.hn_ready), 2 * NWG);
-    mbar_init(smem_u32(&bars.mma_done), 2);  // one commit from each issuer
-    // the softmax warps arrive once per warp (q_free .. hn_ready)
+    mbar_init(smem_u32(&bars.mma_done), 1);
+    // the softmax warps arrive once per warp (q_free, q_ready, p_full)
     fence_mbar_init();
     abort_flag = 0;
     // an earlier CTA of this call timed out: this one does no work (decided once for the CTA)
@@ -256,71 +254,61 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mbar_wait(smem_u32(&bars.q_full[c & 1]), (c >> 1) & 1, nullptr, 0);
       }
     }
-  } else if (warp == 1 || warp == 2) {
-    // --------------------------------------------------------- MMA issuers
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(ROWS, BN, false, false);
+      constexpr uint32_t idO = idesc_bf16_f32(ROWS, DV, false, true);
+      int kc = 0, vc = 0;
+      int sg = 0, pg = 0;  // S / PV tiles issued over the whole CTA (S buffer index and phases)
       bool ok = true;
-      if (warp == 1) {
-        // S(jj) = Q K(jj)^T into S buffer sg % 2 (Q from TMEM); releases the K buffer when done
-        constexpr uint32_t idS = idesc_bf16_f32(ROWS, BN, false, false);
-        int kc = 0, sg = 0;  // K tiles / S tiles issued over the whole CTA (ring and buffer phases)
-        for (int p = 0; p < n_pairs && ok; ++p) {
-          // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
-          ok = mbar_wait(smem_u32(&bars.q_ready), p & 1, a.status, 211, &abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          for (int jj = 0; jj < n_tiles && ok; ++jj) {
-            const int u = sg & 1, sl = kc & 1;
-            // P(sg - 2), which PV(sg - 2) reads, lives in the columns S(sg) overwrites
-            if (sg >= 2 && !mbar_wait(smem_u32(&bars.pv_free[u]), ((sg >> 1) - 1) & 1, a.status, 215, &abort_flag)) {
-              ok = false;
-              break;
-            }
-            if (!mbar_wait(smem_u32(&bars.k_full[sl]), (kc >> 1) & 1, a.status, 212, &abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            // one base descriptor plus compile-time offsets: a few instructions per MMA
-            const uint64_t kd = sdesc_sw128(smem_u32(k_sm + sl * K_BYTES), 16, 1024);
-            const uint32_t dS = tmem + col_s(u), aQ = tmem + kColQ;
+      // S(jj) = Q K(jj)^T into S buffer sg % 2 (Q from TMEM); releases the K buffer when done.
+      // One base descriptor per operand tile plus compile-time offsets: a few instructions
+      // per MMA, so the issue keeps up with the tensor pipe.
+      auto issue_s = [&]() -> bool {
+        const int u = sg & 1, sl = kc & 1;
+        if (!mbar_wait(smem_u32(&bars.k_full[sl]), (kc >> 1) & 1, a.status, 212, &abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t kd = sdesc_sw128(smem_u32(k_sm + sl * K_BYTES), 16, 1024);
+        const uint32_t dS = tmem + col_s(u), aQ = tmem + kColQ;
 #pragma unroll
-            for (int kk = 0; kk < (DN + DR) / 16; ++kk)
-              mma_ts(dS, aQ + kk * 8, kd + (uint64_t)(((kk >> 2) * K_CHUNK + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
-            mma_commit(smem_u32(&bars.s_full[u]));
-            mma_commit(smem_u32(&bars.k_empty[sl]));
-            ++kc;
-            ++sg;
-          }
-        }
-      } else {
-        // O += P(jj) V(jj); releases the V buffer and the S/P buffer when done
-        constexpr uint32_t idO = idesc_bf16_f32(ROWS, DV, false, true);
-        int vc = 0, pg = 0;  // V tiles / PV tiles issued over the whole CTA
-        for (int p = 0; p < n_pairs && ok; ++p) {
-          for (int jj = 0; jj < n_tiles && ok; ++jj) {
-            const int u = pg & 1, sl = vc & 1;
-            if (!mbar_wait(smem_u32(&bars.p_full[u]), (pg >> 1) & 1, a.status, 214, &abort_flag) ||
-                !mbar_wait(smem_u32(&bars.v_full[sl]), (vc >> 1) & 1, a.status, 213, &abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t vd = sdesc_sw128(smem_u32(v_sm + sl * V_BYTES), V_BLOCK, 1024);
-            const uint32_t dO = tmem + kColO, aP = tmem + col_s(u);
+        for (int kk = 0; kk < (DN + DR) / 16; ++kk)
+          mma_ts(dS, aQ + kk * 8, kd + (uint64_t)(((kk >> 2) * K_CHUNK + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
+        mma_commit(smem_u32(&bars.s_full[u]));
+        mma_commit(smem_u32(&bars.k_empty[sl]));
+        ++kc;
+        ++sg;
+        return true;
+      };
+      // O += P(jj) V(jj); releases the V buffer when done
+      auto issue_pv = [&](int jj) -> bool {
+        const int u = pg & 1, sl = vc & 1;
+        if (!mbar_wait(smem_u32(&bars.p_full[u]), (pg >> 1) & 1, a.status, 214, &abort_flag)) return false;
+        if (!mbar_wait(smem_u32(&bars.v_full[sl]), (vc >> 1) & 1, a.status, 213, &abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t vd = sdesc_sw128(smem_u32(v_sm + sl * V_BYTES), V_BLOCK, 1024);
+        const uint32_t dO = tmem + kColO, aP = tmem + col_s(u);
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
-              mma_ts(dO, aP + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idO, (jj > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(smem_u32(&bars.pv_done));
-            mma_commit(smem_u32(&bars.pv_free[u]));
-            mma_commit(smem_u32(&bars.v_empty[sl]));
-            ++pg;
-            ++vc;
-          }
-          // every S MMA of the pair completed before its last P was written, so this
-          // commit covers all tensor-core work on the pair
-          if (ok) mma_commit(smem_u32(&bars.o_full));
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(dO, aP + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idO, (jj > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bars.pv_done));
+        mma_commit(smem_u32(&bars.v_empty[sl]));
+        ++pg;
+        ++vc;
+        return true;
+      };
+      for (int p = 0; p < n_pairs && ok; ++p) {
+        // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
+        ok = mbar_wait(smem_u32(&bars.q_ready), p & 1, a.status, 211, &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        ok = issue_s() && (n_tiles < 2 || issue_s());
+        for (int jj = 0; jj < n_tiles && ok; ++jj) {
+          ok = issue_pv(jj);
+          if (ok && jj + 2 < n_tiles) ok = issue_s();
         }
+        if (!ok) break;
+        mma_commit(smem_u32(&bars.o_full));
       }
       if (!ok) abort_flag = 1;
       // every MMA this thread issued has completed before TMEM is released
@@ -329,6 +317,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------- softmax + epilogue
+    // Every decision that changes the path of these 16 warps (a failed wait, a grown
+    // maximum) is taken by all of them together through a barrier-reduction on named
+    // barrier 1, so no warp ever waits there for one that left.
     const int c = (warp - 4) >> 2;          // column quarter: keys 32c.. of each tile, value dims 32c.. of O
     const int q4 = warp & 3;                // TMEM lane quadrant
     const int r = q4 * 32 + lane;           // stacked row = TMEM lane
@@ -338,20 +329,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const uint32_t tO = tmem + lane_base + kColO + CW * c;
     const uint32_t tQ = tmem + lane_base + kColQ;
-    int tc = 0;                             // tiles processed over the whole CTA
-    bool failed = false;
-    for (int p = 0; p < n_pairs && !failed; ++p) {
-      const int hl = 2 * p + half;
-      // ---- Q of this row into TMEM: thread c moves dims 16c .. 16c+15 of each
-      // content chunk and rotates dims 8c .. 8c+7 with 32+8c .. 32+8c+7 of the rotary chunk
-      bool ok = true;
-      for (int k = 0; k < 3; ++k) {
-        const int qk = 3 * p + k, sl = qk & 1;
-        ok = mbar_wait(smem_u32(&bars.q_full[sl]), (qk >> 1) & 1, a.status, 221, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          failed = true;
-          break;
-        }
+    // this row's RoPE factors for rotary dims 8c .. 8c+7 (the same positions in every
+    // pair), loaded ahead of each pair's rotary chunk (volatile: live only between the
+    // load and that chunk, not across the key tiles)
+    float cs[8], sn[8];
+    const int rope_pos = row_ok ? i : q_end - 1;  // rows past the end are discarded; any table row will do
+    auto load_rope = [&]() {
+      const float* cp = a.cos_tab + (long)rope_pos * (DR / 2) + 8 * c;
+      const float* sp = a.sin_tab + (long)rope_pos * (DR / 2) + 8 * c;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(cs[e]) : "l"(cp + e));
+        asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(sn[e]) : "l"(sp + e));
+      }
+    };
+    load_rope();
+    // chunk k of pair p's stacked Q rows into TMEM: thread c moves dims 16c .. 16c+15 of a
+    // content chunk, or rotates dims 8c .. 8c+7 with 32+8c .. 32+8c+7 of the rotary chunk
+    auto move_q = [&](int p, int k) -> bool {
+      const int qk = 3 * p + k, sl = qk & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.q_full[sl]), (qk >> 1) & 1, a.status, 221, &abort_flag));
+      if (ok) {
         const uint8_t* rowp = qs_sm + sl * QS_BYTES + r * 128;
         const int sw = r & 7;
         if (k < 2) {
@@ -366,42 +364,66 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint4 vh = *reinterpret_cast<const uint4*>(rowp + (((4 + c) ^ sw) << 4));
           const __nv_bfloat162* hl2 = reinterpret_cast<const __nv_bfloat162*>(&vl);
           const __nv_bfloat162* hh2 = reinterpret_cast<const __nv_bfloat162*>(&vh);
-          const int pos = row_ok ? i : q_end - 1;  // rows past the end are discarded; any table row will do
-          const float* cs = a.cos_tab + (long)pos * (DR / 2) + 8 * c;
-          const float* sn = a.sin_tab + (long)pos * (DR / 2) + 8 * c;
           uint32_t lo[4], hi[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 x = __bfloat1622float2(hl2[e]);
             const float2 y = __bfloat1622float2(hh2[e]);
-            const float c0 = cs[2 * e], s0 = sn[2 * e], c1 = cs[2 * e + 1], s1 = sn[2 * e + 1];
-            lo[e] = pack_bf16x2(x.x * c0 - y.x * s0, x.y * c1 - y.y * s1);
-            hi[e] = pack_bf16x2(y.x * c0 + x.x * s0, y.y * c1 + x.y * s1);
+            lo[e] = pack_bf16x2(x.x * cs[2 * e] - y.x * sn[2 * e], x.y * cs[2 * e + 1] - y.y * sn[2 * e + 1]);
+            hi[e] = pack_bf16x2(y.x * cs[2 * e] + x.x * sn[2 * e], y.y * cs[2 * e + 1] + x.y * sn[2 * e + 1]);
           }
           tmem_st4(tQ + 64 + 4 * c, lo);
           tmem_st4(tQ + 64 + 16 + 4 * c, hi);
         }
         mbar_arrive_warp(smem_u32(&bars.q_free[sl]));
       }
-      if (failed) break;
+      return ok;
+    };
+    auto q_done = [&]() {
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(smem_u32(&bars.q_ready));
+    };
+    int tc = 0;                             // tiles processed over the whole CTA
+    bool failed = false;
+    {
+      bool ok = true;
+      for (int k = 0; k < 3; ++k) ok = move_q(0, k) && ok;
+      failed = bar_or512(!ok);
+      if (!failed) q_done();
+    }
+    for (int p = 0; p < n_pairs && !failed; ++p) {
+      const int hl = 2 * p + half;
+      const int cbase = CW * c;             // this warpgroup finishes value columns [cbase, cbase + 32)
+      const bool real = hl < G1;            // the second half of a short last pair is discarded
+      const bool next = p + 1 < n_pairs;
+      const int sh = hl > 0 ? head_of(hl) : 0;  // signal head index
+      const long tok = (long)b * a.q_len + (i - a.q_start);
+      if (hl > 0 && real && row_ok) {
+        // the epilogue's gate and lambda of this row: into L2 while the key tiles stream
+        prefetch_l2(a.gate + (tok * n_S + sh) * DV + cbase);
+        prefetch_l2(a.gate + (tok * n_S + sh) * DV + cbase + CW - 1);
+        prefetch_l2(a.lam + tok * n_S + sh);
+      }
 
-      // ---- online softmax over all key tiles, CW key columns per thread
+      // ---- online softmax over all key tiles, CW key columns per thread. The running
+      // maximum m_ref of a row is kept identical in its four threads; the tile's row
+      // maximum is exchanged only when some row's maximum has grown by more than 2^8
+      // (kRescaleThreshold, log2 units) since its m_ref, so most tiles need no exchange.
       float m_ref = -INFINITY, l_part = 0.f;
       for (int jj = 0; jj < n_tiles; ++jj, ++tc) {
         const int u = tc & 1;
-        ok = mbar_wait(smem_u32(&bars.s_full[u]), (tc >> 1) & 1, a.status, 222, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          failed = true;
-          break;
-        }
-        tc_fence_after();
+        const bool w_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.s_full[u]), (tc >> 1) & 1, a.status, 222, &abort_flag));
         const uint32_t tS = tmem + lane_base + col_s(u);
         uint32_t sr[CW];
-        tmem_ld32(tS + CW * c, sr);
-        tmem_wait_ld();
+        if (w_ok) {
+          tc_fence_after();
+          tmem_ld32(tS + CW * c, sr);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < CW; ++e) sr[e] = __float_as_uint(-INFINITY);
+        }
         const int key0 = (j_lo + jj) * BN + CW * c;
         const bool full_vis = (key0 + CW - 1 <= m0) && (!a.sliding || key0 > m0 + BM - 1 - a.window);
         if (!full_vis) {
@@ -419,30 +441,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mq1 = fmax3(mq1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
         }
         const float pm = fmax3(fmaxf(mq0, mq1), __uint_as_float(sr[CW - 2]), __uint_as_float(sr[CW - 1]));
-        // the row maximum of the whole tile: exchange with the three threads holding the other columns
-        float* xs = xm + (tc & 1) * (NWG * ROWS);
-        xs[c * ROWS + r] = pm;
-        tc_fence_before();  // this thread's S loads are done before another quarter overwrites them with P
-        mbar_arrive_warp(smem_u32(&bars.mx_ready));
-        ok = mbar_wait(smem_u32(&bars.mx_ready), tc & 1, a.status, 227, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          failed = true;
-          break;
+        const bool first = (jj == 0);
+        // sl2 > 0: the maximum commutes with the scale. A first tile always exchanges.
+        const bool exceed = first || pm * a.sl2 > m_ref + kRescaleThreshold;
+        // this thread's S loads are done before another quarter overwrites them with P:
+        // the barrier-reduction below orders them
+        tc_fence_before();
+        if (bar_or512(exceed || !w_ok)) {
+          if (bar_or512(!w_ok)) {
+            failed = true;
+            break;
+          }
+          // the row maximum of the whole tile: exchange with the three threads holding the
+          // other columns (a slot is rewritten only after the next tile's barrier-reduction,
+          // which every thread reaches after reading it here)
+          float* xs = xm + (tc & 1) * (NWG * ROWS);
+          xs[c * ROWS + r] = pm;
+          bar_sync512();
+          const float mr = fmaxf(fmaxf(xs[r], xs[ROWS + r]), fmaxf(xs[2 * ROWS + r], xs[3 * ROWS + r]));
+          const float mx = mr * a.sl2;
+          const bool need = first || (mx > m_ref + kRescaleThreshold);
+          float alpha = 1.f;
+          if (need) {
+            const float m_new = first ? mx : fmaxf(m_ref, mx);
+            if (!first) alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_new);
+            l_part *= alpha;
+            m_ref = m_new;
+          }
+          if (!first && bar_or512(need)) {
+            // O must hold every earlier tile before it is rescaled and PV(jj) adds to it:
+            // PV(jj-1) is the CTA's PV number tc - 1; PV(jj-2) preceded S(jj) in issue
+            // order, so the wait is within one phase
+            const bool r_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.pv_done), (tc - 1) & 1, a.status, 226, &abort_flag));
+            if (bar_or512(!r_ok)) {
+              failed = true;
+              break;
+            }
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, need)) {
+              uint32_t o[32];
+              tmem_ld32(tO, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tO, o);
+            }
+          }
         }
         tc_fence_after();
-        const float mr = fmaxf(fmaxf(xs[r], xs[ROWS + r]), fmaxf(xs[2 * ROWS + r], xs[3 * ROWS + r]));
-        const float mx = mr * a.sl2;  // sl2 > 0: the maximum commutes with the scale
-        const bool first = (jj == 0);
-        const bool need = first || (mx > m_ref + kRescaleThreshold);
-        float alpha = 1.f;
-        if (need) {
-          const float m_new = first ? mx : fmaxf(m_ref, mx);
-          if (!first) alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - m_new);
-          l_part *= alpha;
-          m_ref = m_new;
-        }
         uint32_t pk[CW / 2];
-                {
+        {
           const float nm = (m_ref == -INFINITY) ? 0.f : -m_ref;
           const float2 sl2v = make_float2(a.sl2, a.sl2), nmv = make_float2(nm, nm);
           float2 rs0 = make_float2(0.f, 0.f), rs1 = make_float2(0.f, 0.f);
@@ -457,25 +505,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           l_part += (rs0.x + rs0.y) + (rs1.x + rs1.y);
         }
-        // P columns 16 c .. 16 c + 15 overwrite S columns that every quarter loaded before the exchange
+        // P columns 16 c .. 16 c + 15 overwrite S columns that every quarter loaded before
+        // the barrier-reduction above
         tmem_st16(tS + (CW / 2) * c, pk);
-        if (!first && __any_sync(0xffffffffu, need)) {
-          // this quarter of O must hold every earlier tile before it is rescaled and PV(jj)
-          // adds to it: PV(jj-1) is the CTA's PV number tc - 1; PV(jj-2) completed before
-          // S(jj) was issued, so the wait is within one phase
-          ok = mbar_wait(smem_u32(&bars.pv_done), (tc - 1) & 1, a.status, 226, &abort_flag);
-          if (!__all_sync(0xffffffffu, ok)) {
-            failed = true;
-            break;
-          }
-          tc_fence_after();
-          uint32_t o[32];
-          tmem_ld32(tO, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO, o);
-        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive_warp(smem_u32(&bars.p_full[u]));
@@ -483,28 +515,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (failed) break;
 
       // ---------------------------------------------------------- epilogue
-      ok = mbar_wait(smem_u32(&bars.o_full), p & 1, a.status, 223, &abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-      // row sum: add the other quarters' partial sums (same running maximum everywhere).
-      // Slot tc & 1 was last read two tiles ago.
       {
-        float* xs = xm + (tc & 1) * (NWG * ROWS);
-        xs[c * ROWS + r] = l_part;
-        mbar_arrive_warp(smem_u32(&bars.ml_ready));
-        ok = mbar_wait(smem_u32(&bars.ml_ready), p & 1, a.status, 225, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.o_full), p & 1, a.status, 223, &abort_flag));
+        if (bar_or512(!ok)) {
           failed = true;
           break;
         }
+      }
+      tc_fence_after();
+      if (next) {
+        // every S MMA of this pair is done, so the next pair's Q content chunks may go into
+        // TMEM now; its rotary chunk follows the epilogue, while that copy lands
+        bool ok = move_q(p + 1, 0);
+        ok = move_q(p + 1, 1) && ok;
+        if (bar_or512(!ok)) {
+          failed = true;
+          break;
+        }
+      }
+      // row sum: add the other quarters' partial sums (same running maximum everywhere).
+      // The slot was last read two tiles ago.
+      {
+        float* xs = xm + (tc & 1) * (NWG * ROWS);
+        xs[c * ROWS + r] = l_part;
+        bar_sync512();
         l_part = (xs[r] + xs[ROWS + r]) + (xs[2 * ROWS + r] + xs[3 * ROWS + r]);
       }
       const float inv = l_part > 0.f ? 1.f / l_part : 0.f;
-      const int cbase = CW * c;          // this warpgroup finishes value columns [cbase, cbase + 32)
-      const bool real = hl < G1;         // the second half of a short last pair is discarded
 
       if (hl == 0) {
         // noise head: park the normalised H_N (bf16) for every signal head
@@ -523,16 +560,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             *reinterpret_cast<uint4*>(hn_sm + hn_off(r & (BM - 1), (cbase + 16 * ch) / 8 + q)) = pv;
           }
         }
-        mbar_arrive_warp(smem_u32(&bars.hn_ready));
-      } else if (real) {
+      }
+      // pair 0 holds the noise head: its H_N is parked before any signal row reads it
+      if (p == 0) bar_sync512();
+      if (hl > 0 && real) {
         // signal head: D = H_S - lambda H_N, Y = sigmoid(G) D
-        ok = mbar_wait(smem_u32(&bars.hn_ready), 0, a.status, 224, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          failed = true;
-          break;
-        }
-        const int sh = head_of(hl);  // signal head index
-        const long tok = (long)b * a.q_len + (i - a.q_start);
         const float lam = row_ok ? sigmoidf_(a.lam[tok * n_S + sh]) : 0.f;
         const __nv_bfloat16* gp = a.gate + (tok * n_S + sh) * DV + cbase;
         __nv_bfloat16* op = a.out + (tok * n_S + sh) * DV + cbase;
@@ -564,6 +596,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int q = 0; q < 2; ++q) reinterpret_cast<uint4*>(op + ch * 16)[q] = ov[q];
           }
         }
+      }
+      if (next) {
+        // O of this pair is read: the next pair's rotary Q chunk, then its S MMAs may start
+        load_rope();
+        tc_fence_before();
+        if (bar_or512(!move_q(p + 1, 2))) {
+          failed = true;
+          break;
+        }
+        q_done();
       }
     }
     if (failed) abort_flag = 1;
