@@ -19,7 +19,8 @@ Beside the timed steps (measured after them, outside their timed region):
     where it follows the power-capped prefill;
   * `prefill_cfg2` (B=4 L=4096 g=2 causal), `prefill_cfg4` (B=2 L=65536 g=2,
     4096-token window) and the report's own layout, g=4 (80 heads):
-    `prefill_g4_swa128` (128-token window) and `decode_g4`;
+    `prefill_g4_swa128` (128-token window), `decode_g4`, and `gates` (gate and lambda
+    logits for the bench prefill's tokens);
   * `e2e`: the same prefill through gdla_prefill_host (activations start in
     page-locked host memory, Y ends there; the chunked copies overlap the
     kernels), and `e2e.decode`: q, lambda and gate copied in from page-locked
@@ -137,6 +138,8 @@ def hbm_roofline(gbs: float, pk: dict) -> dict:
             "peak_kind": "measured copy" + (" (fallback)" if pk.get("fallback") else ""),
             "frac_of_nominal": gbs / NOMINAL_HBM_GBS}
 
+
+GATE_D_X = 2048  # width of the layer input x of the lambda projection (the caller's choice)
 
 # The cpu_baseline leg and the reference arm time the oracle on the same sample.
 ORACLE_ROWS = 24
@@ -444,6 +447,20 @@ def run_ours(a):
         if int(gdla.workspace_status(ws4)) != 0:
             raise RuntimeError("device status word reports a failed wait (decode g=4)")
         extra_ms["decode_g4"] = ("b64_t32k_g4", S, t4, None)
+        # the gate logits (tensor cores) and lambda logits (HBM-bound) for the bench
+        # prefill's tokens, with a 2048-wide layer input
+        gi = wl.make_gate_inputs(P, d_x=GATE_D_X, seed=rank_seed(a.seed, rank, "prefill") + 7, device=dev)
+        g_out = torch.empty((P.B, P.L, P.n_S, P.d_v), dtype=torch.bfloat16, device=dev)
+        l_out = torch.empty((P.B, P.L, P.n_S), dtype=torch.float32, device=dev)
+
+        def gate_call():
+            gdla.gates(gi["c_q"], gi["gamma_q"], gi["w_g"], n_signal=P.n_S, d_v=P.d_v, gate_out=g_out)
+
+        def lam_call():
+            gdla.gates(x=gi["x"], w_lambda=gi["w_lambda"], n_signal=P.n_S, lam_out=l_out)
+        extra_ms["gates"] = ("gates", None, time_loop(gate_call, 5, 3, stream), time_loop(lam_call, 10, 3, stream))
+        del gi, g_out, l_out
+        torch.cuda.empty_cache()
 
     vals = [t_exp, t_att, t_dec, t_step, t_dec_alone, t_e2e, t_e2e_dec]
     for key in sorted(extra_ms):
@@ -471,7 +488,16 @@ def run_ours(a):
         name, S, t_first, t_second = extra_ms[key]
         te, ta = vals[i], vals[i + 1]
         i += 2
-        if t_second is None:  # a decode workload
+        if key == "gates":
+            f_g = 2.0 * P.B * P.L * P.d_q * P.n_S * P.d_v
+            b_l = P.B * P.L * (GATE_D_X * 2 + P.n_S * 4) + GATE_D_X * P.n_S * 2
+            extras[key] = {"workload": f"gate and lambda logits, B={P.B} L={P.L}, d_q={P.d_q}, n_S={P.n_S}, "
+                                       f"d_v={P.d_v}, d_x={GATE_D_X}",
+                           "gate_ms": te, "gate_tflops": weak_scaling_value(f_g, world, te * 1e-3) / 1e12,
+                           "gate_roofline": tensor_roofline(f_g / (te * 1e-3) / 1e12, pk),
+                           "lambda_ms": ta, "lambda_gbs": weak_scaling_value(b_l, world, ta * 1e-3) / 1e9,
+                           "lambda_roofline": hbm_roofline(b_l / (ta * 1e-3) / 1e9, pk)}
+        elif t_second is None:  # a decode workload
             gbs = weak_scaling_value(S.algorithmic_bytes(), world, te * 1e-3) / 1e9
             extras[key] = {"workload": S.name, "value": gbs, "unit": "GB/s", "ms": te,
                            "roofline": hbm_roofline(gbs / world, pk)}

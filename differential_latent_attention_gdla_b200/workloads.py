@@ -190,6 +190,22 @@ def make_prefill_inputs(shape: PrefillShape, seed: int = 0, device="cpu", act: s
     return out
 
 
+def make_gate_inputs(shape: PrefillShape, d_x: int = 2048, seed: int = 0, device="cpu"):
+    """Random inputs of the gate and lambda projections for the token layout of
+    ``shape``: c_q [B,L,d_q] (query latent), gamma_q [d_q] = 1 + 0.1 N(0,1),
+    w_g [d_q, n_S*d_v] ~ N(0,1)/sqrt(d_q), x [B,L,d_x] (layer input; its width is
+    the caller's), w_lambda [d_x, n_S] ~ N(0,1)/sqrt(d_x)."""
+    dt = torch_dtype(shape.dtype)
+    gen = _gen(seed, device)
+    out = {}
+    out["c_q"] = _randn((shape.B, shape.L, shape.d_q), gen, device, 1.0, dt)
+    out["gamma_q"] = (_randn((shape.d_q,), gen, device, 0.1) + 1.0).to(dt)
+    out["w_g"] = _randn((shape.d_q, shape.n_S * shape.d_v), gen, device, 1.0 / math.sqrt(shape.d_q), dt)
+    out["x"] = _randn((shape.B, shape.L, d_x), gen, device, 1.0, dt)
+    out["w_lambda"] = _randn((d_x, shape.n_S), gen, device, 1.0 / math.sqrt(d_x), dt)
+    return out
+
+
 def make_decode_inputs(shape: DecodeShape, seed: int = 0, device="cpu", act: str = "fan_in", seqlens=None):
     """Random decode inputs for ``shape`` (dict of tensors on ``device``).
 
