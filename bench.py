@@ -140,6 +140,7 @@ def hbm_roofline(gbs: float, pk: dict) -> dict:
 
 
 GATE_D_X = 2048  # width of the layer input x of the lambda projection (the caller's choice)
+DECODE_WARMUP, DECODE_STEPS = 50, 100  # the decode's own loop (a call is ~0.5 ms)
 
 # The cpu_baseline leg and the reference arm time the oracle on the same sample.
 ORACLE_ROWS = 24
@@ -382,7 +383,9 @@ def run_ours(a):
 
     # ---- measured after the timed steps, outside their region
     # the decode call alone, in its own loop after its own warm-up
-    t_dec_alone = time_loop(decode, a.steps, a.warmup, stream)
+    # its own warm-up long enough (~25 ms) for the clocks to leave the prefill's
+    # power-capped operating point, then 100+ calls
+    t_dec_alone = time_loop(decode, max(a.steps, DECODE_STEPS), max(a.warmup, DECODE_WARMUP), stream)
     if int(gdla.workspace_status(dws)) != 0:
         raise RuntimeError("device status word reports a failed wait (decode)")
 
@@ -443,7 +446,7 @@ def run_ours(a):
             torch.cuda.empty_cache()
         S = wl.DECODE["b64_t32k_g4"]
         _, _, _, ws4, dec4 = decode_case(S, rank_seed(a.seed, rank, "decode"))
-        t4 = time_loop(dec4, 10, 3, stream)
+        t4 = time_loop(dec4, DECODE_STEPS, DECODE_WARMUP, stream)
         if int(gdla.workspace_status(ws4)) != 0:
             raise RuntimeError("device status word reports a failed wait (decode g=4)")
         extra_ms["decode_g4"] = ("b64_t32k_g4", S, t4, None)
