@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const float2 hf = __bfloat1622float2(h2[e]);
               const float y0 = __uint_as_float(o[2 * e]) * inv;
               const float y1 = __uint_as_float(o[2 * e + 1]) * inv;
-              ow[e] = pack_bf16x2(sigmoidf_(gf.x) * (y0 - lam * hf.x), sigmoidf_(gf.y) * (y1 - lam * hf.y));
+              ow[e] = pack_bf16x2(sigmoid_tanh(gf.x) * (y0 - lam * hf.x), sigmoid_tanh(gf.y) * (y1 - lam * hf.y));
             }
 #pragma unroll
             for (int q = 0; q < 2; ++q) reinterpret_cast<uint4*>(op + ch * 16)[q] = ov[q];

@@ -19,6 +19,14 @@ template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
+// sigma(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh approximation (one special-function
+// operation instead of an exponential and a reciprocal; relative error ~2^-11, below the
+// bf16 rounding of the values it scales)
+__device__ __forceinline__ float sigmoid_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
 
 constexpr float kLog2e = 1.4426950408889634f;
 
