@@ -1043,7 +1043,7 @@ __global__ void __launch_bounds__(512, 1)
       for (int q = 0; q < 4; ++q) {
         const float2 gf = __bfloat1622float2(g2[q]);
         const float d0 = hsr[2 * q] - lamv * hnr[2 * q], d1 = hsr[2 * q + 1] - lamv * hnr[2 * q + 1];
-        o[q] = pack_bf16x2(d0 / (1.f + __expf(-gf.x)), d1 / (1.f + __expf(-gf.y)));
+        o[q] = pack_bf16x2(d0 * sigmoid_tanh(gf.x), d1 * sigmoid_tanh(gf.y));
       }
       *reinterpret_cast<uint4*>(a.out + idx) = make_uint4(o[0], o[1], o[2], o[3]);
     }
