@@ -3,7 +3,7 @@
 // Report", Architecture: RoPE only on the rotary parts; signal and noise heads
 // attend independently; D = H_S - lambda (.) Repeat_g(H_N); Y = sigmoid(G) (.) D).
 //
-// One CTA owns (sequence b, KV group h, 64 query rows) and every head that
+// A work item is (sequence b, KV group h, 64 query rows) with every head that
 // reads KV head h: the noise head and its g signal heads, taken two at a time:
 //   pair 0 = (noise, signal 0), pair 1 = (signal 1, signal 2), ...
 // The two heads of a pair are stacked into one 128-row operand (rows 0-63 the
@@ -12,8 +12,13 @@
 // (K = 128 keys, N = 128 value dims), and every K/V tile brought in from L2
 // serves both heads. Both Q (rotated once per pair) and P live in TMEM, so the
 // tensor core reads only K and V from shared memory.
+// The kernel is persistent: one CTA per SM takes work items from a global counter
+// (KV-group-major, heaviest query blocks first) until none is left, so the set-up of a
+// CTA happens once and the next item's Q, K and V copies overlap the current item's
+// last tiles and epilogue; items reach the other roles through a 2-slot ring in shared
+// memory that the producer fills.
 // Warp roles (640 threads):
-//   warp 0      TMA producer: the pair's Q in three 64-dim chunks through a
+//   warp 0      work items; TMA producer: the pair's Q in three 64-dim chunks through a
 //               2-deep staging ring; K tiles (128 keys x 192) and V tiles
 //               (128 keys x 128), each in a 2-deep ring;
 //   warp 1      MMA issuer (one lane): S(j) into S buffer j % 2, then
@@ -71,6 +76,8 @@ struct Bars {
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2], q_full[2], q_free[2];
   uint64_t s_full[2], p_full[2];
   uint64_t pv_done, q_ready, o_full, mma_done;
+  uint64_t item_full[2], item_free[2];  // the ring of work items the producer fetches
+  int item[2];
   uint32_t tmem_slot;
   int abort_flag;
   int skip_cta;
@@ -89,6 +96,8 @@ __device__ __forceinline__ uint32_t hn_off(int r, int c) { return (uint32_t)(r *
 
 struct AttnTcArgs {
   int B, L, n_kv, g, sliding, window, rope_max_pos, n_qtiles;
+  int n_items;  // (sequence, KV group, 64-row query block) work items
+  int* work;    // the next work item (zero before the launch)
   int q_len, q_start;  // query rows: positions q_start .. q_start+q_len-1; keys: 0 .. L-1
   float sl2;  // tau * log2(e)
   const float* cos_tab;
@@ -125,23 +134,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int G1 = a.g + 1;
   const int n_pairs = (G1 + 1) / 2;
   const int n_S = a.g * a.n_kv;
-  // KV-group-major order, heaviest query blocks first within a group: the CTAs
-  // resident at one time stream the K/V of one or two groups, which stay in L2
-  const int t = blockIdx.x;
-  const int m_idx = a.n_qtiles - 1 - t % a.n_qtiles;
-  const int h = (t / a.n_qtiles) % a.n_kv;
-  const int b = t / (a.n_qtiles * a.n_kv);
-  const int m_loc = m_idx * BM;           // first query row of the block within the q/Y tensors
-  const int m0 = a.q_start + m_loc;       // its position in the sequence
   const int q_end = a.q_start + a.q_len;  // one past the last query position
-  const int last_row = min(q_end - 1, m0 + BM - 1);
-  const int key_lo = a.sliding ? max(0, m0 - a.window + 1) : 0;
-  const int j_lo = key_lo / BN;
-  const int n_tiles = last_row / BN - j_lo + 1;
-
-  auto head_of = [&](int hl) { return hl == 0 ? n_S + h : h * a.g + hl - 1; };
+  // Work item t: KV-group-major order, heaviest query blocks first within a group, handed
+  // out dynamically, so that the CTAs running at one time stream the K/V of one or two
+  // groups, which stay in L2, and every SM stays busy to the end
+  struct Item {
+    int b, h, m_loc, m0, j_lo, n_tiles;
+  };
+  auto item_of = [&](int t) {
+    Item it;
+    const int m_idx = a.n_qtiles - 1 - t % a.n_qtiles;
+    it.h = (t / a.n_qtiles) % a.n_kv;
+    it.b = t / (a.n_qtiles * a.n_kv);
+    it.m_loc = m_idx * BM;       // first query row of the block within the q/Y tensors
+    it.m0 = a.q_start + it.m_loc;  // its position in the sequence
+    const int last_row = min(q_end - 1, it.m0 + BM - 1);
+    const int key_lo = a.sliding ? max(0, it.m0 - a.window + 1) : 0;
+    it.j_lo = key_lo / BN;
+    it.n_tiles = last_row / BN - it.j_lo + 1;
+    return it;
+  };
+  auto head_of = [&](int h, int hl) { return hl == 0 ? n_S + h : h * a.g + hl - 1; };
   // head in half s of pair p; a pair without a second head repeats the first (its rows are discarded)
-  auto head_in = [&](int p, int s) { return head_of(2 * p + s < G1 ? 2 * p + s : 2 * p); };
+  auto head_in = [&](int h, int p, int s) { return head_of(h, 2 * p + s < G1 ? 2 * p + s : 2 * p); };
+  // the consumers' side of the work ring: item k sits in slot k & 1
+  auto take_item = [&](int k, bool& ok) -> int {
+    const int sl = k & 1;
+    ok = ok && mbar_wait(smem_u32(&bars.item_full[sl]), (k >> 1) & 1, a.status, 231, &abort_flag);
+    return ok ? *reinterpret_cast<volatile int*>(&bars.item[sl]) : -1;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -158,6 +179,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(smem_u32(&bars.q_ready), 4 * NWG);
     mbar_init(smem_u32(&bars.o_full), 1);
     mbar_init(smem_u32(&bars.mma_done), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars.item_full[i]), 1);
+      mbar_init(smem_u32(&bars.item_free[i]), 1 + 4 * NWG);  // the MMA issuer and the 16 softmax warps
+    }
     // the softmax warps arrive once per warp (q_free, q_ready, p_full)
     fence_mbar_init();
     abort_flag = 0;
@@ -183,22 +208,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       int kc = 0, vc = 0, qk = 0;  // K / V / Q-chunk loads issued so far (ring position and phase)
       bool ok = true;
+      Item it{};
       auto load_k = [&](int jj) -> bool {
         const int sl = kc & 1;
         if (kc >= 2 && !mbar_wait(smem_u32(&bars.k_empty[sl]), ((kc >> 1) & 1) ^ 1, a.status, 202, &abort_flag)) return false;
-        const int key0 = (j_lo + jj) * BN;
+        const int key0 = (it.j_lo + jj) * BN;
         uint8_t* ks = k_sm + sl * K_BYTES;
         const uint32_t bar = smem_u32(&bars.k_full[sl]);
         mbar_expect_tx(bar, K_BYTES);
-        tma_load_4d(smem_u32(ks), &tmKV, bar, 0, h, key0, b);
-        tma_load_4d(smem_u32(ks + K_CHUNK), &tmKV, bar, 64, h, key0, b);
-        tma_load_3d(smem_u32(ks + 2 * K_CHUNK), &tmKR, bar, 0, key0, b);
-        if (jj + kPrefetch < n_tiles) {
+        tma_load_4d(smem_u32(ks), &tmKV, bar, 0, it.h, key0, it.b);
+        tma_load_4d(smem_u32(ks + K_CHUNK), &tmKV, bar, 64, it.h, key0, it.b);
+        tma_load_3d(smem_u32(ks + 2 * K_CHUNK), &tmKR, bar, 0, key0, it.b);
+        if (jj + kPrefetch < it.n_tiles) {
           // bring the tile kPrefetch ahead into L2, so that its ring load later hits
           const int key1 = key0 + kPrefetch * BN;
-          tma_prefetch_4d(&tmKV, 0, h, key1, b);
-          tma_prefetch_4d(&tmKV, 64, h, key1, b);
-          tma_prefetch_3d(&tmKR, 0, key1, b);
+          tma_prefetch_4d(&tmKV, 0, it.h, key1, it.b);
+          tma_prefetch_4d(&tmKV, 64, it.h, key1, it.b);
+          tma_prefetch_3d(&tmKR, 0, key1, it.b);
         }
         ++kc;
         return true;
@@ -206,16 +232,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto load_v = [&](int jj) -> bool {
         const int sl = vc & 1;
         if (vc >= 2 && !mbar_wait(smem_u32(&bars.v_empty[sl]), ((vc >> 1) & 1) ^ 1, a.status, 203, &abort_flag)) return false;
-        const int key0 = (j_lo + jj) * BN;
+        const int key0 = (it.j_lo + jj) * BN;
         uint8_t* vs = v_sm + sl * V_BYTES;
         const uint32_t bar = smem_u32(&bars.v_full[sl]);
         mbar_expect_tx(bar, V_BYTES);
-        tma_load_4d(smem_u32(vs), &tmKV, bar, DN, h, key0, b);
-        tma_load_4d(smem_u32(vs + V_BLOCK), &tmKV, bar, DN + 64, h, key0, b);
-        if (jj + kPrefetch < n_tiles) {
+        tma_load_4d(smem_u32(vs), &tmKV, bar, DN, it.h, key0, it.b);
+        tma_load_4d(smem_u32(vs + V_BLOCK), &tmKV, bar, DN + 64, it.h, key0, it.b);
+        if (jj + kPrefetch < it.n_tiles) {
           const int key1 = key0 + kPrefetch * BN;
-          tma_prefetch_4d(&tmKV, DN, h, key1, b);
-          tma_prefetch_4d(&tmKV, DN + 64, h, key1, b);
+          tma_prefetch_4d(&tmKV, DN, it.h, key1, it.b);
+          tma_prefetch_4d(&tmKV, DN + 64, it.h, key1, it.b);
         }
         ++vc;
         return true;
@@ -227,20 +253,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t bar = smem_u32(&bars.q_full[sl]);
         mbar_expect_tx(bar, QS_BYTES);
         for (int s = 0; s < 2; ++s)
-          tma_load_4d(smem_u32(qs_sm + sl * QS_BYTES + s * (BM * 128)), &tmQ, bar, k * 64, head_in(p, s), m_loc, b);
+          tma_load_4d(smem_u32(qs_sm + sl * QS_BYTES + s * (BM * 128)), &tmQ, bar, k * 64, head_in(it.h, p, s),
+                      it.m_loc, it.b);
         ++qk;
         return true;
       };
-      for (int p = 0; p < n_pairs && ok && !abort_flag; ++p) {
-        // the last Q chunk reuses the staging buffer of the first, which the softmax
-        // warps free only after the previous pair's epilogue: K(0), K(1) go first
-        ok = load_q(p, 0) && load_q(p, 1);
-        // consumption order of the tensor core: S(0), S(1), PV(0), S(2), PV(1), ...
-        if (ok) ok = load_k(0) && (n_tiles < 2 || load_k(1));
-        if (ok) ok = load_q(p, 2);
-        for (int jj = 0; jj < n_tiles && ok; ++jj) {
-          ok = load_v(jj);
-          if (ok && jj + 2 < n_tiles) ok = load_k(jj + 2);
+      // work items: fetched one ahead into the 2-slot ring (a slot is free again once the
+      // issuer and the softmax warps have read it); -1 ends the work of every role
+      for (int ki = 0; ok && !abort_flag; ++ki) {
+        const int sl = ki & 1;
+        if (ki >= 2 && !mbar_wait(smem_u32(&bars.item_free[sl]), ((ki >> 1) - 1) & 1, a.status, 204, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        int t = atomicAdd(a.work, 1);
+        if (t >= a.n_items) t = -1;
+        bars.item[sl] = t;
+        mbar_arrive(smem_u32(&bars.item_full[sl]));
+        if (t < 0) break;
+        it = item_of(t);
+        for (int p = 0; p < n_pairs && ok && !abort_flag; ++p) {
+          // the last Q chunk reuses the staging buffer of the first, which the softmax
+          // warps free only after the previous pair's epilogue: K(0), K(1) go first
+          ok = load_q(p, 0) && load_q(p, 1);
+          // consumption order of the tensor core: S(0), S(1), PV(0), S(2), PV(1), ...
+          if (ok) ok = load_k(0) && (it.n_tiles < 2 || load_k(1));
+          if (ok) ok = load_q(p, 2);
+          for (int jj = 0; jj < it.n_tiles && ok; ++jj) {
+            ok = load_v(jj);
+            if (ok && jj + 2 < it.n_tiles) ok = load_k(jj + 2);
+          }
         }
       }
       if (!ok) {
@@ -297,18 +339,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ++vc;
         return true;
       };
-      for (int p = 0; p < n_pairs && ok; ++p) {
-        // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
-        ok = mbar_wait(smem_u32(&bars.q_ready), p & 1, a.status, 211, &abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        ok = issue_s() && (n_tiles < 2 || issue_s());
-        for (int jj = 0; jj < n_tiles && ok; ++jj) {
-          ok = issue_pv(jj);
-          if (ok && jj + 2 < n_tiles) ok = issue_s();
+      int gp = 0;  // head pairs over the whole CTA (q_ready / o_full phases)
+      for (int ki = 0; ok; ++ki) {
+        const int t = take_item(ki, ok);
+        if (ok) mbar_arrive(smem_u32(&bars.item_free[ki & 1]));
+        if (!ok || t < 0) break;
+        const int n_tiles = item_of(t).n_tiles;
+        for (int p = 0; p < n_pairs && ok; ++p, ++gp) {
+          // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
+          ok = mbar_wait(smem_u32(&bars.q_ready), gp & 1, a.status, 211, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          ok = issue_s() && (n_tiles < 2 || issue_s());
+          for (int jj = 0; jj < n_tiles && ok; ++jj) {
+            ok = issue_pv(jj);
+            if (ok && jj + 2 < n_tiles) ok = issue_s();
+          }
+          if (!ok) break;
+          mma_commit(smem_u32(&bars.o_full));
         }
-        if (!ok) break;
-        mma_commit(smem_u32(&bars.o_full));
       }
       if (!ok) abort_flag = 1;
       // every MMA this thread issued has completed before TMEM is released
@@ -324,16 +373,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q4 = warp & 3;                // TMEM lane quadrant
     const int r = q4 * 32 + lane;           // stacked row = TMEM lane
     const int half = r >> 6;                // 0: first head of the pair, 1: second
-    const int i = m0 + (r & (BM - 1));      // query position
-    const bool row_ok = i < q_end;
+    Item it{};
+    int i = 0;                              // this row's query position in the current item
+    bool row_ok = false;
+    int rope_pos = 0;
+    auto set_rows = [&]() {
+      i = it.m0 + (r & (BM - 1));
+      row_ok = i < q_end;
+      rope_pos = row_ok ? i : q_end - 1;  // rows past the end are discarded; any table row will do
+    };
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const uint32_t tO = tmem + lane_base + kColO + CW * c;
     const uint32_t tQ = tmem + lane_base + kColQ;
-    // this row's RoPE factors for rotary dims 8c .. 8c+7 (the same positions in every
-    // pair), loaded ahead of each pair's rotary chunk (volatile: live only between the
-    // load and that chunk, not across the key tiles)
+    // this row's RoPE factors for rotary dims 8c .. 8c+7, loaded ahead of each pair's
+    // rotary chunk (volatile: live only between the load and that chunk, not across the
+    // key tiles)
     float cs[8], sn[8];
-    const int rope_pos = row_ok ? i : q_end - 1;  // rows past the end are discarded; any table row will do
     auto load_rope = [&]() {
       const float* cp = a.cos_tab + (long)rope_pos * (DR / 2) + 8 * c;
       const float* sp = a.sin_tab + (long)rope_pos * (DR / 2) + 8 * c;
@@ -343,7 +398,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(sn[e]) : "l"(sp + e));
       }
     };
-    load_rope();
     // chunk k of pair p's stacked Q rows into TMEM: thread c moves dims 16c .. 16c+15 of a
     // content chunk, or rotates dims 8c .. 8c+7 with 32+8c .. 32+8c+7 of the rotary chunk
     auto move_q = [&](int p, int k) -> bool {
@@ -385,20 +439,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_arrive_warp(smem_u32(&bars.q_ready));
     };
     int tc = 0;                             // tiles processed over the whole CTA
+    int ki = 0, gp = 0;                     // work items taken, head pairs begun over the whole CTA
+    // the next work item from the ring (every softmax thread; the slot is released at once)
+    auto next_item = [&](bool& ok) -> int {
+      const int t = take_item(ki, ok);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) mbar_arrive_warp(smem_u32(&bars.item_free[ki & 1]));
+      ++ki;
+      return t;
+    };
     bool failed = false;
+    int t = -1;
     {
       bool ok = true;
-      for (int k = 0; k < 3; ++k) ok = move_q(0, k) && ok;
+      t = next_item(ok);
       failed = bar_or512(!ok);
-      if (!failed) q_done();
+      if (!failed && t >= 0) {
+        it = item_of(t);
+        set_rows();
+        load_rope();
+        for (int k = 0; k < 3; ++k) ok = move_q(0, k) && ok;
+        failed = bar_or512(!ok);
+        if (!failed) q_done();
+      }
     }
-    for (int p = 0; p < n_pairs && !failed; ++p) {
+    for (int p = 0; t >= 0 && !failed;) {
       const int hl = 2 * p + half;
       const int cbase = CW * c;             // this warpgroup finishes value columns [cbase, cbase + 32)
       const bool real = hl < G1;            // the second half of a short last pair is discarded
-      const bool next = p + 1 < n_pairs;
-      const int sh = hl > 0 ? head_of(hl) : 0;  // signal head index
-      const long tok = (long)b * a.q_len + (i - a.q_start);
+      const int sh = hl > 0 ? head_of(it.h, hl) : 0;  // signal head index
+      const long tok = (long)it.b * a.q_len + (i - a.q_start);
+      const int m0 = it.m0, j_lo = it.j_lo, n_tiles = it.n_tiles;
       if (hl > 0 && real && row_ok) {
         // the epilogue's gate and lambda of this row: into L2 while the key tiles stream
         prefetch_l2(a.gate + (tok * n_S + sh) * DV + cbase);
@@ -516,18 +587,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
       // ---------------------------------------------------------- epilogue
       {
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.o_full), p & 1, a.status, 223, &abort_flag));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.o_full), gp & 1, a.status, 223, &abort_flag));
         if (bar_or512(!ok)) {
           failed = true;
           break;
         }
       }
       tc_fence_after();
+      // the next head pair: the item's next one, or the next item's first
+      int t_next = t, p_next = p + 1;
+      if (p_next == n_pairs) {
+        bool ok = true;
+        t_next = next_item(ok);
+        p_next = 0;
+        if (bar_or512(!ok)) {
+          failed = true;
+          break;
+        }
+      }
+      const bool next = t_next >= 0;
       if (next) {
         // every S MMA of this pair is done, so the next pair's Q content chunks may go into
         // TMEM now; its rotary chunk follows the epilogue, while that copy lands
-        bool ok = move_q(p + 1, 0);
-        ok = move_q(p + 1, 1) && ok;
+        bool ok = move_q(gp + 1, 0);
+        ok = move_q(gp + 1, 1) && ok;
         if (bar_or512(!ok)) {
           failed = true;
           break;
@@ -598,15 +681,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (next) {
-        // O of this pair is read: the next pair's rotary Q chunk, then its S MMAs may start
+        // O of this pair is read: the next pair's rotary Q chunk (at the positions of the
+        // next item's rows when the item changes), then its S MMAs may start
+        if (p_next == 0) {
+          it = item_of(t_next);
+          set_rows();
+        }
         load_rope();
         tc_fence_before();
-        if (bar_or512(!move_q(p + 1, 2))) {
+        if (bar_or512(!move_q(gp + 1, 2))) {
           failed = true;
           break;
         }
         q_done();
       }
+      t = t_next;
+      p = p_next;
+      ++gp;
     }
     if (failed) abort_flag = 1;
   }
@@ -651,10 +742,19 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   a.gate = reinterpret_cast<const __nv_bfloat16*>(p.gate);
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
   a.status = p.status;
+  a.work = p.work;
+  const long n_items = (long)a.n_qtiles * p.n_kv * p.B;
+  if (n_items > INT_MAX) return cudaErrorInvalidValue;
+  a.n_items = (int)n_items;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const long nblocks = (long)a.n_qtiles * p.n_kv * p.B;
-  attn_tc_kernel<<<(unsigned)nblocks, NTHREADS, SMEM_BYTES, s>>>(tq, tkv, tkr, a);
+  // persistent: one CTA per SM takes work items until none is left
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(p.work, 0, sizeof(int), s)) != cudaSuccess) return e;
+  const int grid = (int)(n_items < sms ? n_items : sms);
+  attn_tc_kernel<<<(unsigned)grid, NTHREADS, SMEM_BYTES, s>>>(tq, tkv, tkr, a);
   return cudaGetLastError();
 }
 

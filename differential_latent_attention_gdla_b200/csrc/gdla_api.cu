@@ -345,7 +345,13 @@ gdla_status gdla_latent_expand(const gdla_expand_args* a, void* stream) {
   return cuda_status(expand_rows(a, (long)a->B * a->L, a->L, 0, nullptr, (cudaStream_t)stream));
 }
 
-static gdla_status attend_impl(const gdla_attend_args* a, cudaStream_t s, bool clear_status) {
+// The status area (kStatusBytes at the workspace start) holds the status word (ints 0, 1)
+// and, from int kWorkCounterInt, one work-item counter per stream that may run an attention
+// launch at the same time as another (the persistent tensor-core kernel hands out its items
+// through it; each launch zeroes its own counter on its own stream first).
+constexpr int kWorkCounterInt = 16;
+static_assert((kWorkCounterInt + kComputeStreams) * sizeof(int) <= kStatusBytes, "work counters in the status area");
+static gdla_status attend_impl(const gdla_attend_args* a, cudaStream_t s, bool clear_status, int counter = 0) {
   AttnParams ap{};
   ap.B = a->B; ap.L = a->L; ap.n_kv = a->n_kv; ap.g = a->g; ap.d_nope = a->d_nope; ap.d_rope = a->d_rope;
   ap.d_v = a->d_v; ap.sliding = a->mask == GDLA_MASK_SLIDING; ap.window = ap.sliding ? a->window : 0;
@@ -353,6 +359,7 @@ static gdla_status attend_impl(const gdla_attend_args* a, cudaStream_t s, bool c
   ap.rope_max_pos = a->rope_max_pos; ap.scale = default_scale(a->softmax_scale, a->d_nope, a->d_rope);
   ap.q = a->q; ap.kv = a->kv; ap.kr = a->k_rope_rot; ap.cos_tab = a->rope_cos; ap.sin_tab = a->rope_sin;
   ap.lam = a->lam_logits; ap.gate = a->gate_logits; ap.out = a->out; ap.status = (int*)a->workspace;
+  ap.work = (int*)a->workspace + kWorkCounterInt + counter;
   cudaError_t e = cudaSuccess;
   if (clear_status) e = cudaMemsetAsync(a->workspace, 0, kStatusBytes, s);
   if (e != cudaSuccess) return cuda_status(e);
@@ -563,7 +570,7 @@ gdla_status gdla_prefill_host(const gdla_prefill_args* a, int chunk_tokens, void
         aa.L = t0 + n; aa.q_len = n; aa.q_start = t0;
         aa.q = d_q; aa.lam_logits = (const float*)d_lam; aa.gate_logits = d_gate; aa.out = d_out;
         aa.kv = kv + (size_t)b * a->L * b_kv; aa.k_rope_rot = k_rot + (size_t)b * a->L * b_kr;
-        const gdla_status as = attend_impl(&aa, cs, /*clear_status=*/false);
+        const gdla_status as = attend_impl(&aa, cs, /*clear_status=*/false, (int)(k % kComputeStreams));
         if (as != GDLA_OK) e = cudaErrorLaunchFailure;
       }
       if (e == cudaSuccess) e = cudaEventRecord(ev_comp[sl], cs);

@@ -52,6 +52,7 @@ struct AttnParams {
   const void* gate;     // [B, q_len, n_S, d_v]
   void* out;            // [B, q_len, n_S, d_v]
   int* status;
+  int* work;            // the tensor-core kernel's work-item counter (zeroed on the launch stream)
 };
 cudaError_t launch_attn_simt(const AttnParams& p, gdla_dtype dt, cudaStream_t s);
 // shapes the tcgen05/TMA attention takes (bf16, heads of 128 + 64 rotary, d_v = 128)
