@@ -13,10 +13,15 @@
 //   warp 1      MMA issuer (one lane): tcgen05.mma 128 x BN x 16 into one of two
 //               TMEM accumulators (BN columns each), alternating per tile;
 //   warps 4-7   epilogue: warp w drains TMEM lanes 32(w-4) .. +31 (one output row
-//               per thread) of the finished accumulator and stores the row, while
-//               the MMAs of the next tile fill the other accumulator.
+//               per thread) of the finished accumulator while the MMAs of the next
+//               tile fill the other accumulator. bf16 output goes 64 columns at a
+//               time through a double-buffered, 128-byte-swizzled 32 x 64 staging box
+//               per warp and leaves by TMA store (whole lines, asynchronous); fp32
+//               output is stored from registers (16-byte pieces of each row).
 // Tails: rows of A beyond M and columns of B beyond N are zero-filled by TMA and
 // not stored; a K that is not a multiple of 64 is zero-filled the same way.
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -32,7 +37,9 @@ struct Cfg {
   static constexpr int A_BYTES = GM * GK * 2;  // 16 KB
   static constexpr int B_BYTES = GK * BN * 2;  // BN/64 boxes of 8 KB
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int OFF_BARS = STAGES * STAGE;
+  static constexpr int OFF_EPI = STAGES * STAGE;       // bf16 output staging: 4 warps x 2 x [32 x 128 B]
+  static constexpr int EPI_BYTES = 4 * 2 * 32 * 128;
+  static constexpr int OFF_BARS = OFF_EPI + EPI_BYTES;
   static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
   static_assert(BN % 64 == 0 && BN <= 256, "B is loaded in 64-column boxes; one MMA covers N <= 256");
   static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation: a power of two <= 512");
@@ -83,7 +90,7 @@ struct GemmTcArgs {
 template <int BN, int STAGES, typename OutT>
 __global__ void __launch_bounds__(gtc::GTHREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmTcArgs a) {
+                   const __grid_constant__ CUtensorMap tmC, const GemmTcArgs a) {
   using namespace sm100;
   using namespace gtc;
   using C_ = Cfg<BN, STAGES>;
@@ -199,6 +206,9 @@ __global__ void __launch_bounds__(gtc::GTHREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int q4 = warp - 4;
     OutT* C = reinterpret_cast<OutT*>(a.C);
+    constexpr bool kTmaOut = std::is_same<OutT, __nv_bfloat16>::value;
+    uint8_t* stg = smem + C_::OFF_EPI + q4 * 8192;  // this warp's two 4 KB staging boxes
+    int nb = 0;                                      // 64-column chunks this warp has stored
     for (int i = 0; i < my_tiles; ++i) {
       const int buf = i & 1;
       bool ok = mbar_wait(smem_u32(&bars.acc_full[buf]), (i >> 1) & 1, a.status, 103, &abort_flag);
@@ -208,19 +218,54 @@ __global__ void __launch_bounds__(gtc::GTHREADS, 1)
       }
       tc_fence_after();
       const long t = blockIdx.x + (long)i * gridDim.x;
-      const long row = (t / a.n_tn) * GM + q4 * 32 + lane;
+      const long row0 = (t / a.n_tn) * GM + q4 * 32;  // first output row of this warp
       const int n0 = (int)(t % a.n_tn) * BN;
+      const uint32_t tacc = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN);
+      if constexpr (kTmaOut) {
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN + ch * 32), r);
-        tmem_wait_ld();
-        const int c0 = n0 + ch * 32;
-        if (row < a.M && c0 < a.N) store_chunk<OutT>(C + row * a.N + c0, r, a.N - c0);
+        for (int cc = 0; cc < BN / 64; ++cc, ++nb) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tacc + cc * 64, r0);
+          tmem_ld32(tacc + cc * 64 + 32, r1);
+          tmem_wait_ld();
+          const int b = nb & 1;
+          // the store issued from this box two chunks ago has finished reading it
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          // row `lane` of the box: 16-byte piece j (columns 8j .. 8j+7) at slot j ^ (row & 7)
+          uint8_t* rowp = stg + b * 4096 + lane * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* r = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
+            const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                                       pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                                       pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                                       pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+            *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < a.M && n0 + cc * 64 < a.N) tma_store_2d(&tmC, smem_u32(stg + b * 4096), n0 + cc * 64, (int)row0);
+            bulk_commit();
+          }
+        }
+      } else {
+        const long row = row0 + lane;
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(tacc + ch * 32, r);
+          tmem_wait_ld();
+          const int c0 = n0 + ch * 32;
+          if (row < a.M && c0 < a.N) store_chunk<OutT>(C + row * a.N + c0, r, a.N - c0);
+        }
       }
       tc_fence_before();
       mbar_arrive_warp(smem_u32(&bars.acc_empty[buf]));
     }
+    // the output stores have completed before the CTA exits
+    if (kTmaOut && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -245,6 +290,14 @@ static cudaError_t launch_cfg(const GemmParams& p, int* status, cudaStream_t s) 
   const uint32_t bbox[2] = {64, gtc::GK};
   if (!make_tmap_bf16(&ta, p.A, 2, adims, astr, abox) || !make_tmap_bf16(&tb, p.Bm, 2, bdims, bstr, bbox))
     return cudaErrorInvalidValue;
+  // bf16 output: 32 x 64 store boxes (one warp's rows, 128 bytes of columns); the fp32
+  // path stores from registers and does not use the map
+  CUtensorMap tc = tb;
+  if (std::is_same<OutT, __nv_bfloat16>::value) {
+    const uint64_t cdims[2] = {(uint64_t)p.N, (uint64_t)p.M}, cstr[1] = {(uint64_t)p.N * 2};
+    const uint32_t cbox[2] = {64, 32};
+    if (!make_tmap_bf16(&tc, p.C, 2, cdims, cstr, cbox)) return cudaErrorInvalidValue;
+  }
   GemmTcArgs a{};
   a.M = p.M; a.N = p.N; a.K = p.K;
   a.n_tm = (int)((p.M + gtc::GM - 1) / gtc::GM);
@@ -255,7 +308,7 @@ static cudaError_t launch_cfg(const GemmParams& p, int* status, cudaStream_t s) 
   if (e != cudaSuccess) return e;
   const long tiles = (long)a.n_tm * a.n_tn;
   const int grid = (int)(tiles < gtc::kNumSMs ? tiles : gtc::kNumSMs);
-  kern<<<grid, gtc::GTHREADS, SMEM, s>>>(ta, tb, a);
+  kern<<<grid, gtc::GTHREADS, SMEM, s>>>(ta, tb, tc, a);
   return cudaGetLastError();
 }
 

@@ -59,6 +59,14 @@ def test_gates_odd_widths():
     check(inp, 6, 64, torch.bfloat16, "bf16 odd widths")
 
 
+def test_gates_gate_width_not_a_multiple_of_64():
+    # gate: n_S * d_v = 200 columns = three full 64-column store boxes and one of 8 columns,
+    # 90 tokens = a ragged 128-row tile (rows 90 .. 127 are not written); d_q = 136 is a
+    # K tail of the 64-deep block
+    inp = make(2, 45, 136, 72, 5, 40, torch.bfloat16, seed=9)
+    check(inp, 5, 40, torch.bfloat16, "bf16 gate width 200")
+
+
 def test_gates_many_tiles_per_block():
     # 1024 tokens x 6144 gate columns = 192 output tiles of 128 x 256 on 148 blocks, and
     # 40000 tokens of lambda = 313 tiles of 128 x 64 (fp32): both walk several tiles per
