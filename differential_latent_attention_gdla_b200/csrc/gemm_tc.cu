@@ -45,6 +45,20 @@ struct Cfg {
   static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM allocation: a power of two <= 512");
 };
 
+// Pair tiles (two CTAs of a cluster, one M = 256 MMA): each CTA stages its own 128 rows of A
+// and its own 128 of the tile's 256 columns of B, so a K-block brings 32 KB into each SM
+// for 128 x 256 outputs (48 KB for the single-CTA tile)
+template <int STAGES>
+struct PairCfg {
+  static constexpr int BN = 256;                     // output columns of a pair tile
+  static constexpr int A_BYTES = GM * GK * 2;        // 16 KB: this CTA's 128 rows
+  static constexpr int B_BYTES = GK * (BN / 2) * 2;  // 16 KB: this CTA's 128 columns, two 64 x 64 boxes
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int OFF_EPI = STAGES * STAGE;
+  static constexpr int EPI_BYTES = 4 * 2 * 32 * 128;
+  static constexpr int OFF_BARS = OFF_EPI + EPI_BYTES;
+};
+
 template <int STAGES>
 struct Bars {
   uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], mma_done;
@@ -86,6 +100,46 @@ struct GemmTcArgs {
   void* C;
   int* status;
 };
+
+namespace gtc {
+// Drains BN accumulator columns of one warp's 32 rows (TMEM lanes of `tacc`) to global
+// memory: 64 columns at a time into one of the warp's two 4 KB staging boxes (bf16,
+// 128-byte swizzle: 16-byte piece j of row r at slot j ^ (r & 7)), then a TMA store of
+// the box at (row0, n0 + 64 c); rows at or past M and columns at or past N are not
+// written. nb counts the chunks this warp has stored (it picks the staging box).
+template <int BN>
+__device__ __forceinline__ void drain_tma_bf16(uint32_t tacc, uint8_t* stg, int& nb, int lane, long row0, int n0,
+                                               long M, int N, const CUtensorMap* tmC) {
+  using namespace sm100;
+#pragma unroll 1
+  for (int cc = 0; cc < BN / 64; ++cc, ++nb) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(tacc + cc * 64, r0);
+    tmem_ld32(tacc + cc * 64 + 32, r1);
+    tmem_wait_ld();
+    const int b = nb & 1;
+    // the store issued from this box two chunks ago has finished reading it
+    if (lane == 0) bulk_wait_read<1>();
+    __syncwarp();
+    uint8_t* rowp = stg + b * 4096 + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t* r = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
+      const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                                 pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                                 pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                                 pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+      *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (row0 < M && n0 + cc * 64 < N) tma_store_2d(tmC, smem_u32(stg + b * 4096), n0 + cc * 64, (int)row0);
+      bulk_commit();
+    }
+  }
+}
+}  // namespace gtc
 
 template <int BN, int STAGES, typename OutT>
 __global__ void __launch_bounds__(gtc::GTHREADS, 1)
@@ -222,34 +276,7 @@ __global__ void __launch_bounds__(gtc::GTHREADS, 1)
       const int n0 = (int)(t % a.n_tn) * BN;
       const uint32_t tacc = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN);
       if constexpr (kTmaOut) {
-#pragma unroll 1
-        for (int cc = 0; cc < BN / 64; ++cc, ++nb) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tacc + cc * 64, r0);
-          tmem_ld32(tacc + cc * 64 + 32, r1);
-          tmem_wait_ld();
-          const int b = nb & 1;
-          // the store issued from this box two chunks ago has finished reading it
-          if (lane == 0) bulk_wait_read<1>();
-          __syncwarp();
-          // row `lane` of the box: 16-byte piece j (columns 8j .. 8j+7) at slot j ^ (row & 7)
-          uint8_t* rowp = stg + b * 4096 + lane * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t* r = j < 4 ? r0 + 8 * j : r1 + 8 * (j - 4);
-            const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                                       pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                                       pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                                       pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
-            *reinterpret_cast<uint4*>(rowp + ((j ^ (lane & 7)) << 4)) = v;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (row0 < a.M && n0 + cc * 64 < a.N) tma_store_2d(&tmC, smem_u32(stg + b * 4096), n0 + cc * 64, (int)row0);
-            bulk_commit();
-          }
-        }
+        drain_tma_bf16<BN>(tacc, stg, nb, lane, row0, n0, a.M, a.N, &tmC);
       } else {
         const long row = row0 + lane;
 #pragma unroll 1
@@ -271,6 +298,173 @@ __global__ void __launch_bounds__(gtc::GTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, C_::TMEM_COLS);
+}
+
+// The same product on CTA pairs (bf16 output, 256 x 256 tiles): cluster c of two CTAs walks
+// tiles c, c + clusters, ...; rank r's producer stages rows 128 r .. 128 r + 127 of A and
+// columns 128 r .. 128 r + 127 of B's tile, both ranks' copies completing on rank 0's
+// ring barrier; rank 0's MMA warp issues M = 256 x N = 256 x 16 MMAs into a
+// double-buffered accumulator present in both CTAs' TMEM (each CTA's 128 rows, all 256
+// columns) and commits to the ring and accumulator barriers of both CTAs; each CTA's
+// epilogue drains its own rows and reports the drained accumulator to rank 0. Both CTAs
+// reach the cluster barriers at the start and the end whatever happens in between (every
+// other wait is bounded), so neither leaves while the other may still address it.
+template <int STAGES>
+__global__ void __launch_bounds__(gtc::GTHREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const GemmTcArgs a) {
+  using namespace sm100;
+  using namespace gtc;
+  using C_ = PairCfg<STAGES>;
+  constexpr int BN = C_::BN;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  Bars<STAGES>& bars = *reinterpret_cast<Bars<STAGES>*>(smem + C_::OFF_BARS);
+  volatile int& abort_flag = bars.abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  // the dynamic shared-memory base is the same in every CTA, so both CTAs of a pair take
+  // the same decision here
+  const bool misaligned = (smem_u32(smem) & 1023u) != 0;
+  if (misaligned && threadIdx.x == 0 && a.status) {
+    atomicCAS(a.status, 0, (int)GDLA_ERR_CUDA);
+    atomicCAS(a.status + 1, 0, 198);
+  }
+  const long n_tiles = (long)a.n_tm * a.n_tn;  // pair tiles: n_tm counts 256-row blocks
+  const int KT = (a.K + GK - 1) / GK;
+  const long cl = blockIdx.x >> 1, n_cl = gridDim.x >> 1;
+  const int my_tiles = cl < n_tiles ? (int)((n_tiles - cl + n_cl - 1) / n_cl) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&bars.full[s]), 1);   // rank 0's arrive.expect_tx (both CTAs' bytes)
+      mbar_init(smem_u32(&bars.empty[s]), 1);  // one commit of rank 0's MMA warp
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars.acc_full[i]), 1);
+      mbar_init(smem_u32(&bars.acc_empty[i]), 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(smem_u32(&bars.mma_done), 1);
+    fence_mbar_init();
+    abort_flag = 0;
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(smem_u32(&bars.tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barrier inits of both CTAs are visible before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_slot;
+
+  if (misaligned) {
+    // nothing to do but the final cluster barrier
+  } else if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      long kc = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const long t = cl + (long)i * n_cl;
+        const long m0 = (t / a.n_tn) * (2 * GM) + (long)rank * GM;
+        const int n0 = (int)(t % a.n_tn) * BN + (int)rank * (BN / 2);
+        for (int kb = 0; kb < KT; ++kb, ++kc) {
+          const int s = (int)(kc % STAGES);
+          if (kc >= STAGES &&
+              !mbar_wait(smem_u32(&bars.empty[s]), (int)((kc / STAGES) & 1) ^ 1, a.status, 111, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = smem_u32(smem + s * C_::STAGE), b_dst = a_dst + C_::A_BYTES;
+          const uint32_t bar = mapa_shared(smem_u32(&bars.full[s]), 0);
+          if (rank == 0) mbar_expect_tx(smem_u32(&bars.full[s]), 2 * C_::STAGE);
+          tma_load_2d_pair(a_dst, &tmA, bar, kb * GK, (int)m0);
+#pragma unroll
+          for (int j = 0; j < BN / 128; ++j) tma_load_2d_pair(b_dst + j * (GK * 128), &tmB, bar, n0 + 64 * j, kb * GK);
+        }
+      }
+      if (!ok) abort_flag = 1;
+      // the copies still in flight complete on rank 0's ring barriers: rank 0 waits for
+      // them (bounded) before the final cluster barrier, after which the peer may leave
+      if (rank == 0)
+        for (long c = (kc > STAGES ? kc - STAGES : 0); c < kc; ++c)
+          mbar_wait(smem_u32(&bars.full[c % STAGES]), (int)((c / STAGES) & 1), nullptr, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = true;
+      if (rank == 0) {
+        // ---------------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc = idesc_bf16_f32(2 * GM, BN, false, true);
+        long kc = 0;
+        for (int i = 0; i < my_tiles && ok; ++i) {
+          const int buf = i & 1;
+          // both CTAs' epilogues have drained this accumulator (tile i - 2)
+          if (i >= 2)
+            ok = mbar_wait(smem_u32(&bars.acc_empty[buf]), ((i >> 1) & 1) ^ 1, a.status, 114, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t acc = tmem + (uint32_t)(buf * BN);
+          for (int kb = 0; kb < KT; ++kb, ++kc) {
+            const int s = (int)(kc % STAGES);
+            ok = mbar_wait(smem_u32(&bars.full[s]), (int)((kc / STAGES) & 1), a.status, 112, &abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t as = smem_u32(smem + s * C_::STAGE), bs = as + C_::A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < GK / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(as + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(bs + kk * 2048, GK * 128, 1024);
+              mma_ss_pair(acc, ad, bd, idesc, (kb | kk) != 0);
+            }
+            mma_commit_pair(mapa_shared(smem_u32(&bars.empty[s]), 0));
+            mma_commit_pair(mapa_shared(smem_u32(&bars.empty[s]), 1));
+          }
+          if (ok) {
+            mma_commit_pair(mapa_shared(smem_u32(&bars.acc_full[buf]), 0));
+            mma_commit_pair(mapa_shared(smem_u32(&bars.acc_full[buf]), 1));
+          }
+        }
+        if (!ok) abort_flag = 1;
+        // every pair MMA has completed before either CTA releases its TMEM or leaves
+        mma_commit_pair(mapa_shared(smem_u32(&bars.mma_done), 0));
+        mma_commit_pair(mapa_shared(smem_u32(&bars.mma_done), 1));
+      }
+      // both CTAs: the last commit's arrival has landed in this CTA's shared memory
+      mbar_wait(smem_u32(&bars.mma_done), 0, nullptr, 115);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp - 4;
+    uint8_t* stg = smem + C_::OFF_EPI + q4 * 8192;
+    int nb = 0;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int buf = i & 1;
+      bool ok = mbar_wait(smem_u32(&bars.acc_full[buf]), (i >> 1) & 1, a.status, 113, &abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const long t = cl + (long)i * n_cl;
+      const long row0 = (t / a.n_tn) * (2 * GM) + (long)rank * GM + q4 * 32;
+      const int n0 = (int)(t % a.n_tn) * BN;
+      drain_tma_bf16<BN>(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN), stg, nb, lane, row0, n0, a.M,
+                         a.N, &tmC);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars.acc_empty[buf]), 0));
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc_pair(tmem, 512);
 }
 
 bool gemm_tc_shape(const GemmParams& p) {
@@ -312,8 +506,57 @@ static cudaError_t launch_cfg(const GemmParams& p, int* status, cudaStream_t s) 
   return cudaGetLastError();
 }
 
-// bf16 output: 128 x 256 tiles (the expansion, the gate projection), 128 x 64 when N is narrow
+// CTA pairs: 256 x 256 tiles, one cluster of two CTAs per pair of SMs
+template <int STAGES>
+static cudaError_t launch_pair(const GemmParams& p, int* status, cudaStream_t s) {
+  using C_ = gtc::PairCfg<STAGES>;
+  constexpr int SMEM = C_::OFF_BARS + (int)sizeof(gtc::Bars<STAGES>);
+  static_assert(SMEM <= 232448, "shared memory budget of one CTA");
+  CUtensorMap ta, tb, tc;
+  const uint64_t adims[2] = {(uint64_t)p.K, (uint64_t)p.M}, astr[1] = {(uint64_t)p.K * 2};
+  const uint32_t abox[2] = {64, gtc::GM};
+  const uint64_t bdims[2] = {(uint64_t)p.N, (uint64_t)p.K}, bstr[1] = {(uint64_t)p.N * 2};
+  const uint32_t bbox[2] = {64, gtc::GK};
+  const uint64_t cdims[2] = {(uint64_t)p.N, (uint64_t)p.M}, cstr[1] = {(uint64_t)p.N * 2};
+  const uint32_t cbox[2] = {64, 32};
+  if (!make_tmap_bf16(&ta, p.A, 2, adims, astr, abox) || !make_tmap_bf16(&tb, p.Bm, 2, bdims, bstr, bbox) ||
+      !make_tmap_bf16(&tc, p.C, 2, cdims, cstr, cbox))
+    return cudaErrorInvalidValue;
+  GemmTcArgs a{};
+  a.M = p.M; a.N = p.N; a.K = p.K;
+  a.n_tm = (int)((p.M + 2 * gtc::GM - 1) / (2 * gtc::GM));
+  a.n_tn = (p.N + C_::BN - 1) / C_::BN;
+  a.C = p.C; a.status = status;
+  auto kern = gemm_pair_kernel<STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.blockDim = dim3(gtc::GTHREADS);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = s;
+  // as many clusters as can be resident at once (a persistent grid), at most one per tile
+  cfg.gridDim = dim3(2 * (gtc::kNumSMs / 2));
+  int max_cl = 0;
+  e = cudaOccupancyMaxActiveClusters(&max_cl, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  if (max_cl < 1) return cudaErrorInvalidConfiguration;
+  const long tiles = (long)a.n_tm * a.n_tn;
+  const int clusters = (int)(tiles < max_cl ? tiles : max_cl);
+  cfg.gridDim = dim3(2 * clusters);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, a);
+}
+
+// bf16 output: 256 x 256 tiles on CTA pairs when there are 256 rows or more, else
+// 128 x 256 tiles on single CTAs (the expansion, the gate projection); 128 x 64 when N is narrow
 cudaError_t launch_gemm_tc(const GemmParams& p, int* status, cudaStream_t s) {
+  if (p.N > 64 && p.M >= 2 * gtc::GM) return launch_pair<6>(p, status, s);
   return p.N > 64 ? launch_cfg<256, 4, __nv_bfloat16>(p, status, s) : launch_cfg<64, 8, __nv_bfloat16>(p, status, s);
 }
 
