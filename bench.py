@@ -53,8 +53,8 @@ CSRC = os.path.join(ROOT, "differential_latent_attention_gdla_b200", "csrc")
 # were taken on: once a kernel changes, its figure no longer applies and the bench
 # reports null.
 MEASURED_TRAFFIC = {
-    ("attn_tc_kernel", "b1_l32k_g3"): (2.172e9, ("attn_tc.cu", "sm100.cuh"), "8be5e6943ee8e6bc"),
-    ("decode_tc_kernel", "b64_t32k"): (2.429e9, ("decode_tc.cu", "sm100.cuh"), "b06a10276bcf375f"),
+    ("attn_tc_kernel", "b1_l32k_g3"): (2.172e9, ("attn_tc.cu", "sm100.cuh"), "434f80305053d633"),
+    ("decode_tc_kernel", "b64_t32k"): (2.429e9, ("decode_tc.cu", "sm100.cuh"), "3559fd5f6339878d"),
 }
 
 
