@@ -845,6 +845,7 @@ constexpr int CB_M = 64, CB_N = 128, CB_K = 512;
 constexpr int CB_A = CB_M * CB_K * 2;   // 64 KB: 8 chunks of [64 rows x 128 B]
 constexpr int CB_B = CB_K * CB_N * 2;   // 128 KB: 2 MN blocks of [512 K rows x 128 B]
 constexpr int CB_SMEM = CB_A + CB_B + 64;
+constexpr int kCombineSMs = 148;  // B200
 }  // namespace dtc
 
 __global__ void __launch_bounds__(512, 1)
@@ -1062,7 +1063,15 @@ cudaError_t launch_decode_combine_tc(const DecodeParams& p, cudaStream_t s) {
   if (!make_tmap_bf16(&tw, p.w_ukv, 2, dims, str, box)) return cudaErrorInvalidValue;
   CombineTcArgs a{};
   a.B = p.B; a.n_kv = p.n_kv; a.g = p.g; a.H_q = p.n_kv * (p.g + 1); a.n_hg = p.n_hg; a.hpc = p.hpc;
-  a.n_ranges = p.n_ranges; a.part_heads = p.part_heads; a.spb = dtc::CB_M / (p.g + 1);
+  a.n_ranges = p.n_ranges; a.part_heads = p.part_heads;
+  // sequences per block: as few as fill one wave of blocks over the SMs (every block stages
+  // its group's W_UV and runs one M = 64 MMA chain, so more, smaller blocks shorten the tail
+  // behind the split kernel), at most a full 64-row MMA tile
+  {
+    const int per_group = dtc::kCombineSMs / p.n_kv > 1 ? dtc::kCombineSMs / p.n_kv : 1;
+    const int spb = (p.B + per_group - 1) / per_group, cap = dtc::CB_M / (p.g + 1);
+    a.spb = spb < 1 ? 1 : (spb > cap ? cap : spb);
+  }
   a.seqinfo = p.seqinfo; a.part_o = p.part_o; a.part_ml = p.part_ml; a.lam = p.lam;
   a.gate = reinterpret_cast<const __nv_bfloat16*>(p.gate);
   a.out = reinterpret_cast<__nv_bfloat16*>(p.out);
