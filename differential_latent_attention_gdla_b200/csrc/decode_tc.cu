@@ -620,8 +620,9 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
 // ---------------------------------------------------------------- absorb
 // The absorbed query of the tensor-core path, on the tensor cores: for KV group h
 // and a tile of 128 query rows (row = (sequence b, head u of the group)),
-//   Qabs[rows x 256 latent dims] = Q_nope[rows x 128] . W_UK,h^T[128 x 256]
-// (half nh of the 512 latent dims per block), scaled by tau*log2(e) and written as
+//   Qabs[rows x 128 latent dims] = Q_nope[rows x 128] . W_UK,h^T[128 x 128]
+// (quarter nh of the 512 latent dims per block: four blocks per row tile, so that a
+// call's blocks cover most SMs and each is short), scaled by tau*log2(e) and written as
 // bf16 straight into the split kernel's query images; the nh = 0 blocks also rotate
 // the rotary query parts (RoPE at position seqlen-1) into the images, and the
 // blocks of KV group 0 zero the image rows of padding heads.
@@ -637,9 +638,10 @@ struct AbsorbTcArgs {
 };
 
 namespace dtc {
-constexpr int AB_M = 128, AB_N = 256, AB_K = 128;
+constexpr int AB_M = 128, AB_N = 128, AB_K = 128;
 constexpr int AB_A = AB_M * AB_K * 2;   // 32 KB: two 64-dim chunks of [128 rows x 128 B]
-constexpr int AB_B = AB_N * AB_K * 2;   // 64 KB: two 64-dim chunks of [256 latent rows x 128 B]
+constexpr int AB_B = AB_N * AB_K * 2;   // 32 KB: two 64-dim chunks of [128 latent rows x 128 B]
+constexpr int AB_Z = 512 / AB_N;        // blocks per row tile (latent dims in AB_N slices)
 constexpr int AB_SMEM = AB_A + AB_B + 64;
 }  // namespace dtc
 
@@ -813,7 +815,7 @@ cudaError_t launch_decode_absorb_tc(const DecodeParams& p, cudaStream_t s) {
                                        dtc::AB_SMEM);
   if (e != cudaSuccess) return e;
   const int rows = p.B * (p.g + 1);
-  dim3 grid((unsigned)p.n_kv, (unsigned)((rows + dtc::AB_M - 1) / dtc::AB_M), 2);
+  dim3 grid((unsigned)p.n_kv, (unsigned)((rows + dtc::AB_M - 1) / dtc::AB_M), dtc::AB_Z);
   decode_absorb_tc_kernel<<<grid, 256, dtc::AB_SMEM, s>>>(tw, a);
   return cudaGetLastError();
 }
