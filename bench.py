@@ -15,8 +15,9 @@ needed between steps.
 
 Beside the timed steps (outside their timed region):
   * `decode`: the decode call timed in its own loop after its own warm-up, before the
-    prefill steps (the `roofline` of the decode), and its time inside the steps
-    (`in_step_ms`), where it follows the power-capped prefill;
+    prefill steps (the `roofline` of the decode, with the SM clocks sampled over that
+    loop), and its time inside the steps (`in_step_ms`), where it follows the
+    power-capped prefill;
   * `prefill_cfg2` (B=4 L=4096 g=2 causal), `prefill_cfg4` (B=2 L=65536 g=2,
     4096-token window) and the report's own layout, g=4 (80 heads):
     `prefill_g4_swa128` (128-token window), `decode_g4`, and `gates` (gate and lambda
@@ -140,7 +141,7 @@ def hbm_roofline(gbs: float, pk: dict) -> dict:
 
 
 GATE_D_X = 2048  # width of the layer input x of the lambda projection (the caller's choice)
-DECODE_WARMUP, DECODE_STEPS = 100, 200  # the decode's own loop (a call is ~0.5 ms)
+DECODE_WARMUP, DECODE_STEPS = 100, 600  # the decode's own loop (a call is ~0.5 ms)
 
 # The cpu_baseline leg and the reference arm time the oracle on the same sample.
 ORACLE_ROWS = 24
@@ -224,12 +225,13 @@ def run_reference(a):
 
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
-    def __init__(self, index: int):
+    def __init__(self, index: int, tag: str = ""):
         self.proc = None
-        # raw samples go to $GDLA_CLOCKS_DIR/clocks_rank<i>.csv when set (to keep them), else to /tmp
+        # raw samples go to $GDLA_CLOCKS_DIR/clocks_<tag>rank<i>.csv when set (to keep them), else to /tmp
         out_dir = os.environ.get("GDLA_CLOCKS_DIR")
-        self.path = (os.path.join(out_dir, f"clocks_rank{index}.csv") if out_dir
-                     else f"/tmp/gdla_clocks_{os.getpid()}_{index}.csv")
+        pre = f"{tag}_" if tag else ""
+        self.path = (os.path.join(out_dir, f"clocks_{pre}rank{index}.csv") if out_dir
+                     else f"/tmp/gdla_clocks_{pre}{os.getpid()}_{index}.csv")
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -353,7 +355,11 @@ def run_ours(a):
 
     # ---- the decode call in its own loop, at its own steady state (its own warm-up,
     # not right after the power-capped prefill, whose decode time is `in_step_ms`)
+    # (SM clocks sampled over it too: nvidia-smi gets half a second to start sampling)
+    dclocks = ClockSampler(local, "decode")
+    time.sleep(0.5)
     t_dec_alone = time_loop(decode, max(a.steps, DECODE_STEPS), max(a.warmup, DECODE_WARMUP), stream)
+    dclk = dclocks.stop()
     if int(gdla.workspace_status(dws)) != 0:
         raise RuntimeError("device status word reports a failed wait (decode)")
 
@@ -537,7 +543,8 @@ def run_ours(a):
                         "algorithmic_tflop": pf / 1e12},
             "decode": {"value": dec_gbs, "unit": "GB/s", "ms": t_dec_alone, "algorithmic_gb": db / 1e9,
                        "timing": "own loop after its own warm-up, before the prefill steps", "in_step_ms": t_dec,
-                       "in_step_value": weak_scaling_value(db, world, t_dec * 1e-3) / 1e9, "roofline": droof},
+                       "in_step_value": weak_scaling_value(db, world, t_dec * 1e-3) / 1e9, "roofline": droof,
+                       "clocks": dclk},
             "roofline": roof, **extras,
             "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": launches_per_step * a.steps, "clocks": clk,
             "wall_s": wall,
