@@ -55,7 +55,7 @@ CSRC = os.path.join(ROOT, "differential_latent_attention_gdla_b200", "csrc")
 # reports null.
 MEASURED_TRAFFIC = {
     ("attn_tc_kernel", "b1_l32k_g3"): (2.172e9, ("attn_tc.cu", "sm100.cuh"), "434f80305053d633"),
-    ("decode_tc_kernel", "b64_t32k"): (2.429e9, ("decode_tc.cu", "sm100.cuh"), "3559fd5f6339878d"),
+    ("decode_tc_kernel", "b64_t32k"): (2.432e9, ("decode_tc.cu", "sm100.cuh"), "c513bdaa672dd3e1"),
 }
 
 
@@ -232,17 +232,21 @@ class ClockSampler:
         pre = f"{tag}_" if tag else ""
         self.path = (os.path.join(out_dir, f"clocks_{pre}rank{index}.csv") if out_dir
                      else f"/tmp/gdla_clocks_{pre}{os.getpid()}_{index}.csv")
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+        q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                          "-lms", "50", "-i", str(index)], stdout=self.f, stderr=subprocess.DEVNULL)
+                                          "-lms", "20", "-i", str(index)], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, window=None):
+        """Summary of the samples; with window = (t0, t1) (host time.time()), only the
+        samples taken inside it."""
+        import datetime
+
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -252,14 +256,17 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             p = [x.strip() for x in line.split(",")]
-            if len(p) < 9:
+            if len(p) < 10:
                 continue
             try:
-                sm.append(float(p[1]))
-                mx.append(float(p[2]))
+                ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if window is not None and not (window[0] <= ts <= window[1]):
+                    continue
+                sm.append(float(p[2]))
+                mx.append(float(p[3]))
             except ValueError:
                 continue
-            for n, v in zip(names, p[5:9]):
+            for n, v in zip(names, p[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         load = [s for s in sm if s > 0.5 * max(sm)] if sm else []
@@ -358,8 +365,9 @@ def run_ours(a):
     # (SM clocks sampled over it too: nvidia-smi gets half a second to start sampling)
     dclocks = ClockSampler(local, "decode")
     time.sleep(0.5)
+    w0 = time.time()
     t_dec_alone = time_loop(decode, max(a.steps, DECODE_STEPS), max(a.warmup, DECODE_WARMUP), stream)
-    dclk = dclocks.stop()
+    dclk = dclocks.stop((w0, time.time()))
     if int(gdla.workspace_status(dws)) != 0:
         raise RuntimeError("device status word reports a failed wait (decode)")
 
@@ -371,8 +379,10 @@ def run_ours(a):
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
     clocks = ClockSampler(local)
+    time.sleep(0.5)  # nvidia-smi's first samples land before the timed steps
     barrier()
     torch.cuda.synchronize()
+    w0 = time.time()
     t0 = time.perf_counter()
     for k in range(a.steps):
         ev[k][0].record(stream)
@@ -385,7 +395,7 @@ def run_ours(a):
     torch.cuda.synchronize()
     barrier()
     wall = time.perf_counter() - t0
-    clk = clocks.stop()
+    clk = clocks.stop((w0, time.time()))
     if int(gdla.workspace_status(status)) != 0 or int(gdla.workspace_status(dws)) != 0:
         raise RuntimeError("device status word reports a failed wait")
 
