@@ -3,22 +3,21 @@
 // Report", Architecture: RoPE only on the rotary parts; signal and noise heads
 // attend independently; D = H_S - lambda (.) Repeat_g(H_N); Y = sigmoid(G) (.) D).
 //
-// A work item is (sequence b, KV group h, 64 query rows) with every head that
-// reads KV head h: the noise head and its g signal heads, taken two at a time:
-//   pair 0 = (noise, signal 0), pair 1 = (signal 1, signal 2), ...
-// The two heads of a pair are stacked into one 128-row operand (rows 0-63 the
-// first head, rows 64-127 the second), so every tensor-core instruction is
-// M = 128 x N = 128: S = Q K^T over a 128-key tile (K = 192) and O += P V
-// (K = 128 keys, N = 128 value dims), and every K/V tile brought in from L2
-// serves both heads. Both Q (rotated once per pair) and P live in TMEM, so the
-// tensor core reads only K and V from shared memory.
+// A work item is (sequence b, KV group h, 128 query rows) with every head that
+// reads KV head h: the noise head and its g signal heads, one after the other
+// (pass 0 the noise head, pass u the signal head u-1). A pass stacks the head's
+// 128 consecutive query rows into one 128-row operand, so every tensor-core
+// instruction is M = 128 x N = 128: S = Q K^T over a 128-key tile (K = 192) and
+// O += P V (K = 128 keys, N = 128 value dims), for any g without padding rows.
+// Both Q (rotated once per pass) and P live in TMEM, so the tensor core reads only
+// K and V from shared memory.
 // The kernel is persistent: one CTA per SM takes work items from a global counter
 // (KV-group-major, heaviest query blocks first) until none is left, so the set-up of a
 // CTA happens once and the next item's Q, K and V copies overlap the current item's
 // last tiles and epilogue; items reach the other roles through a 2-slot ring in shared
 // memory that the producer fills.
 // Warp roles (640 threads):
-//   warp 0      work items; TMA producer: the pair's Q in three 64-dim chunks through a
+//   warp 0      work items; TMA producer: the pass's Q in three 64-dim chunks through a
 //               2-deep staging ring; K tiles (128 keys x 192) and V tiles
 //               (128 keys x 128), each in a 2-deep ring;
 //   warp 1      MMA issuer (one lane): S(j) into S buffer j % 2, then
@@ -34,8 +33,8 @@
 // tensor core runs the MMAs of one thread in issue order, so S(j+2) (issued after
 // PV(j)) never overwrites P(j) too early.
 // The noise head's normalised output H_N is parked in shared memory (bf16) for
-// the epilogues of all g signal heads, so neither H_S nor H_N goes to global
-// memory. O is rescaled only when a row's running maximum grows by more than
+// the epilogues of all g signal heads (thread r writes and later reads row r's
+// own columns), so neither H_S nor H_N goes to global memory. O is rescaled only when a row's running maximum grows by more than
 // 2^8.
 #include <limits.h>
 #include <math.h>
@@ -46,10 +45,11 @@
 namespace gdla {
 namespace {
 
-constexpr int BM = 64;    // query rows per head
+constexpr int BM = 64;    // query rows of one Q copy (a 64-row TMA box)
+constexpr int IM = 2 * BM;  // query rows of a work item (one pass: one head, these 128 rows)
 constexpr int BN = 128;   // keys per tile
 constexpr int DN = 128, DR = 64, DV = 128;
-constexpr int ROWS = 2 * BM;                // stacked rows of a pair
+constexpr int ROWS = IM;                    // rows of a pass's operand
 constexpr int NWG = 4;                      // softmax warpgroups
 constexpr int CW = BN / NWG;                // key columns per softmax thread
 constexpr int QS_BYTES = ROWS * 128;        // 16 KB: one 64-dim chunk of the stacked Q rows
@@ -57,8 +57,8 @@ constexpr int K_CHUNK = BN * 128;           // 16 KB: 128 keys x 64 dims
 constexpr int K_BYTES = 3 * K_CHUNK;        // 48 KB
 constexpr int V_BLOCK = BN * 128;           // 16 KB: 128 keys x 64 value dims
 constexpr int V_BYTES = 2 * V_BLOCK;        // 32 KB
-constexpr int HN_BYTES = BM * DV * 2;       // 16 KB: parked H_N (bf16)
-constexpr int XM_BYTES = 2 * NWG * ROWS * 4;  // 4 KB: per-warpgroup row maxima / sums, double-buffered
+constexpr int HN_BYTES = IM * DV * 2;       // 32 KB: parked H_N (bf16)
+constexpr int XM_BYTES = NWG * ROWS * 4;    // 2 KB: per-warpgroup row maxima / sums
 constexpr int OFF_K = 2 * QS_BYTES;
 constexpr int OFF_V = OFF_K + 2 * K_BYTES;
 constexpr int OFF_HN = OFF_V + 2 * V_BYTES;
@@ -89,7 +89,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 __device__ __forceinline__ bool bar_or512(bool pred) { return sm100::named_bar_or(1, 128 * NWG, pred); }
 __device__ __forceinline__ void bar_sync512() { sm100::named_bar_sync(1, 128 * NWG); }
 
-// parked H_N: row r (of 64), 16-byte chunk c (of 16) stored at chunk c ^ (r & 15)
+// parked H_N: row r (of 128), 16-byte chunk c (of 16) stored at chunk c ^ (r & 15)
 __device__ __forceinline__ uint32_t hn_off(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 15)) << 4)); }
 
 }  // namespace
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G1 = a.g + 1;
-  const int n_pairs = (G1 + 1) / 2;
+  const int n_pairs = G1;  // passes of an item, one head each (the loops below call them pairs p)
   const int n_S = a.g * a.n_kv;
   const int q_end = a.q_start + a.q_len;  // one past the last query position
   // Work item t: KV-group-major order, heaviest query blocks first within a group, handed
@@ -146,17 +146,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int m_idx = a.n_qtiles - 1 - t % a.n_qtiles;
     it.h = (t / a.n_qtiles) % a.n_kv;
     it.b = t / (a.n_qtiles * a.n_kv);
-    it.m_loc = m_idx * BM;       // first query row of the block within the q/Y tensors
+    it.m_loc = m_idx * IM;       // first query row of the block within the q/Y tensors
     it.m0 = a.q_start + it.m_loc;  // its position in the sequence
-    const int last_row = min(q_end - 1, it.m0 + BM - 1);
+    const int last_row = min(q_end - 1, it.m0 + IM - 1);
     const int key_lo = a.sliding ? max(0, it.m0 - a.window + 1) : 0;
     it.j_lo = key_lo / BN;
     it.n_tiles = last_row / BN - it.j_lo + 1;
     return it;
   };
+  // head of pass hl of KV group h: the noise head first, then the signal heads
   auto head_of = [&](int h, int hl) { return hl == 0 ? n_S + h : h * a.g + hl - 1; };
-  // head in half s of pair p; a pair without a second head repeats the first (its rows are discarded)
-  auto head_in = [&](int h, int p, int s) { return head_of(h, 2 * p + s < G1 ? 2 * p + s : 2 * p); };
   // the consumers' side of the work ring: item k sits in slot k & 1
   auto take_item = [&](int k, bool& ok) -> int {
     const int sl = k & 1;
@@ -246,15 +245,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ++vc;
         return true;
       };
-      // one 64-dim chunk of the pair's stacked Q rows into staging buffer qk % 2
+      // one 64-dim chunk of the pass's 128 Q rows (two 64-row boxes) into staging buffer qk % 2
       auto load_q = [&](int p, int k) -> bool {
         const int sl = qk & 1;
         if (qk >= 2 && !mbar_wait(smem_u32(&bars.q_free[sl]), ((qk >> 1) & 1) ^ 1, a.status, 201, &abort_flag)) return false;
         const uint32_t bar = smem_u32(&bars.q_full[sl]);
         mbar_expect_tx(bar, QS_BYTES);
         for (int s = 0; s < 2; ++s)
-          tma_load_4d(smem_u32(qs_sm + sl * QS_BYTES + s * (BM * 128)), &tmQ, bar, k * 64, head_in(it.h, p, s),
-                      it.m_loc, it.b);
+          tma_load_4d(smem_u32(qs_sm + sl * QS_BYTES + s * (BM * 128)), &tmQ, bar, k * 64, head_of(it.h, p),
+                      it.m_loc + s * BM, it.b);
         ++qk;
         return true;
       };
@@ -274,7 +273,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         it = item_of(t);
         for (int p = 0; p < n_pairs && ok && !abort_flag; ++p) {
           // the last Q chunk reuses the staging buffer of the first, which the softmax
-          // warps free only after the previous pair's epilogue: K(0), K(1) go first
+          // warps free only after the previous pass's epilogue: K(0), K(1) go first
           ok = load_q(p, 0) && load_q(p, 1);
           // consumption order of the tensor core: S(0), S(1), PV(0), S(2), PV(1), ...
           if (ok) ok = load_k(0) && (it.n_tiles < 2 || load_k(1));
@@ -339,14 +338,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ++vc;
         return true;
       };
-      int gp = 0;  // head pairs over the whole CTA (q_ready / o_full phases)
+      int gp = 0;  // passes over the whole CTA (q_ready / o_full phases)
       for (int ki = 0; ok; ++ki) {
         const int t = take_item(ki, ok);
         if (ok) mbar_arrive(smem_u32(&bars.item_free[ki & 1]));
         if (!ok || t < 0) break;
         const int n_tiles = item_of(t).n_tiles;
         for (int p = 0; p < n_pairs && ok; ++p, ++gp) {
-          // the softmax warps write the rotated Q into TMEM after the previous pair's epilogue
+          // the softmax warps write the rotated Q into TMEM after the previous pass's epilogue
           ok = mbar_wait(smem_u32(&bars.q_ready), gp & 1, a.status, 211, &abort_flag);
           if (!ok) break;
           tc_fence_after();
@@ -372,20 +371,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int c = (warp - 4) >> 2;          // column quarter: keys 32c.. of each tile, value dims 32c.. of O
     const int q4 = warp & 3;                // TMEM lane quadrant
     const int r = q4 * 32 + lane;           // stacked row = TMEM lane
-    const int half = r >> 6;                // 0: first head of the pair, 1: second
     Item it{};
     int i = 0;                              // this row's query position in the current item
     bool row_ok = false;
     int rope_pos = 0;
     auto set_rows = [&]() {
-      i = it.m0 + (r & (BM - 1));
+      i = it.m0 + r;
       row_ok = i < q_end;
       rope_pos = row_ok ? i : q_end - 1;  // rows past the end are discarded; any table row will do
     };
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const uint32_t tO = tmem + lane_base + kColO + CW * c;
     const uint32_t tQ = tmem + lane_base + kColQ;
-    // this row's RoPE factors for rotary dims 8c .. 8c+7, loaded ahead of each pair's
+    // this row's RoPE factors for rotary dims 8c .. 8c+7, loaded ahead of each pass's
     // rotary chunk (volatile: live only between the load and that chunk, not across the
     // key tiles)
     float cs[8], sn[8];
@@ -398,7 +396,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(sn[e]) : "l"(sp + e));
       }
     };
-    // chunk k of pair p's stacked Q rows into TMEM: thread c moves dims 16c .. 16c+15 of a
+    // chunk k of pass p's 128 Q rows into TMEM: thread c moves dims 16c .. 16c+15 of a
     // content chunk, or rotates dims 8c .. 8c+7 with 32+8c .. 32+8c+7 of the rotary chunk
     auto move_q = [&](int p, int k) -> bool {
       const int qk = 3 * p + k, sl = qk & 1;
@@ -439,7 +437,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_arrive_warp(smem_u32(&bars.q_ready));
     };
     int tc = 0;                             // tiles processed over the whole CTA
-    int ki = 0, gp = 0;                     // work items taken, head pairs begun over the whole CTA
+    int ki = 0, gp = 0;                     // work items taken, passes begun over the whole CTA
     // the next work item from the ring (every softmax thread; the slot is released at once)
     auto next_item = [&](bool& ok) -> int {
       const int t = take_item(ki, ok);
@@ -464,13 +462,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
     for (int p = 0; t >= 0 && !failed;) {
-      const int hl = 2 * p + half;
+      const int hl = p;                     // 0: the noise head, u: signal head u-1
       const int cbase = CW * c;             // this warpgroup finishes value columns [cbase, cbase + 32)
-      const bool real = hl < G1;            // the second half of a short last pair is discarded
       const int sh = hl > 0 ? head_of(it.h, hl) : 0;  // signal head index
       const long tok = (long)it.b * a.q_len + (i - a.q_start);
       const int m0 = it.m0, j_lo = it.j_lo, n_tiles = it.n_tiles;
-      if (hl > 0 && real && row_ok) {
+      if (hl > 0 && row_ok) {
         // the epilogue's gate and lambda of this row: into L2 while the key tiles stream
         prefetch_l2(a.gate + (tok * n_S + sh) * DV + cbase);
         prefetch_l2(a.gate + (tok * n_S + sh) * DV + cbase + CW - 1);
@@ -496,7 +493,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int e = 0; e < CW; ++e) sr[e] = __float_as_uint(-INFINITY);
         }
         const int key0 = (j_lo + jj) * BN + CW * c;
-        const bool full_vis = (key0 + CW - 1 <= m0) && (!a.sliding || key0 > m0 + BM - 1 - a.window);
+        const bool full_vis = (key0 + CW - 1 <= m0) && (!a.sliding || key0 > m0 + IM - 1 - a.window);
         if (!full_vis) {
           // key column e of this quarter is visible iff e_lo <= e <= e_hi
           const int e_hi = i - key0;
@@ -524,9 +521,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           }
           // the row maximum of the whole tile: exchange with the three threads holding the
-          // other columns (a slot is rewritten only after the next tile's barrier-reduction,
+          // other columns (the buffer is rewritten only after a later barrier-reduction,
           // which every thread reaches after reading it here)
-          float* xs = xm + (tc & 1) * (NWG * ROWS);
+          float* xs = xm;
           xs[c * ROWS + r] = pm;
           bar_sync512();
           const float mr = fmaxf(fmaxf(xs[r], xs[ROWS + r]), fmaxf(xs[2 * ROWS + r], xs[3 * ROWS + r]));
@@ -594,7 +591,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       tc_fence_after();
-      // the next head pair: the item's next one, or the next item's first
+      // the next pass: the item's next head, or the next item's first
       int t_next = t, p_next = p + 1;
       if (p_next == n_pairs) {
         bool ok = true;
@@ -607,7 +604,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       const bool next = t_next >= 0;
       if (next) {
-        // every S MMA of this pair is done, so the next pair's Q content chunks may go into
+        // every S MMA of this pass is done, so the next pass's Q content chunks may go into
         // TMEM now; its rotary chunk follows the epilogue, while that copy lands
         bool ok = move_q(gp + 1, 0);
         ok = move_q(gp + 1, 1) && ok;
@@ -617,9 +614,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       // row sum: add the other quarters' partial sums (same running maximum everywhere).
-      // The slot was last read two tiles ago.
+      // Every thread has passed the barrier-reduction after o_full since it last read
+      // the buffer (a tile's maximum exchange).
       {
-        float* xs = xm + (tc & 1) * (NWG * ROWS);
+        float* xs = xm;
         xs[c * ROWS + r] = l_part;
         bar_sync512();
         l_part = (xs[r] + xs[ROWS + r]) + (xs[2 * ROWS + r] + xs[3 * ROWS + r]);
@@ -640,13 +638,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pv.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
             pv.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
             pv.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(hn_sm + hn_off(r & (BM - 1), (cbase + 16 * ch) / 8 + q)) = pv;
+            *reinterpret_cast<uint4*>(hn_sm + hn_off(r, (cbase + 16 * ch) / 8 + q)) = pv;
           }
         }
       }
-      // pair 0 holds the noise head: its H_N is parked before any signal row reads it
+      // pass 0 is the noise head: its H_N is parked before any signal row reads it
       if (p == 0) bar_sync512();
-      if (hl > 0 && real) {
+      if (hl > 0) {
         // signal head: D = H_S - lambda H_N, Y = sigmoid(G) D
         const float lam = row_ok ? sigmoidf_(a.lam[tok * n_S + sh]) : 0.f;
         const __nv_bfloat16* gp = a.gate + (tok * n_S + sh) * DV + cbase;
@@ -661,7 +659,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
               gv[q] = reinterpret_cast<const uint4*>(gp + ch * 16)[q];
-              hv[q] = *reinterpret_cast<const uint4*>(hn_sm + hn_off(r & (BM - 1), (cbase + 16 * ch) / 8 + q));
+              hv[q] = *reinterpret_cast<const uint4*>(hn_sm + hn_off(r, (cbase + 16 * ch) / 8 + q));
             }
             const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(hv);
@@ -681,7 +679,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (next) {
-        // O of this pair is read: the next pair's rotary Q chunk (at the positions of the
+        // O of this pass is read: the next pass's rotary Q chunk (at the positions of the
         // next item's rows when the item changes), then its S MMAs may start
         if (p_next == 0) {
           it = item_of(t_next);
@@ -736,7 +734,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   }
   AttnTcArgs a{};
   a.B = p.B; a.L = p.L; a.n_kv = p.n_kv; a.g = p.g; a.sliding = p.sliding; a.window = p.window;
-  a.rope_max_pos = p.rope_max_pos; a.n_qtiles = (p.q_len + BM - 1) / BM;
+  a.rope_max_pos = p.rope_max_pos; a.n_qtiles = (p.q_len + IM - 1) / IM;
   a.q_len = p.q_len; a.q_start = p.q_start; a.sl2 = p.scale * kLog2e;
   a.cos_tab = p.cos_tab; a.sin_tab = p.sin_tab; a.lam = p.lam;
   a.gate = reinterpret_cast<const __nv_bfloat16*>(p.gate);
