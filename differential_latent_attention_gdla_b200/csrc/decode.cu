@@ -153,8 +153,8 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
       const int b = b0 + bl, d = c0 + 4 * lane;
       if (p.tc) {
         const int hgi = head / p.hpc, lh = head - hgi * p.hpc;
-        uint8_t* img = p.qimg + ((long)b * p.n_hg + hgi) * kDtcImageBytes;
-        *reinterpret_cast<uint2*>(img + dtc_image_offset(lh, d)) =
+        uint8_t* img = p.qimg + ((long)b * p.n_hg + hgi) * dtc_image_bytes(p.img_heads);
+        *reinterpret_cast<uint2*>(img + dtc_image_offset(lh, d, p.img_heads)) =
             make_uint2(sm100::pack_bf16x2(acc[i][0] * isc, acc[i][1] * isc),
                        sm100::pack_bf16x2(acc[i][2] * isc, acc[i][3] * isc));
       } else {
@@ -178,9 +178,10 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
     const float y1 = x1 * cs - x2 * sn, y2 = x2 * cs + x1 * sn;
     if (p.tc) {
       const int hgi = head / p.hpc, lh = head - hgi * p.hpc;
-      uint8_t* img = p.qimg + ((long)b * p.n_hg + hgi) * kDtcImageBytes;
-      *reinterpret_cast<__nv_bfloat16*>(img + dtc_image_offset(lh, p.d_c + k)) = __float2bfloat16_rn(y1 * isc);
-      *reinterpret_cast<__nv_bfloat16*>(img + dtc_image_offset(lh, p.d_c + k + half)) =
+      uint8_t* img = p.qimg + ((long)b * p.n_hg + hgi) * dtc_image_bytes(p.img_heads);
+      *reinterpret_cast<__nv_bfloat16*>(img + dtc_image_offset(lh, p.d_c + k, p.img_heads)) =
+          __float2bfloat16_rn(y1 * isc);
+      *reinterpret_cast<__nv_bfloat16*>(img + dtc_image_offset(lh, p.d_c + k + half, p.img_heads)) =
           __float2bfloat16_rn(y2 * isc);
     } else {
       float* o = p.q_rot + ((long)b * H_q + head) * p.d_rope;
@@ -193,11 +194,11 @@ __global__ void __launch_bounds__(256) decode_absorb_kernel(DecodeParams p) {
     for (int bl = 0; bl < nb; ++bl)
       for (int hgi = 0; hgi < p.n_hg; ++hgi) {
         const int nh = min(p.hpc, H_q - hgi * p.hpc);
-        uint8_t* img = p.qimg + ((long)(b0 + bl) * p.n_hg + hgi) * kDtcImageBytes;
-        const int chunks = (kDtcHeads - nh) * 9 * 8;  // 16-byte chunks of the padding rows
+        uint8_t* img = p.qimg + ((long)(b0 + bl) * p.n_hg + hgi) * dtc_image_bytes(p.img_heads);
+        const int chunks = (p.img_heads - nh) * 9 * 8;  // 16-byte chunks of the padding rows
         for (int e = threadIdx.x; e < chunks; e += blockDim.x) {
           const int lh = nh + e / 72, bx = (e % 72) / 8, c = e % 8;
-          *reinterpret_cast<uint4*>(img + bx * (kDtcHeads * 128) + lh * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(img + bx * (p.img_heads * 128) + lh * 128 + c * 16) = make_uint4(0, 0, 0, 0);
         }
       }
   }

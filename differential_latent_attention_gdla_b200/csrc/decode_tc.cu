@@ -627,7 +627,7 @@ __global__ void __launch_bounds__(dtc::DTHREADS, 1)
 // the rotary query parts (RoPE at position seqlen-1) into the images, and the
 // blocks of KV group 0 zero the image rows of padding heads.
 struct AbsorbTcArgs {
-  int B, T_max, n_kv, g, H_q, n_hg, hpc, rope_max_pos;
+  int B, T_max, n_kv, g, H_q, n_hg, hpc, rope_max_pos, img_heads;
   float isc;
   const __nv_bfloat16* q;  // [B, H_q, 192]
   const int* seqlens;
@@ -734,7 +734,7 @@ __global__ void __launch_bounds__(256, 1)
     head = head_of(R % G1);
     hgi = head / a.hpc;
     lh = head - hgi * a.hpc;
-    img = a.qimg + ((long)b * a.n_hg + hgi) * kDtcImageBytes;
+    img = a.qimg + ((long)b * a.n_hg + hgi) * dtc_image_bytes(a.img_heads);
   }
 #pragma unroll 1
   for (int ch = (warp >> 2) * (AB_N / 64); ch < ((warp >> 2) + 1) * (AB_N / 64); ++ch) {
@@ -749,7 +749,7 @@ __global__ void __launch_bounds__(256, 1)
         o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * a.isc, __uint_as_float(v[8 * q + 3]) * a.isc);
         o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * a.isc, __uint_as_float(v[8 * q + 5]) * a.isc);
         o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * a.isc, __uint_as_float(v[8 * q + 7]) * a.isc);
-        *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, nh * AB_N + ch * 32 + q * 8)) = o;
+        *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, nh * AB_N + ch * 32 + q * 8, a.img_heads)) = o;
       }
     }
   }
@@ -775,8 +775,9 @@ __global__ void __launch_bounds__(256, 1)
         lo[e] = pack_bf16x2((x1.x * c0 - x2.x * s0) * a.isc, (x1.y * c1 - x2.y * s1) * a.isc);
         hi[e] = pack_bf16x2((x2.x * c0 + x1.x * s0) * a.isc, (x2.y * c1 + x1.y * s1) * a.isc);
       }
-      *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, 512 + 8 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, 512 + 32 + 8 * c)) =
+      *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, 512 + 8 * c, a.img_heads)) =
+          make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(img + dtc_image_offset(lh, 512 + 32 + 8 * c, a.img_heads)) =
           make_uint4(hi[0], hi[1], hi[2], hi[3]);
     }
   }
@@ -787,10 +788,10 @@ __global__ void __launch_bounds__(256, 1)
     for (int bb = b_lo; bb < b_hi; ++bb)
       for (int hg2 = 0; hg2 < a.n_hg; ++hg2) {
         const int nhd = min(a.hpc, a.H_q - hg2 * a.hpc);
-        uint8_t* im = a.qimg + ((long)bb * a.n_hg + hg2) * kDtcImageBytes;
-        for (int e = tid; e < (kDtcHeads - nhd) * 72; e += 256) {
+        uint8_t* im = a.qimg + ((long)bb * a.n_hg + hg2) * dtc_image_bytes(a.img_heads);
+        for (int e = tid; e < (a.img_heads - nhd) * 72; e += 256) {
           const int l2 = nhd + e / 72, bx = (e % 72) / 8, c = e % 8;
-          *reinterpret_cast<uint4*>(im + bx * (kDtcHeads * 128) + l2 * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(im + bx * (a.img_heads * 128) + l2 * 128 + c * 16) = make_uint4(0, 0, 0, 0);
         }
       }
   }
@@ -809,6 +810,7 @@ cudaError_t launch_decode_absorb_tc(const DecodeParams& p, cudaStream_t s) {
   AbsorbTcArgs a{};
   a.B = p.B; a.T_max = p.T_max; a.n_kv = p.n_kv; a.g = p.g; a.H_q = p.n_kv * (p.g + 1);
   a.n_hg = p.n_hg; a.hpc = p.hpc; a.rope_max_pos = p.rope_max_pos; a.isc = p.scale * kLog2e;
+  a.img_heads = p.img_heads;
   a.q = reinterpret_cast<const __nv_bfloat16*>(p.q); a.seqlens = p.seqlens;
   a.cos_tab = p.cos_tab; a.sin_tab = p.sin_tab; a.qimg = p.qimg; a.status = p.status;
   cudaError_t e = cudaFuncSetAttribute(decode_absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1094,6 +1096,526 @@ cudaError_t launch_decode_combine_tc(const DecodeParams& p, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, decode_combine_tc_kernel, tw, a);
 }
 
+// ---------------------------------------------------------------- wide split kernel
+// The split-KV pass for 49 .. 80 query heads in one CTA (the report's own layout, g = 4,
+// has 80), so that the cache is streamed once for all heads of a sequence instead of once
+// per head group. What the narrow kernel's 48 heads allow and 80 do not, and what this
+// one does instead:
+//  * a 92 KB query image: 48-token tiles, two ring stages of 55 KB;
+//  * TMEM: one S^T accumulator pair (two K halves of 80 columns) instead of two; the
+//    softmax frees it as soon as it has loaded the scores (s_free), so the score MMAs
+//    of the next tile start while the softmax still computes;
+//  * P stored K-major, one 128-byte row of tokens per head (the value MMA's B operand
+//    at N = 80), written with 2-byte stores;
+//  * 20 softmax warps, five per TMEM lane quarter and 16 heads each (lanes 0-15 take
+//    eight heads of the quarter's 16 tokens, lanes 16-31 the other eight), so that a
+//    thread holds the state of 8 heads (768 threads, 80 registers each).
+namespace dtcw {
+using dtc::DC;
+using dtc::DRD;
+using dtc::NBOX;
+constexpr int NQ = kDtcHeadsWide;   // query heads of the CTA (N of both MMAs)
+constexpr int TT = kDtcTileWide;    // cache tokens per ring stage
+constexpr int STAGES = 2, PST = 2;
+constexpr int NSW = 20;             // softmax warps
+constexpr int NT = 32 * (4 + NSW);  // threads
+constexpr int HW = NQ / (NSW / 4);  // heads per softmax warp
+constexpr int HT = HW / 2;          // heads per softmax thread
+constexpr int QT_BYTES = dtc_image_bytes(NQ);
+constexpr int BOX = TT * 128;
+constexpr int TILE = NBOX * BOX;
+constexpr int PT = NQ * 128;        // P: one 128-byte row of tokens per head
+constexpr int OFF_TILES = QT_BYTES;
+constexpr int OFF_PT = OFF_TILES + STAGES * TILE;
+constexpr int OFF_SH = OFF_PT + PST * PT;
+constexpr uint32_t COL_ST = 0;       // S^T half hk at COL_ST + NQ hk
+constexpr uint32_t COL_OT = 2 * NQ;  // O^T M-tile mt at COL_OT + NQ mt
+constexpr int KSPLIT = NBOX * 2;
+static_assert(HW == 16 && HT == 8, "a warp's heads are one 16-column TMEM load of each K half");
+static_assert(COL_OT + 4 * NQ <= 512, "TMEM columns");
+static_assert(QT_BYTES % 1024 == 0 && BOX % 1024 == 0 && PT % 1024 == 0, "1024-byte swizzle atoms");
+static_assert(TT % 16 == 0 && TT <= 64 && TT <= 64, "tile rows: a multiple of the MMA K step, at most M = 64");
+
+struct Shared {
+  uint64_t full[STAGES], empty[STAGES];
+  uint64_t s_full, s_free, p_full[2], p_free[PST];
+  uint64_t q_full, q_free, seg_done, mma_done;
+  uint32_t tmem_slot;
+  int abort_flag;
+  int b0;
+  long long p0, start, end, W;
+  int R;
+  long long red[NT / 32];
+  float wmax[4][NQ];
+  float alpha_s[NQ];
+};
+constexpr int SMEM = OFF_SH + (int)sizeof(Shared);
+static_assert(SMEM <= 232448, "shared memory budget of one CTA");
+
+// barrier 1 over the softmax threads, OR-reducing a predicate; and a plain sync
+__device__ __forceinline__ bool bar_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "n"(32 * NSW)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * NSW) : "memory"); }
+}  // namespace dtcw
+
+__global__ void __launch_bounds__(dtcw::NT, 1)
+    decode_tc_wide_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
+                          const DecodeTcArgs a) {
+  using namespace sm100;
+  using namespace dtcw;
+  using dtc::Walker;
+  using dtc::seq_tiles;
+  using dtc::range_of;
+  using dtc::ex2f;
+  using dtc::kThr;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* qt = smem;                 // query image: 9 boxes of [80 heads x 128 B]
+  uint8_t* tiles = smem + OFF_TILES;  // stages: 9 boxes of [TT tokens x 128 B]
+  uint8_t* pt = smem + OFF_PT;        // P buffers: [80 heads x 128 B (tokens)]
+  Shared& sh = *reinterpret_cast<Shared*>(smem + OFF_SH);
+  volatile int& abort_flag = sh.abort_flag;
+
+  grid_dep_launch();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hg = blockIdx.x, r = blockIdx.y;
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) {
+      atomicCAS(a.status, 0, (int)GDLA_ERR_CUDA);
+      atomicCAS(a.status + 1, 0, 389);
+    }
+    return;
+  }
+  if (earlier_failure(a.status)) return;
+
+  // ---- this CTA's share of the W tiles (as in the narrow kernel)
+  {
+    long long loc = 0;
+    for (int b = tid; b < a.B; b += NT) {
+      const int raw = __ldg(a.seqlens + b);
+      if ((raw < 1 || raw > a.T_max) && r == 0 && hg == 0) atomicCAS(a.status, 0, (int)GDLA_ERR_INVALID_ARG);
+      loc += seq_tiles<TT>(a, b).n;
+    }
+    for (int o = 16; o; o >>= 1) loc += __shfl_xor_sync(0xffffffffu, loc, o);
+    if (lane == 0) sh.red[warp] = loc;
+    __syncthreads();
+    if (tid == 0) {
+      long long W = 0;
+      for (int w = 0; w < NT / 32; ++w) W += sh.red[w];
+      const long long R = min((long long)a.n_ranges, W);
+      sh.start = r < R ? (long long)r * W / R : 0;
+      sh.end = r < R ? (long long)(r + 1) * W / R : 0;
+      sh.R = (int)R;
+      sh.b0 = -1;
+      sh.W = W;
+    }
+    __syncthreads();
+    const long long start = sh.start;
+    if (start < sh.end) {
+      long long base = 0;
+      for (int c0 = 0; c0 < a.B; c0 += NT) {
+        const int b = c0 + tid;
+        const long long n = b < a.B ? seq_tiles<TT>(a, b).n : 0;
+        long long incl = n;
+        for (int o = 1; o < 32; o <<= 1) {
+          const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        if (lane == 31) sh.red[warp] = incl;
+        __syncthreads();
+        long long wbase = base;
+        for (int w = 0; w < warp; ++w) wbase += sh.red[w];
+        long long total = 0;
+        for (int w = 0; w < NT / 32; ++w) total += sh.red[w];
+        const long long p = wbase + incl - n;
+        if (b < a.B && n > 0 && p <= start && start < p + n) {
+          sh.b0 = b;
+          sh.p0 = p;
+        }
+        base += total;
+        __syncthreads();
+        if (sh.b0 >= 0) break;
+      }
+    }
+  }
+  const long long start = sh.start, end = sh.end, W = sh.W;
+  const int R = sh.R;
+  if (start >= end || sh.b0 < 0) return;
+  const int b0 = sh.b0;
+  const long long p0 = sh.p0;
+  const int n_tiles = (int)(end - start);
+  const int nh = min(a.hpc, a.H_q - hg * a.hpc);
+
+  if (tid == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(smem_u32(&sh.full[i]), 1);
+      mbar_init(smem_u32(&sh.empty[i]), 1);
+    }
+    mbar_init(smem_u32(&sh.s_full), 2);    // one commit per score warp
+    mbar_init(smem_u32(&sh.s_free), NSW);  // one arrival per softmax warp, once it has loaded S^T
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&sh.p_full[i]), NSW);
+    for (int i = 0; i < PST; ++i) mbar_init(smem_u32(&sh.p_free[i]), 1);
+    mbar_init(smem_u32(&sh.q_full), 1);
+    mbar_init(smem_u32(&sh.q_free), 2);
+    mbar_init(smem_u32(&sh.seg_done), 1);
+    mbar_init(smem_u32(&sh.mma_done), 3);
+    fence_mbar_init();
+    abort_flag = 0;
+    prefetch_tmap(&tmC);
+    prefetch_tmap(&tmR);
+  }
+  for (int e = tid; e < PST * PT / 16; e += NT) reinterpret_cast<uint4*>(pt)[e] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sh.tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      Walker<TT> wl, wp;
+      wl.init(a, b0, p0);
+      wp.init(a, b0, p0);
+      int k = 0;
+      for (; k < n_tiles && !abort_flag; ++k) {
+        const int st = k % STAGES;
+        {
+          // the tile into L2 as one contiguous request per cache, just ahead of its boxes
+          const long long t = start + k;
+          wp.seek(t);
+          const int j = (wp.st.jt0 + (int)(t - wp.pb)) * TT;
+          const int rows = min(TT, a.T_max - j);
+          const long long row0 = (long long)wp.b * a.T_max + j;
+          bulk_prefetch_l2(a.c_cache + row0 * DC, (uint32_t)rows * DC * 2);
+          bulk_prefetch_l2(a.kr_cache + row0 * DRD, (uint32_t)rows * DRD * 2);
+        }
+        if (k >= STAGES &&
+            !mbar_wait(smem_u32(&sh.empty[st]), ((k / STAGES) & 1) ^ 1, a.status, 361, &abort_flag)) {
+          abort_flag = 1;
+          break;
+        }
+        const long long t = start + k;
+        wl.seek(t);
+        const int tl = (int)(t - wl.pb);
+        if (tl == 0 && hg == 0) a.seqinfo[wl.b] = make_int2(r, range_of(wl.pb + wl.st.n - 1, W, R));
+        const int j0 = (wl.st.jt0 + tl) * TT;
+        const uint32_t bar = smem_u32(&sh.full[st]);
+        const uint32_t dst = smem_u32(tiles + st * TILE);
+        mbar_expect_tx(bar, TILE);
+        for (int bx = 0; bx < NBOX - 1; ++bx) tma_load_3d(dst + bx * BOX, &tmC, bar, bx * 64, j0, wl.b);
+        tma_load_3d(dst + (NBOX - 1) * BOX, &tmR, bar, 0, j0, wl.b);
+      }
+      if (abort_flag)
+        for (int q = (k > STAGES ? k - STAGES : 0); q < k; ++q)
+          mbar_wait(smem_u32(&sh.full[q % STAGES]), (q / STAGES) & 1, nullptr, 0);
+    }
+  } else if (warp >= 1 && warp <= 3) {
+    if (lane == 0) {
+      constexpr uint32_t id1 = idesc_bf16_f32(64, NQ, false, false);
+      constexpr uint32_t id2 = idesc_bf16_f32(128, NQ, true, false);
+      const uint64_t qd0 = sdesc_sw128(smem_u32(qt), 16, 1024);
+      Walker<TT> w;
+      w.init(a, b0, p0);
+      int seg = -1;
+      bool ok = true;
+      if (warp != 2) {
+        const int hk = warp == 1 ? 0 : 1;
+        const int kk0 = hk ? KSPLIT : 0, kk1 = hk ? NBOX * 4 : KSPLIT;
+        for (int k = 0; k < n_tiles && ok; ++k) {
+          const long long t = start + k;
+          w.seek(t);
+          const bool first = (k == 0) || t == w.pb, last = (k == n_tiles - 1) || t == w.pb + w.st.n - 1;
+          if (first) {
+            ++seg;
+            if (hk) {
+              if (seg == 0)
+                grid_dep_wait();
+              else
+                ok = mbar_wait(smem_u32(&sh.q_free), (seg - 1) & 1, a.status, 371, &abort_flag);
+              if (ok) {
+                const uint32_t bar = smem_u32(&sh.q_full);
+                mbar_expect_tx(bar, QT_BYTES);
+                bulk_load(smem_u32(qt), a.qimg + ((long long)w.b * a.n_hg + hg) * QT_BYTES, QT_BYTES, bar);
+              }
+            }
+            if (ok) ok = mbar_wait(smem_u32(&sh.q_full), seg & 1, a.status, 370, &abort_flag);
+          }
+          if (ok) ok = mbar_wait(smem_u32(&sh.full[k % STAGES]), (k / STAGES) & 1, a.status, 372, &abort_flag);
+          // the single S^T pair: the softmax has loaded tile k-1's scores
+          if (ok && k >= 1) ok = mbar_wait(smem_u32(&sh.s_free), (k - 1) & 1, a.status, 373, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t c0 = sdesc_sw128(smem_u32(tiles + (k % STAGES) * TILE), 16, 1024);
+          const uint32_t dcol = tmem + COL_ST + NQ * hk;
+#pragma unroll 6
+          for (int kk = kk0; kk < kk1; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            mma_ss(dcol, c0 + (((kk >> 2) * BOX + off) >> 4), qd0 + (((kk >> 2) * (NQ * 128) + off) >> 4), id1,
+                   kk > kk0);
+          }
+          mma_commit(smem_u32(&sh.s_full));
+          if (last) mma_commit(smem_u32(&sh.q_free));
+        }
+        if (!ok && hk) {
+          if (seg >= 0) mbar_wait(smem_u32(&sh.q_full), seg & 1, nullptr, 0);
+        }
+      } else {
+        for (int k = 0; k < n_tiles && ok; ++k) {
+          const long long t = start + k;
+          w.seek(t);
+          const bool first = (k == 0) || t == w.pb, last = (k == n_tiles - 1) || t == w.pb + w.st.n - 1;
+          ok = mbar_wait(smem_u32(&sh.p_full[k & 1]), (k >> 1) & 1, a.status, 374, &abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          // O^T += C^T . P^T for tile k: A MN-major (latent dims x tokens), B K-major P
+          const uint32_t tb = smem_u32(tiles + (k % STAGES) * TILE);
+          const uint64_t a0 = sdesc_sw128(tb, BOX, 1024);
+          const uint64_t b0d = sdesc_sw128(smem_u32(pt + (k % PST) * PT), 16, 1024);
+#pragma unroll
+          for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int kk = 0; kk < TT / 16; ++kk)
+              mma_ss(tmem + COL_OT + NQ * mt, a0 + ((2 * mt * BOX + kk * 2048) >> 4), b0d + ((kk * 32) >> 4), id2,
+                     (!first || kk > 0) ? 1u : 0u);
+          mma_commit(smem_u32(&sh.empty[k % STAGES]));
+          mma_commit(smem_u32(&sh.p_free[k % PST]));
+          if (last) mma_commit(smem_u32(&sh.seg_done));
+        }
+      }
+      if (!ok) abort_flag = 1;
+      mma_commit(smem_u32(&sh.mma_done));
+      mbar_wait(smem_u32(&sh.mma_done), 0, nullptr, 375);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- softmax
+    const int q4 = warp & 3, part = (warp - 4) >> 2;
+    const int hf = lane >> 4;
+    const int hp = part * HW;     // first head of the warp (a 16-column TMEM load)
+    const int hb = hp + hf * HT;  // first head of the thread
+    const int tok_local = q4 * 16 + (lane & 15);
+    const bool tok_real = tok_local < TT;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    Walker<TT> w;
+    w.init(a, b0, p0);
+    int seg = -1;
+    float m_ref[HT], lp[HT], thr[HT];
+    bool ok = true;
+    for (int k = 0; k < n_tiles; ++k) {
+      const long long t = start + k;
+      w.seek(t);
+      const bool first = (k == 0) || t == w.pb, last = (k == n_tiles - 1) || t == w.pb + w.st.n - 1;
+      if (first) {
+        ++seg;
+#pragma unroll
+        for (int h = 0; h < HT; ++h) {
+          m_ref[h] = -INFINITY;
+          lp[h] = 0.f;
+          thr[h] = (hb + h < nh) ? -INFINITY : INFINITY;
+        }
+      }
+      bool w_ok = mbar_wait(smem_u32(&sh.s_full), k & 1, a.status, 382, &abort_flag);
+      w_ok = __all_sync(0xffffffffu, w_ok);
+      float y[HT];
+      bool exceed = false;
+      if (w_ok) {
+        tc_fence_after();
+        uint32_t xr[HW], xr2[HW];
+        tmem_ld16(tmem + lane_base + COL_ST + hp, xr);
+        tmem_ld16(tmem + lane_base + COL_ST + NQ + hp, xr2);
+        tmem_wait_ld();
+        // the scores are in registers: the S^T pair may take the next tile's
+        tc_fence_before();
+        mbar_arrive_warp(smem_u32(&sh.s_free));
+        const int j = (w.st.jt0 + (int)(t - w.pb)) * TT + tok_local;
+        const bool valid = tok_real && j >= w.st.lo && j < w.st.Tb;
+#pragma unroll
+        for (int h = 0; h < HT; ++h) {
+          const float lo_h = __uint_as_float(xr[h]) + __uint_as_float(xr2[h]);
+          const float hi_h = __uint_as_float(xr[HT + h]) + __uint_as_float(xr2[HT + h]);
+          const float hi = __shfl_sync(0xffffffffu, hi_h, lane & 15);
+          y[h] = valid ? (hf ? hi : lo_h) : -INFINITY;
+        }
+#pragma unroll
+        for (int h = 0; h < HT; ++h) exceed |= y[h] > thr[h];
+      }
+      if (bar_or(exceed || !w_ok)) {
+        if (bar_or(!w_ok)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int h = 0; h < HT; ++h) {
+          float v = y[h];
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+          if ((lane & 15) == 0) sh.wmax[q4][hb + h] = v;
+        }
+        bar_sync();
+        bool resc = false;
+#pragma unroll
+        for (int h = 0; h < HT; ++h) {
+          const float tm = fmaxf(fmaxf(sh.wmax[0][hb + h], sh.wmax[1][hb + h]),
+                                 fmaxf(sh.wmax[2][hb + h], sh.wmax[3][hb + h]));
+          const bool up = tm > m_ref[h] + kThr || (m_ref[h] == -INFINITY && tm > -INFINITY);
+          const float mn = up ? fmaxf(m_ref[h], tm) : m_ref[h];
+          const float al = (!up || m_ref[h] == -INFINITY) ? (up ? 0.f : 1.f) : ex2f(m_ref[h] - mn);
+          resc |= up && m_ref[h] != -INFINITY;
+          lp[h] *= al;
+          m_ref[h] = mn;
+          if (hb + h < nh) thr[h] = mn + kThr;
+          if (q4 == 0 && (lane & 15) == 0) sh.alpha_s[hb + h] = al;
+        }
+        if (bar_or(resc)) {
+          bool r_ok = mbar_wait(smem_u32(&sh.p_free[(k - 1) % PST]), ((k - 1) / PST) & 1, a.status, 383,
+                                &abort_flag);
+          r_ok = __all_sync(0xffffffffu, r_ok);
+          if (bar_or(!r_ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // this warp's 16 heads of O^T, one M-tile at a time
+#pragma unroll 1
+          for (int mt = 0; mt < 4; ++mt) {
+            uint32_t o[HW];
+            const uint32_t ta = tmem + lane_base + COL_OT + NQ * mt + hp;
+            tmem_ld16(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < HW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * sh.alpha_s[hp + h]);
+            tmem_st16(ta, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (k >= PST) {
+        bool f_ok = mbar_wait(smem_u32(&sh.p_free[k % PST]), ((k / PST) & 1) ^ 1, a.status, 384, &abort_flag);
+        f_ok = __all_sync(0xffffffffu, f_ok);
+        if (bar_or(!f_ok)) {
+          ok = false;
+          break;
+        }
+      }
+      // P of this token for heads [hb, hb + 8): element (head, token) of the K-major operand,
+      // head rows of 128 bytes, 16-byte piece (token / 8) ^ (head & 7)
+      {
+        uint8_t* pbuf = pt + (k % PST) * PT + (tok_local & 7) * 2;
+#pragma unroll
+        for (int h = 0; h < HT; ++h) {
+          const float pv = ex2f(y[h] - (m_ref[h] == -INFINITY ? 0.f : m_ref[h]));
+          lp[h] += pv;
+          const int head = hb + h;
+          if (tok_real)
+            *reinterpret_cast<__nv_bfloat16*>(pbuf + head * 128 + (((tok_local >> 3) ^ (head & 7)) << 4)) =
+                __float2bfloat16_rn(pv);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive_warp(smem_u32(&sh.p_full[k & 1]));
+
+      if (last) {
+        bool d_ok = mbar_wait(smem_u32(&sh.seg_done), seg & 1, a.status, 385, &abort_flag);
+        if (bar_or(!__all_sync(0xffffffffu, d_ok))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < HT; ++h) {
+          float v = lp[h];
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          if ((lane & 15) == 0) sh.wmax[q4][hb + h] = v;
+        }
+        bar_sync();
+        const long long rec = ((long long)(r + w.b) * a.n_hg + hg) * NQ;
+        if (q4 == 0 && (lane & 15) == 0) {
+#pragma unroll
+          for (int h = 0; h < HT; ++h)
+            if (hb + h < nh) {
+              a.part_ml[(rec + hb + h) * 2 + 0] = m_ref[h];
+              a.part_ml[(rec + hb + h) * 2 + 1] =
+                  (sh.wmax[0][hb + h] + sh.wmax[1][hb + h]) + (sh.wmax[2][hb + h] + sh.wmax[3][hb + h]);
+            }
+        }
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+          uint32_t o[HW];
+          tmem_ld16(tmem + lane_base + COL_OT + NQ * mt + hp, o);
+          tmem_wait_ld();
+          const int dim = mt * 128 + q4 * 32 + lane;
+#pragma unroll
+          for (int h = 0; h < HW; ++h)
+            if (hp + h < nh) a.part_o[(rec + hp + h) * DC + dim] = __uint_as_float(o[h]);
+        }
+        tc_fence_before();
+        bar_sync();
+      }
+    }
+    if (!ok) abort_flag = 1;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+cudaError_t launch_decode_split_tc_wide(const DecodeParams& p, cudaStream_t s) {
+  using namespace dtcw;
+  CUtensorMap tc, tr;
+  {
+    const uint64_t dims[3] = {(uint64_t)DC, (uint64_t)p.T_max, (uint64_t)p.B};
+    const uint64_t str[2] = {(uint64_t)DC * 2, (uint64_t)p.T_max * DC * 2};
+    const uint32_t box[3] = {64, (uint32_t)TT, 1};
+    if (!make_tmap_bf16(&tc, p.c_cache, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)DRD, (uint64_t)p.T_max, (uint64_t)p.B};
+    const uint64_t str[2] = {(uint64_t)DRD * 2, (uint64_t)p.T_max * DRD * 2};
+    const uint32_t box[3] = {64, (uint32_t)TT, 1};
+    if (!make_tmap_bf16(&tr, p.kr_cache, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  DecodeTcArgs a{};
+  a.B = p.B; a.T_max = p.T_max; a.sliding = p.sliding; a.window = p.window;
+  a.H_q = p.n_kv * (p.g + 1); a.n_hg = p.n_hg; a.hpc = p.hpc; a.n_ranges = p.n_ranges;
+  a.seqlens = p.seqlens;
+  a.c_cache = reinterpret_cast<const __nv_bfloat16*>(p.c_cache);
+  a.kr_cache = reinterpret_cast<const __nv_bfloat16*>(p.kr_cache);
+  a.qimg = p.qimg; a.seqinfo = p.seqinfo; a.part_o = p.part_o; a.part_ml = p.part_ml; a.status = p.status;
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)p.n_hg, (unsigned)p.n_ranges);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tc_wide_kernel, tc, tr, a);
+}
+
 template <int TT, int STAGES, int PST, int PF>
 cudaError_t launch_decode_split_tc_cfg(const DecodeParams& p, cudaStream_t s) {
   using Lay = dtc::Layout<TT, STAGES, PST>;
@@ -1141,6 +1663,7 @@ cudaError_t launch_decode_split_tc_cfg(const DecodeParams& p, cudaStream_t s) {
 // MMA and softmax work does not shrink with the tile); an L2 prefetch one or two
 // tiles ahead 0.593 / 0.606 ms.
 cudaError_t launch_decode_split_tc(const DecodeParams& p, cudaStream_t s) {
+  if (p.img_heads == kDtcHeadsWide) return launch_decode_split_tc_wide(p, s);
   return launch_decode_split_tc_cfg<kDtcTile, 2, 2, 0>(p, s);
 }
 

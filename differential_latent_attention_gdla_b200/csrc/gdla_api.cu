@@ -179,7 +179,7 @@ bool decode_uses_tc(const gdla_decode_args* a) {
 
 struct DecodeLayout {
   size_t status, q_abs, q_rot, qimg, seqinfo, part_o, part_ml, total;
-  int tc, n_splits, split_len, n_ranges, n_hg, hpc, part_heads;
+  int tc, n_splits, split_len, n_ranges, n_hg, hpc, part_heads, img_heads;
 };
 
 DecodeLayout decode_layout(const gdla_decode_args* a) {
@@ -191,17 +191,21 @@ DecodeLayout decode_layout(const gdla_decode_args* a) {
   off += kStatusBytes;
   size_t records = 0;
   if (l.tc) {
-    // head groups of at most kDtcHeads heads; per head group, ranges of equal shares
-    // of all cache tiles, one CTA each: all CTAs together fill the SMs once, and a
-    // share is at least two tiles
-    l.n_hg = (H_q + kDtcHeads - 1) / kDtcHeads;
+    // 49 .. 80 heads: one head group on the wide split kernel (the cache is streamed once
+    // for all heads); otherwise head groups of at most kDtcHeads heads. Per head group,
+    // ranges of equal shares of all cache tiles, one CTA each: all CTAs together fill
+    // the SMs once, and a share is at least two tiles
+    const bool wide = H_q > kDtcHeads && H_q <= kDtcHeadsWide;
+    l.img_heads = wide ? kDtcHeadsWide : kDtcHeads;
+    const int tile = wide ? kDtcTileWide : kDtcTile;
+    l.n_hg = (H_q + l.img_heads - 1) / l.img_heads;
     l.hpc = (H_q + l.n_hg - 1) / l.n_hg;
-    l.part_heads = kDtcHeads;
-    const long tiles_max = (long)a->B * ((a->T_max + kDtcTile - 1) / kDtcTile);
+    l.part_heads = l.img_heads;
+    const long tiles_max = (long)a->B * ((a->T_max + tile - 1) / tile);
     l.n_ranges = (int)std::max(1L, std::min((long)std::max(1, kNumSMs / l.n_hg), tiles_max / 2));
     records = ((size_t)l.n_ranges + a->B) * l.n_hg;  // record (r + b) of every head group
     l.qimg = off;
-    off = align256(off + (size_t)a->B * l.n_hg * kDtcImageBytes);
+    off = align256(off + (size_t)a->B * l.n_hg * dtc_image_bytes(l.img_heads));
     l.seqinfo = off;
     off = align256(off + sizeof(int2) * (size_t)a->B);
   } else {
@@ -618,6 +622,7 @@ gdla_status gdla_decode(const gdla_decode_args* a, void* stream) {
   p.scale = default_scale(a->softmax_scale, a->d_nope, a->d_rope);
   p.tc = lay.tc; p.n_splits = lay.n_splits; p.split_len = lay.split_len;
   p.n_ranges = lay.n_ranges; p.n_hg = lay.n_hg; p.hpc = lay.hpc; p.part_heads = lay.part_heads;
+  p.img_heads = lay.img_heads;
   p.seqlens = a->seqlens;
   p.c_cache = a->c_cache; p.kr_cache = a->kr_cache; p.q = a->q; p.w_ukv = a->w_ukv;
   p.cos_tab = a->rope_cos; p.sin_tab = a->rope_sin; p.lam = a->lam_logits; p.gate = a->gate_logits;

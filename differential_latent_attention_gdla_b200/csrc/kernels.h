@@ -69,13 +69,20 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
 //    names the first and last range that cover sequence b;
 //  * CUDA-core path (other shapes and fp32): fixed splits of [0, T_max), the
 //    partial of (b, split s) in record b * n_splits + s; q_abs / q_rot in fp32.
-constexpr int kDtcHeads = 48;                     // query heads of one split CTA
-constexpr int kDtcTile = 64;                      // cache tokens per ring stage
-constexpr int kDtcImageBytes = kDtcHeads * 576 * 2;  // query image: 9 boxes of [48 heads x 128 B]
+//    A call with 49 .. 80 query heads (the report's g = 4) uses the wide split kernel
+//    instead: one head group of up to kDtcHeadsWide heads, kDtcTileWide-token tiles.
+constexpr int kDtcHeads = 48;                     // query heads of one (narrow) split CTA
+constexpr int kDtcTile = 64;                      // cache tokens per ring stage (narrow)
+constexpr int kDtcHeadsWide = 80;                 // query heads of one wide split CTA
+constexpr int kDtcTileWide = 48;                  // cache tokens per ring stage (wide)
+// query image of `heads` heads: 9 boxes of [heads x 128 B]
+__host__ __device__ constexpr int dtc_image_bytes(int heads) { return heads * 576 * 2; }
+constexpr int kDtcImageBytes = dtc_image_bytes(kDtcHeads);
 // byte offset of dimension d (of the 576-wide [latent | rotary] query) of local head lh
-// in a query image: 64-column boxes, rows of 128 bytes, 16-byte chunks swizzled by row
-__host__ __device__ inline int dtc_image_offset(int lh, int d) {
-  return (d >> 6) * (kDtcHeads * 128) + lh * 128 + ((((d & 63) >> 3) ^ (lh & 7)) << 4) + (d & 7) * 2;
+// in a query image of `heads` heads: 64-column boxes, rows of 128 bytes, 16-byte chunks
+// swizzled by row
+__host__ __device__ inline int dtc_image_offset(int lh, int d, int heads = kDtcHeads) {
+  return (d >> 6) * (heads * 128) + lh * 128 + ((((d & 63) >> 3) ^ (lh & 7)) << 4) + (d & 7) * 2;
 }
 
 struct DecodeParams {
@@ -86,13 +93,14 @@ struct DecodeParams {
   int n_splits, split_len;  // CUDA-core path
   int n_ranges, n_hg, hpc;  // tensor-core path: ranges per head group, head groups, heads per group
   int part_heads;           // heads per partial record
+  int img_heads;            // tensor-core path: heads per query image and split CTA (kDtcHeads or kDtcHeadsWide)
   const int* seqlens;
   const void* c_cache; const void* kr_cache; const void* q; const void* w_ukv;
   const float* cos_tab; const float* sin_tab;
   const float* lam; const void* gate; void* out;
   float* q_abs;     // CUDA-core path: [B, H_q, d_c] W_UK-absorbed content query
   float* q_rot;     // CUDA-core path: [B, H_q, d_rope] rotated rotary query
-  uint8_t* qimg;    // tensor-core path: [B * n_hg][kDtcImageBytes]
+  uint8_t* qimg;    // tensor-core path: [B * n_hg][dtc_image_bytes(img_heads)]
   int2* seqinfo;    // tensor-core path: [B]
   float* part_o;    // [records, part_heads, d_c]
   float* part_ml;   // [records, part_heads, 2]  (running max in log2 units, sum)

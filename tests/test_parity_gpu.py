@@ -184,7 +184,7 @@ def test_decode_full_size_every_sequence():
 
 def test_decode_80_heads_g4():
     """The report's head layout in decode: 16 KV heads with g = 4 (64 signal + 16
-    noise = 80 query heads), split over two head groups of the split kernel."""
+    noise = 80 query heads), all in one CTA of the wide split kernel."""
     for mask, window in (("causal", 0), ("sliding", 128)):
         shape = wl.DecodeShape("decode 80 heads", B=5, T=700, n_kv=16, g=4)
         inp = wl.make_decode_inputs(shape, seed=51, device=DEV, act="unit", seqlens=[700, 513, 129, 48, 1])
@@ -194,6 +194,37 @@ def test_decode_80_heads_g4():
         torch.cuda.synchronize()
         ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=mask, window=window)
         assert_parity(f64(y), ref, torch.bfloat16, f"decode 80 heads g=4 {mask}")
+
+
+@pytest.mark.parametrize("n_kv,g", [(16, 3), (12, 4), (10, 6)])
+def test_decode_wide_split_every_element(n_kv, g):
+    """49 .. 80 query heads take the wide split kernel (one head group of up to 80 heads,
+    48-token tiles, K-major P): 64, 60 and 70 heads leave 16, 20 and 10 of its 80 heads as
+    padding; lengths that end inside a tile and a one-token sequence; causal and a
+    100-token window."""
+    for mask, window in (("causal", 0), ("sliding", 100)):
+        shape = wl.DecodeShape(f"decode wide n_kv={n_kv} g={g}", B=4, T=500, n_kv=n_kv, g=g)
+        inp = wl.make_decode_inputs(shape, seed=60 + g, device=DEV, act="unit", seqlens=[500, 257, 49, 1])
+        cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+        y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                        inp["gate_logits"], inp["seqlens"], g=shape.g, mask=mask, window=window)
+        torch.cuda.synchronize()
+        ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=mask, window=window)
+        assert_parity(f64(y), ref, torch.bfloat16, f"{shape.name} {mask}")
+
+
+def test_decode_80_heads_g4_sequences_over_many_blocks():
+    """80 heads over 8 sequences of up to 3000 tokens: ~500 tiles of 48 tokens over 148
+    split CTAs, so every sequence is merged from the partials of several CTAs."""
+    shape = wl.DecodeShape("decode 80 heads, 8 x 3000", B=8, T=3000, n_kv=16, g=4)
+    inp = wl.make_decode_inputs(shape, seed=77, device=DEV, act="unit",
+                                seqlens=[3000, 2999, 2400, 1777, 1200, 600, 97, 48])
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    y = gdla.decode(inp["c_cache"], inp["kr_cache"], inp["q"], inp["w_ukv"], cos, sin, inp["lam_logits"],
+                    inp["gate_logits"], inp["seqlens"], g=shape.g)
+    torch.cuda.synchronize()
+    ref = oracle_decode(inp, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
+    assert_parity(f64(y), ref, torch.bfloat16, shape.name)
 
 
 def test_decode_many_sequences_per_split_block():
