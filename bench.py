@@ -55,7 +55,7 @@ CSRC = os.path.join(ROOT, "differential_latent_attention_gdla_b200", "csrc")
 # reports null.
 MEASURED_TRAFFIC = {
     ("attn_tc_kernel", "b1_l32k_g3"): (2.183e9, ("attn_tc.cu", "sm100.cuh"), "da06ebe13f571fd0"),
-    ("decode_tc_kernel", "b64_t32k"): (2.433e9, ("decode_tc.cu", "sm100.cuh"), "92c0a374a3055740"),
+    ("decode_tc_kernel", "b64_t32k"): (2.433e9, ("decode_tc.cu", "sm100.cuh"), "45965a23734dcc7d"),
 }
 
 

@@ -40,6 +40,8 @@
 // more than 2^8. Every wait is bounded and reports GDLA_ERR_TIMEOUT instead of
 // hanging. A sequence length outside [1, T_max] is clamped into it and reported
 // as GDLA_ERR_INVALID_ARG in the status word.
+// That is the narrow kernel (up to 48 heads per CTA, TT = 64); calls with 49 .. 80
+// heads use the wide kernel further down (80 heads per CTA, TT = 48, N = 80).
 #include <math.h>
 
 #include "kernels.h"

@@ -20,6 +20,8 @@
 //               output is stored from registers (16-byte pieces of each row).
 // Tails: rows of A beyond M and columns of B beyond N are zero-filled by TMA and
 // not stored; a K that is not a multiple of 64 is zero-filled the same way.
+// bf16 products with 256 rows or more run on gemm_pair_kernel instead (further down):
+// the same roles on clusters of two CTAs sharing M = 256 MMAs over 256 x 256 tiles.
 #include <type_traits>
 
 #include "kernels.h"
