@@ -385,15 +385,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tQ = tmem + lane_base + kColQ;
     // this row's RoPE factors for rotary dims 8c .. 8c+7, loaded ahead of each pass's
     // rotary chunk (volatile: live only between the load and that chunk, not across the
-    // key tiles)
+    // key tiles). Four 16-byte loads per thread (the tables are 16-byte aligned, a row is
+    // 128 bytes): one scalar load per factor made 16 warp requests of 32 rows each, a
+    // queue that held every pass boundary up by about 3 us.
     float cs[8], sn[8];
     auto load_rope = [&]() {
       const float* cp = a.cos_tab + (long)rope_pos * (DR / 2) + 8 * c;
       const float* sp = a.sin_tab + (long)rope_pos * (DR / 2) + 8 * c;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(cs[e]) : "l"(cp + e));
-        asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(sn[e]) : "l"(sp + e));
+      for (int h = 0; h < 2; ++h) {
+        asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(cs[4 * h]), "=f"(cs[4 * h + 1]), "=f"(cs[4 * h + 2]), "=f"(cs[4 * h + 3])
+                     : "l"(cp + 4 * h));
+        asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(sn[4 * h]), "=f"(sn[4 * h + 1]), "=f"(sn[4 * h + 2]), "=f"(sn[4 * h + 3])
+                     : "l"(sp + 4 * h));
       }
     };
     // chunk k of pass p's 128 Q rows into TMEM: thread c moves dims 16c .. 16c+15 of a
