@@ -108,6 +108,10 @@ struct AttnTcArgs {
   int* status;
 };
 
+// IO32: gate and output are 32-byte aligned, so the epilogue moves a thread's 16 values of
+// a row with one 32-byte access instead of two 16-byte ones (each warp access touches 32
+// rows; halving their number shortens the pass boundary)
+template <bool IO32>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
                    const __grid_constant__ CUtensorMap tmKR, const AttnTcArgs a) {
@@ -662,11 +666,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_wait_ld();
           if (row_ok) {
             uint4 gv[2], hv[2];
+            if constexpr (IO32) {
+              asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                           : "=r"(gv[0].x), "=r"(gv[0].y), "=r"(gv[0].z), "=r"(gv[0].w), "=r"(gv[1].x), "=r"(gv[1].y),
+                             "=r"(gv[1].z), "=r"(gv[1].w)
+                           : "l"(gp + ch * 16));
+            } else {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              gv[q] = reinterpret_cast<const uint4*>(gp + ch * 16)[q];
-              hv[q] = *reinterpret_cast<const uint4*>(hn_sm + hn_off(r, (cbase + 16 * ch) / 8 + q));
+              for (int q = 0; q < 2; ++q) gv[q] = reinterpret_cast<const uint4*>(gp + ch * 16)[q];
             }
+#pragma unroll
+            for (int q = 0; q < 2; ++q) hv[q] = *reinterpret_cast<const uint4*>(hn_sm + hn_off(r, (cbase + 16 * ch) / 8 + q));
             const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(hv);
             uint4 ov[2];
@@ -679,8 +689,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const float y1 = __uint_as_float(o[2 * e + 1]) * inv;
               ow[e] = pack_bf16x2(sigmoid_tanh(gf.x) * (y0 - lam * hf.x), sigmoid_tanh(gf.y) * (y1 - lam * hf.y));
             }
+            if constexpr (IO32) {
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(op + ch * 16), "r"(ov[0].x),
+                           "r"(ov[0].y), "r"(ov[0].z), "r"(ov[0].w), "r"(ov[1].x), "r"(ov[1].y), "r"(ov[1].z), "r"(ov[1].w)
+                           : "memory");
+            } else {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) reinterpret_cast<uint4*>(op + ch * 16)[q] = ov[q];
+              for (int q = 0; q < 2; ++q) reinterpret_cast<uint4*>(op + ch * 16)[q] = ov[q];
+            }
           }
         }
       }
@@ -750,7 +766,9 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   const long n_items = (long)a.n_qtiles * p.n_kv * p.B;
   if (n_items > INT_MAX) return cudaErrorInvalidValue;
   a.n_items = (int)n_items;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  const bool io32 = ((reinterpret_cast<uintptr_t>(p.gate) | reinterpret_cast<uintptr_t>(p.out)) & 31) == 0;
+  const auto kernel = io32 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM takes work items until none is left
   int dev = 0, sms = 0;
@@ -758,7 +776,7 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(p.work, 0, sizeof(int), s)) != cudaSuccess) return e;
   const int grid = (int)(n_items < sms ? n_items : sms);
-  attn_tc_kernel<<<(unsigned)grid, NTHREADS, SMEM_BYTES, s>>>(tq, tkv, tkr, a);
+  kernel<<<(unsigned)grid, NTHREADS, SMEM_BYTES, s>>>(tq, tkv, tkr, a);
   return cudaGetLastError();
 }
 

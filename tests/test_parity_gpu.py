@@ -81,6 +81,33 @@ def test_latent_expand_against_oracle_expansion(dtype):
         assert_parity(f64(krot[b]), kr, wl.torch_dtype(dtype), "k_rope_rot")
 
 
+def _at_byte_offset(t, offset):
+    """A contiguous copy of t whose data starts `offset` bytes past a 256-byte boundary."""
+    n, es = t.numel(), t.element_size()
+    buf = torch.empty(n + 256 // es, dtype=t.dtype, device=t.device)
+    v = buf[offset // es: offset // es + n].view(t.shape)
+    v.copy_(t)
+    assert v.data_ptr() % 256 == offset
+    return v
+
+
+def test_prefill_gate_and_output_only_16_byte_aligned():
+    # gate logits and output 16-byte but not 32-byte aligned: the epilogue's 16-byte
+    # access path, bit-identical to the 32-byte one and within tolerance of the oracle
+    shape = wl.PrefillShape("bf16 small causal g=3 ragged", B=2, L=300, n_kv=2, g=3)
+    inp = wl.make_prefill_inputs(shape, seed=5, device=DEV)
+    y32 = run_prefill(shape, inp)
+    inp16 = dict(inp, gate_logits=_at_byte_offset(inp["gate_logits"], 16))
+    out16 = _at_byte_offset(torch.zeros_like(y32), 48)
+    y16 = run_prefill(shape, inp16, out=out16)
+    torch.cuda.synchronize()
+    assert y16.data_ptr() == out16.data_ptr()
+    assert torch.equal(y16, y32)
+    ref = oracle_prefill_rows(inp, all_rows(shape), g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=shape.mask,
+                              window=shape.window)
+    assert_parity(f64(y16).reshape(ref.shape), ref, torch.bfloat16, "16-byte aligned gate/out")
+
+
 @pytest.mark.parametrize("name", ["b4_l4k_g2", "b1_l32k_g3", "b2_l64k_swa4k"])
 def test_prefill_full_size_sampled_rows(name):
     shape = wl.PREFILL[name]
