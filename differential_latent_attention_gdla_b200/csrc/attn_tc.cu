@@ -108,9 +108,10 @@ struct AttnTcArgs {
   int* status;
 };
 
-// IO32: gate and output are 32-byte aligned, so the epilogue moves a thread's 16 values of
-// a row with one 32-byte access instead of two 16-byte ones (each warp access touches 32
-// rows; halving their number shortens the pass boundary)
+// IO32: gate, output and the RoPE tables are 32-byte aligned, so a thread moves its 16
+// values of a gate or output row, or its 8 factors of a table row, with one 32-byte access
+// instead of two 16-byte ones (each warp access touches 32 rows; halving their number
+// shortens the pass boundary)
 template <bool IO32>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKV,
@@ -389,21 +390,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tQ = tmem + lane_base + kColQ;
     // this row's RoPE factors for rotary dims 8c .. 8c+7, loaded ahead of each pass's
     // rotary chunk (volatile: live only between the load and that chunk, not across the
-    // key tiles). Four 16-byte loads per thread (the tables are 16-byte aligned, a row is
-    // 128 bytes): one scalar load per factor made 16 warp requests of 32 rows each, a
-    // queue that held every pass boundary up by about 3 us.
+    // key tiles). Two 32-byte loads per thread, or four 16-byte ones when the tables are
+    // only 16-byte aligned (a row is 128 bytes): one scalar load per factor made 16 warp
+    // requests of 32 rows each, a queue that held every pass boundary up by about 3 us.
     float cs[8], sn[8];
     auto load_rope = [&]() {
       const float* cp = a.cos_tab + (long)rope_pos * (DR / 2) + 8 * c;
       const float* sp = a.sin_tab + (long)rope_pos * (DR / 2) + 8 * c;
+      if constexpr (IO32) {
+        asm volatile("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=f"(cs[0]), "=f"(cs[1]), "=f"(cs[2]), "=f"(cs[3]), "=f"(cs[4]), "=f"(cs[5]), "=f"(cs[6]),
+                       "=f"(cs[7])
+                     : "l"(cp));
+        asm volatile("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=f"(sn[0]), "=f"(sn[1]), "=f"(sn[2]), "=f"(sn[3]), "=f"(sn[4]), "=f"(sn[5]), "=f"(sn[6]),
+                       "=f"(sn[7])
+                     : "l"(sp));
+      } else {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(cs[4 * h]), "=f"(cs[4 * h + 1]), "=f"(cs[4 * h + 2]), "=f"(cs[4 * h + 3])
-                     : "l"(cp + 4 * h));
-        asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(sn[4 * h]), "=f"(sn[4 * h + 1]), "=f"(sn[4 * h + 2]), "=f"(sn[4 * h + 3])
-                     : "l"(sp + 4 * h));
+        for (int h = 0; h < 2; ++h) {
+          asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(cs[4 * h]), "=f"(cs[4 * h + 1]), "=f"(cs[4 * h + 2]), "=f"(cs[4 * h + 3])
+                       : "l"(cp + 4 * h));
+          asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(sn[4 * h]), "=f"(sn[4 * h + 1]), "=f"(sn[4 * h + 2]), "=f"(sn[4 * h + 3])
+                       : "l"(sp + 4 * h));
+        }
       }
     };
     // chunk k of pass p's 128 Q rows into TMEM: thread c moves dims 16c .. 16c+15 of a
@@ -766,7 +778,8 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   const long n_items = (long)a.n_qtiles * p.n_kv * p.B;
   if (n_items > INT_MAX) return cudaErrorInvalidValue;
   a.n_items = (int)n_items;
-  const bool io32 = ((reinterpret_cast<uintptr_t>(p.gate) | reinterpret_cast<uintptr_t>(p.out)) & 31) == 0;
+  const bool io32 = ((reinterpret_cast<uintptr_t>(p.gate) | reinterpret_cast<uintptr_t>(p.out) |
+                      reinterpret_cast<uintptr_t>(p.cos_tab) | reinterpret_cast<uintptr_t>(p.sin_tab)) & 31) == 0;
   const auto kernel = io32 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;

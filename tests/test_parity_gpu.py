@@ -91,9 +91,9 @@ def _at_byte_offset(t, offset):
     return v
 
 
-def test_prefill_gate_and_output_only_16_byte_aligned():
-    # gate logits and output 16-byte but not 32-byte aligned: the epilogue's 16-byte
-    # access path, bit-identical to the 32-byte one and within tolerance of the oracle
+def test_prefill_gate_output_and_rope_tables_only_16_byte_aligned():
+    # gate logits and output (then the RoPE tables) 16-byte but not 32-byte aligned: the
+    # 16-byte access path, bit-identical to the 32-byte one and within tolerance of the oracle
     shape = wl.PrefillShape("bf16 small causal g=3 ragged", B=2, L=300, n_kv=2, g=3)
     inp = wl.make_prefill_inputs(shape, seed=5, device=DEV)
     y32 = run_prefill(shape, inp)
@@ -106,6 +106,13 @@ def test_prefill_gate_and_output_only_16_byte_aligned():
     ref = oracle_prefill_rows(inp, all_rows(shape), g=shape.g, d_nope=shape.d_n, d_v=shape.d_v, mask=shape.mask,
                               window=shape.window)
     assert_parity(f64(y16).reshape(ref.shape), ref, torch.bfloat16, "16-byte aligned gate/out")
+    # the RoPE tables only 16-byte aligned (gate and output 32-byte aligned)
+    cos, sin = gdla.rope_tables(shape.L, shape.d_R, device=DEV)
+    cos16, sin16 = _at_byte_offset(cos, 16), _at_byte_offset(sin, 80)
+    y_t = gdla.prefill(inp["c_kv"], inp["gamma"], inp["k_rope"], inp["q"], inp["w_ukv"], cos16, sin16,
+                       inp["lam_logits"], inp["gate_logits"], g=shape.g, mask=shape.mask, window=shape.window)
+    torch.cuda.synchronize()
+    assert torch.equal(y_t, y32)
 
 
 @pytest.mark.parametrize("name", ["b4_l4k_g2", "b1_l32k_g3", "b2_l64k_swa4k"])
