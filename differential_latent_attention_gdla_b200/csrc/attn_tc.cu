@@ -12,7 +12,8 @@
 // Both Q (rotated once per pass) and P live in TMEM, so the tensor core reads only
 // K and V from shared memory.
 // The kernel is persistent: one CTA per SM takes work items from a global counter
-// (KV-group-major, heaviest query blocks first) until none is left, so the set-up of a
+// (blocks of (sequence, KV group) pairs whose keys fit in a share of L2; heaviest query
+// blocks of the whole block first) until none is left, so the set-up of a
 // CTA happens once and the next item's Q, K and V copies overlap the current item's
 // last tiles and epilogue; items reach the other roles through a 2-slot ring in shared
 // memory that the producer fills.
@@ -38,6 +39,8 @@
 // 2^8.
 #include <limits.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -96,7 +99,8 @@ __device__ __forceinline__ uint32_t hn_off(int r, int c) { return (uint32_t)(r *
 
 struct AttnTcArgs {
   int B, L, n_kv, g, sliding, window, rope_max_pos, n_qtiles;
-  int n_items;  // (sequence, KV group, 64-row query block) work items
+  int n_items;  // (sequence, KV group, 128-row query block) work items
+  int grp_block;  // (sequence, KV group) pairs per block of the work order
   int* work;    // the next work item (zero before the launch)
   int q_len, q_start;  // query rows: positions q_start .. q_start+q_len-1; keys: 0 .. L-1
   float sl2;  // tau * log2(e)
@@ -146,11 +150,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   struct Item {
     int b, h, m_loc, m0, j_lo, n_tiles;
   };
+  // Work order: the (sequence, KV group) pairs in blocks of a.grp_block; inside a block the
+  // query blocks with the most keys come first, taken across all of its pairs, so that the
+  // long items of the block start early and the short ones fill the end (a block's K/V
+  // stays small enough to be reused from L2 by the CTAs working on it).
   auto item_of = [&](int t) {
     Item it;
-    const int m_idx = a.n_qtiles - 1 - t % a.n_qtiles;
-    it.h = (t / a.n_qtiles) % a.n_kv;
-    it.b = t / (a.n_qtiles * a.n_kv);
+    const int n_grp = a.B * a.n_kv;
+    const int g0 = t / (a.grp_block * a.n_qtiles) * a.grp_block;  // first pair of t's block
+    const int gsz = min(a.grp_block, n_grp - g0);                  // pairs in that block
+    const int w = t - g0 * a.n_qtiles;                             // position inside the block
+    const int grp = g0 + w % gsz;
+    const int m_idx = a.n_qtiles - 1 - w / gsz;
+    it.h = grp % a.n_kv;
+    it.b = grp / a.n_kv;
     it.m_loc = m_idx * IM;       // first query row of the block within the q/Y tensors
     it.m0 = a.q_start + it.m_loc;  // its position in the sequence
     const int last_row = min(q_end - 1, it.m0 + IM - 1);
@@ -778,6 +791,14 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
   const long n_items = (long)a.n_qtiles * p.n_kv * p.B;
   if (n_items > INT_MAX) return cudaErrorInvalidValue;
   a.n_items = (int)n_items;
+  // pairs per block of the work order: as many as keep the keys that a block's items can
+  // read (the window plus one query block, or the whole sequence) within 32 MiB of L2
+  {
+    const long keys = p.sliding ? std::min<long>(p.L, (long)p.window + IM) : (long)p.L;
+    const long bytes = keys * (DN + DV) * 2;
+    const long n_grp = (long)p.B * p.n_kv;
+    a.grp_block = (int)std::max<long>(1, std::min<long>(n_grp, (32l << 20) / std::max<long>(bytes, 1)));
+  }
   const bool io32 = ((reinterpret_cast<uintptr_t>(p.gate) | reinterpret_cast<uintptr_t>(p.out) |
                       reinterpret_cast<uintptr_t>(p.cos_tab) | reinterpret_cast<uintptr_t>(p.sin_tab)) & 31) == 0;
   const auto kernel = io32 ? attn_tc_kernel<true> : attn_tc_kernel<false>;
