@@ -16,7 +16,9 @@
 // blocks of the whole block first) until none is left, so the set-up of a
 // CTA happens once and the next item's Q, K and V copies overlap the current item's
 // last tiles and epilogue; items reach the other roles through a 2-slot ring in shared
-// memory that the producer fills.
+// memory that the producer fills. At every pass boundary the next pass's Q goes into
+// TMEM before the epilogue (its content chunks while the last PV runs), so the next
+// pass's first S MMAs overlap the epilogue.
 // Warp roles (640 threads):
 //   warp 0      work items; TMA producer: the pass's Q in three 64-dim chunks through a
 //               2-deep staging ring; K tiles (128 keys x 192) and V tiles
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         it = item_of(t);
         for (int p = 0; p < n_pairs && ok && !abort_flag; ++p) {
           // the last Q chunk reuses the staging buffer of the first, which the softmax
-          // warps free only after the previous pass's epilogue: K(0), K(1) go first
+          // warps free only after the previous pass's last tile: K(0), K(1) go first
           ok = load_q(p, 0) && load_q(p, 1);
           // consumption order of the tensor core: S(0), S(1), PV(0), S(2), PV(1), ...
           if (ok) ok = load_k(0) && (it.n_tiles < 2 || load_k(1));
@@ -363,7 +365,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!ok || t < 0) break;
         const int n_tiles = item_of(t).n_tiles;
         for (int p = 0; p < n_pairs && ok; ++p, ++gp) {
-          // the softmax warps write the rotated Q into TMEM after the previous pass's epilogue
+          // the softmax warps write the rotated Q into TMEM after the previous pass's last
+          // PV, before its epilogue (which then overlaps this pass's first S MMAs)
           ok = mbar_wait(smem_u32(&bars.q_ready), gp & 1, a.status, 211, &abort_flag);
           if (!ok) break;
           tc_fence_after();
@@ -407,9 +410,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // only 16-byte aligned (a row is 128 bytes): one scalar load per factor made 16 warp
     // requests of 32 rows each, a queue that held every pass boundary up by about 3 us.
     float cs[8], sn[8];
-    auto load_rope = [&]() {
-      const float* cp = a.cos_tab + (long)rope_pos * (DR / 2) + 8 * c;
-      const float* sp = a.sin_tab + (long)rope_pos * (DR / 2) + 8 * c;
+    auto load_rope = [&](int pos) {
+      const float* cp = a.cos_tab + (long)pos * (DR / 2) + 8 * c;
+      const float* sp = a.sin_tab + (long)pos * (DR / 2) + 8 * c;
       if constexpr (IO32) {
         asm volatile("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                      : "=f"(cs[0]), "=f"(cs[1]), "=f"(cs[2]), "=f"(cs[3]), "=f"(cs[4]), "=f"(cs[5]), "=f"(cs[6]),
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!failed && t >= 0) {
         it = item_of(t);
         set_rows();
-        load_rope();
+        load_rope(rope_pos);
         for (int k = 0; k < 3; ++k) ok = move_q(0, k) && ok;
         failed = bar_or512(!ok);
         if (!failed) q_done();
@@ -617,15 +620,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (failed) break;
 
-      // ---------------------------------------------------------- epilogue
-      {
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.o_full), gp & 1, a.status, 223, &abort_flag));
-        if (bar_or512(!ok)) {
-          failed = true;
-          break;
-        }
-      }
-      tc_fence_after();
       // the next pass: the item's next head, or the next item's first
       int t_next = t, p_next = p + 1;
       if (p_next == n_pairs) {
@@ -639,8 +633,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       const bool next = t_next >= 0;
       if (next) {
-        // every S MMA of this pass is done, so the next pass's Q content chunks may go into
-        // TMEM now; its rotary chunk follows the epilogue, while that copy lands
+        // every S MMA of this pass is done (the last tile's S was read), so the next
+        // pass's Q content chunks may go into TMEM while the last PV runs; that also frees
+        // the staging buffer of its rotary chunk
         bool ok = move_q(gp + 1, 0);
         ok = move_q(gp + 1, 1) && ok;
         if (bar_or512(!ok)) {
@@ -648,6 +643,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           break;
         }
       }
+
+      // ---------------------------------------------------------- epilogue
+      {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&bars.o_full), gp & 1, a.status, 223, &abort_flag));
+        if (bar_or512(!ok)) {
+          failed = true;
+          break;
+        }
+      }
+      tc_fence_after();
       // row sum: add the other quarters' partial sums (same running maximum everywhere).
       // Every thread has passed the barrier-reduction after o_full since it last read
       // the buffer (a tile's maximum exchange).
@@ -658,6 +663,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         l_part = (xs[r] + xs[ROWS + r]) + (xs[2 * ROWS + r] + xs[3 * ROWS + r]);
       }
       const float inv = l_part > 0.f ? 1.f / l_part : 0.f;
+      if (next) {
+        // the next pass's rotary Q chunk (RoPE at the positions of the next item's rows when
+        // the item changes), then its S MMAs run while this pass's epilogue does: they
+        // write only S buffers, and PV(0) of that pass, which overwrites O, waits for a P
+        // that these threads store after the epilogue has read O
+        int pos = rope_pos;
+        if (p_next == 0) {
+          const int i_next = item_of(t_next).m0 + r;
+          pos = i_next < q_end ? i_next : q_end - 1;
+        }
+        load_rope(pos);
+        tc_fence_before();
+        if (bar_or512(!move_q(gp + 1, 2))) {
+          failed = true;
+          break;
+        }
+        q_done();
+      }
 
       if (hl == 0) {
         // noise head: park the normalised H_N (bf16) for every signal head
@@ -725,20 +748,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      if (next) {
-        // O of this pass is read: the next pass's rotary Q chunk (at the positions of the
-        // next item's rows when the item changes), then its S MMAs may start
-        if (p_next == 0) {
-          it = item_of(t_next);
-          set_rows();
-        }
-        load_rope();
-        tc_fence_before();
-        if (bar_or512(!move_q(gp + 1, 2))) {
-          failed = true;
-          break;
-        }
-        q_done();
+      if (next && p_next == 0) {
+        it = item_of(t_next);
+        set_rows();
       }
       t = t_next;
       p = p_next;
