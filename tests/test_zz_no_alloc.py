@@ -14,7 +14,7 @@ import torch
 import differential_latent_attention_gdla_b200 as gdla
 from differential_latent_attention_gdla_b200 import _abi
 from differential_latent_attention_gdla_b200 import workloads as wl
-from gdla_testutil import assert_parity, f64
+from gdla_testutil import assert_parity, f64, oracle_decode
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -44,6 +44,41 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls(case):
         # the same kernels on the same inputs: identical bytes (decode is bit-reproducible)
         assert torch.equal(y, ref), f"noalloc call {call}: max diff {(y.float() - ref.float()).abs().max()}"
         assert_parity(f64(y), f64(ref), torch.bfloat16, f"noalloc call {call}")
+
+
+def test_noalloc_decode_replays_from_a_cuda_graph():
+    # the serving-loop use: one eager call (the scratch address is looked up and the
+    # kernels' attributes set), then the call captured in a CUDA graph and replayed
+    # twice, with new query values copied into the captured input between replays
+    shape = wl.DecodeShape("noalloc graph B=8 T=2048 g=2", B=8, T=2048, g=2)
+    inp = wl.make_decode_inputs(shape, seed=23, device=DEV, act="unit", seqlens=[2048, 1500, 1, 129, 700, 2048, 64, 1024])
+    cos, sin = gdla.rope_tables(shape.T, shape.d_R, device=DEV)
+    q_in = inp["q"].clone()
+    q_next = wl.make_decode_inputs(shape, seed=24, device=DEV, act="unit")["q"]
+
+    def args(q):
+        return (inp["c_cache"], inp["kr_cache"], q, inp["w_ukv"], cos, sin, inp["lam_logits"], inp["gate_logits"],
+                inp["seqlens"])
+
+    ref1 = gdla.decode(*args(inp["q"]), g=shape.g)
+    ref2 = gdla.decode(*args(q_next), g=shape.g)
+    y = torch.empty_like(ref1)
+    gdla.decode_noalloc(*args(q_in), g=shape.g, out=y)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        gdla.decode_noalloc(*args(q_in), g=shape.g, out=y)
+    for q_new, ref in ((inp["q"], ref1), (q_next, ref2)):
+        q_in.copy_(q_new)
+        y.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref)
+    # the second replay against the oracle
+    inp2 = dict(inp, q=q_next)
+    ref_o = oracle_decode(inp2, g=shape.g, d_nope=shape.d_n, d_v=shape.d_v)
+    assert_parity(f64(y), ref_o, torch.bfloat16, "noalloc graph replay")
+    del graph
 
 
 def test_noalloc_rejects_a_batch_beyond_its_scratch():
