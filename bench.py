@@ -454,8 +454,11 @@ def run_ours(a):
                           ("prefill_g4_swa128", "b1_l32k_g4_swa128")):
             S = wl.PREFILL[name]
             _, _, ex, at, st = prefill_case(S, rank_seed(a.seed, rank, "prefill"))
-            t_e = time_loop(ex, 3, 2, stream)
-            t_a = time_loop(at, 3, 2, stream)
+            # the short workloads (about 1 ms a call) get more calls, so that a clock
+            # excursion of a few ms does not decide their number
+            n_t, n_w = (3, 2) if S.B * S.L >= 131072 else (20, 5)
+            t_e = time_loop(ex, n_t, n_w, stream)
+            t_a = time_loop(at, n_t, n_w, stream)
             if int(gdla.workspace_status(st)) != 0:
                 raise RuntimeError(f"device status word reports a failed wait ({name})")
             extra_ms[key] = (name, S, t_e, t_a)
