@@ -15,7 +15,10 @@
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller, dense
- *    row-major in the layout stated beside them, 16-byte aligned. The library
+ *    row-major in the layout stated beside them, 16-byte aligned. (The bf16
+ *    attention uses 32-byte accesses when gate_logits, out and both RoPE
+ *    tables are 32-byte aligned, which allocators normally give; with only
+ *    16-byte alignment it returns the same bytes a little more slowly.) The library
  *    allocates no memory and keeps no per-call state; scratch comes from the
  *    caller's workspace, sized by the matching *_workspace_size function.
  *    Three entry points state their exceptions beside them: gdla_prefill_host
